@@ -1,0 +1,18 @@
+"""CPU float64 oracle for exact softmax attention (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+leg of ``bench.py`` may import this package.  The CUDA library never imports,
+links or calls it, and it never imports the CUDA library.
+"""
+
+from .attention_ref import (  # noqa: F401
+    BLOCK,
+    attention_backward,
+    attention_forward,
+    dropout_keep,
+    dropout_threshold,
+    head_backward,
+    safe_softmax,
+    valid_mask,
+)
+from .philox_ref import philox4x32_10, philox_block, weyl_constants  # noqa: F401

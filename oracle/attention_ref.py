@@ -1,0 +1,224 @@
+"""Standard (materialising) softmax attention in float64: the oracle.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference leg of ``bench.py`` may import this module.  It shares
+no code with the CUDA path and never receives a value computed by it.
+
+What it computes, and where that is defined
+-------------------------------------------
+The method (FlashAttention) is *exact*: it returns the same result as standard
+attention and differs only in how it moves data (researchpapers.dev
+"FlashAttention 详解:IO 感知精确注意力,提速 2-4 倍", sections "快速答案" and the
+FAQ entry asking whether it is exact or approximate).  So this oracle is the
+textbook definition written out, one (batch, head) at a time, materialising the
+full score matrix exactly as the "standard attention" the pages describe
+(suanlizi.com FlashAttention summary, sections "核心操作融合" and "分块计算"):
+
+    S = scale * Q K^T                   score matrix, N x N
+    P = softmax over the valid keys     row-wise, safe form (subtract the row max)
+    O = dropout(P) V
+
+and the backward is the plain chain rule through those three steps.  The safe
+softmax (subtracting the row maximum before exp) is the form the pages require
+to avoid overflow at scores like +20000 and a vanishing denominator at -20000
+(llm-deploy "tensorrt-llm/flash-attention.md", safe-softmax section on
+上溢出 / 下溢出).  The saved statistic is the per-row log-sum-exp
+LSE = m + ln(l), the (m, l) pair of the online softmax collapsed to one number
+(same page, closing "解决方案" paragraph, whose symbol list is garbled; the
+running max m and row sum l are the readings used here).
+
+Readings taken where the pages are silent (all are repeated in the design doc):
+  * scale is a caller-given float applied to Q K^T before masking and the max;
+  * causal: query i may attend key j iff j <= i (0-based, N_q = N_k = N);
+  * key padding: per-batch length L_b, keys j >= L_b are invalid; query rows
+    are not masked (they still attend the valid keys);
+  * block mask: uint8 [ceil(N/128)]^2 shared by all (b, h); entry 0 removes the
+    whole 128 x 128 block of (query, key) pairs;
+  * all masks combine by logical AND;
+  * a row with no valid key has P = 0, O = 0 and LSE = -inf;
+  * dropout is inverted dropout on the normalised P: P_drop = P * Z / (1 - p),
+    Z the keep bit; LSE is that of the undropped softmax;
+  * keep bit Z(b,h,i,j): Philox4x32-10 with key (seed mod 2^32, seed >> 32),
+    counter (j >> 2, i, h, b), output word (j & 3); keep iff word >= t with
+    t = min(floor(p * 2^32), 2^32 - 1), p the float32 value the library receives.
+
+Parity pins for every function here live in ``tests/test_oracle_pins.py``.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from .philox_ref import philox4x32_10
+
+BLOCK = 128  # block-mask granularity (128 x 128 blocks of (query, key) pairs)
+
+
+# ----------------------------------------------------------------------------
+# masks and dropout bits
+# ----------------------------------------------------------------------------
+
+def valid_mask(n, rows, causal=False, kv_len=None, block_mask=None):
+    """Boolean [len(rows), n]: which (query i, key j) pairs take part.
+
+    rows: query indices (int array).  kv_len: valid key count for this batch
+    entry (None = n).  block_mask: uint8 [nb, nb] or None.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    i = rows[:, None]
+    j = np.arange(n, dtype=np.int64)[None, :]
+    ok = np.ones((rows.size, n), dtype=bool)
+    if kv_len is not None:
+        ok &= j < int(kv_len)
+    if causal:
+        ok &= j <= i
+    if block_mask is not None:
+        bm = np.asarray(block_mask).astype(bool)
+        ok &= bm[i // BLOCK, j // BLOCK]
+    return ok
+
+
+def dropout_threshold(p):
+    """Integer threshold t for keep-iff-word >= t, from the float32 value of p."""
+    p32 = float(np.float32(p))
+    if not (0.0 <= p32 < 1.0):
+        raise ValueError("dropout probability must lie in [0, 1)")
+    return min(int(math.floor(p32 * 4294967296.0)), 4294967295)
+
+
+def dropout_keep(seed, p, b, h, rows, n):
+    """Keep bits Z[i, j] (bool) for query rows ``rows`` and keys 0..n-1."""
+    t = dropout_threshold(p)
+    if t == 0:
+        return np.ones((len(rows), n), dtype=bool)
+    seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+    k0, k1 = seed & 0xFFFFFFFF, seed >> 32
+    rows = np.asarray(rows, dtype=np.uint64)[:, None]
+    groups = np.arange((n + 3) // 4, dtype=np.uint64)[None, :]
+    words = philox4x32_10(groups, rows, np.uint64(h), np.uint64(b), k0, k1)
+    # words[w][r, g] is the word for key 4 g + w
+    w = np.stack(words, axis=-1).reshape(len(rows), -1)[:, :n]
+    return w >= np.uint32(t)
+
+
+# ----------------------------------------------------------------------------
+# the softmax step
+# ----------------------------------------------------------------------------
+
+def safe_softmax(s, valid):
+    """Row-wise softmax over the valid entries of s, max-subtracted.
+
+    Returns (P, lse, m, l).  Rows without a valid entry: P = 0, lse = -inf.
+    """
+    s = np.asarray(s, dtype=np.float64)
+    masked = np.where(valid, s, -np.inf)
+    m = masked.max(axis=1)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    e = np.where(valid, np.exp(masked - m_safe[:, None]), 0.0)
+    l = e.sum(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        p = np.where(l[:, None] > 0, e / np.where(l > 0, l, 1.0)[:, None], 0.0)
+        lse = np.where(l > 0, m_safe + np.log(np.where(l > 0, l, 1.0)), -np.inf)
+    return p, lse, m, l
+
+
+# ----------------------------------------------------------------------------
+# forward
+# ----------------------------------------------------------------------------
+
+def _head_forward(q, k, v, scale, rows, causal, kv_len, block_mask, keep, rscale):
+    s = scale * (q[rows] @ k.T)
+    valid = valid_mask(k.shape[0], rows, causal, kv_len, block_mask)
+    p, lse, _, _ = safe_softmax(s, valid)
+    pd = p if keep is None else p * keep * rscale
+    return pd @ v, lse
+
+
+def attention_forward(q, k, v, scale, causal=False, seqlens=None, dropout_p=0.0,
+                      seed=0, block_mask=None, heads=None, rows=None, slab=256):
+    """O and LSE of standard attention.
+
+    q, k, v: float64 [B, H, N, d].  Returns (O [B,H,R,d], LSE [B,H,R]) where R
+    indexes ``rows`` (default all N rows).  ``heads`` optionally restricts the
+    computation to a list of (b, h) pairs (other entries are left NaN).  Rows
+    are processed in slabs of ``slab`` rows only to bound memory: every row is
+    computed independently, so the slab size does not change any value.
+    """
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    B, H, N, d = q.shape
+    rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.full((B, H, rows.size, d), np.nan)
+    lse = np.full((B, H, rows.size), np.nan)
+    pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    p32 = float(np.float32(dropout_p))
+    rscale = 1.0 / (1.0 - p32) if p32 > 0 else 1.0
+    for b, h in pairs:
+        kv_len = None if seqlens is None else int(seqlens[b])
+        for r0 in range(0, rows.size, slab):
+            rr = rows[r0:r0 + slab]
+            keep = None
+            if p32 > 0:
+                keep = dropout_keep(seed, p32, b, h, rr, N)
+            o, l = _head_forward(q[b, h], k[b, h], v[b, h], scale, rr, causal,
+                                 kv_len, block_mask, keep, rscale)
+            out[b, h, r0:r0 + rr.size] = o
+            lse[b, h, r0:r0 + rr.size] = l
+    return out, lse
+
+
+# ----------------------------------------------------------------------------
+# backward
+# ----------------------------------------------------------------------------
+
+def head_backward(q, k, v, dout, scale, causal=False, kv_len=None, block_mask=None,
+                  keep=None, dropout_p=0.0):
+    """dQ, dK, dV of one (b, h) by the chain rule through S, P, dropout, PV.
+
+    The recomputation of the pages (rebuild P in the backward from saved
+    statistics, suanlizi.com summary "重计算" and researchpapers.dev
+    "分块与重计算") gives the same numbers as keeping P, which is what a
+    standard implementation does; the oracle simply recomputes S and P here.
+    """
+    n = k.shape[0]
+    rows = np.arange(q.shape[0])
+    s = scale * (q @ k.T)
+    valid = valid_mask(n, rows, causal, kv_len, block_mask)
+    p, _, _, _ = safe_softmax(s, valid)
+    p32 = float(np.float32(dropout_p))
+    if keep is None or p32 == 0:
+        z = np.ones_like(p)
+        rscale = 1.0
+    else:
+        z = keep.astype(np.float64)
+        rscale = 1.0 / (1.0 - p32)
+    pd = p * z * rscale                 # dropped, rescaled P that multiplies V
+    dv = pd.T @ dout                    # O = Pd V  ->  dV = Pd^T dO
+    dpd = dout @ v.T                    # gradient w.r.t. Pd
+    dp = dpd * z * rscale               # gradient w.r.t. P through the dropout
+    dsum = (p * dp).sum(axis=1)         # softmax Jacobian term: sum_j P_ij dP_ij
+    ds = p * (dp - dsum[:, None])       # gradient w.r.t. S
+    dq = scale * (ds @ k)
+    dk = scale * (ds.T @ q)
+    return dq, dk, dv, dsum
+
+
+def attention_backward(q, k, v, dout, scale, causal=False, seqlens=None,
+                       dropout_p=0.0, seed=0, block_mask=None, heads=None):
+    """dQ, dK, dV (float64 [B,H,N,d]) for every (b, h) in ``heads`` (default all)."""
+    q, k, v, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    B, H, N, d = q.shape
+    dq = np.full_like(q, np.nan)
+    dk = np.full_like(k, np.nan)
+    dv = np.full_like(v, np.nan)
+    pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    p32 = float(np.float32(dropout_p))
+    for b, h in pairs:
+        kv_len = None if seqlens is None else int(seqlens[b])
+        keep = dropout_keep(seed, p32, b, h, np.arange(N), N) if p32 > 0 else None
+        g = head_backward(q[b, h], k[b, h], v[b, h], dout[b, h], scale, causal,
+                          kv_len, block_mask, keep, p32)
+        dq[b, h], dk[b, h], dv[b, h] = g[0], g[1], g[2]
+    return dq, dk, dv
+

@@ -1,0 +1,430 @@
+"""Pins for the float64 oracle: each checks it against something other than itself.
+
+A pin is a value the pages print, a closed form, an invariant of the
+mathematics, an independent library routine or brute force.  Each test names
+the plausible oracle mistake it would catch.
+"""
+
+import json
+import math
+import os
+from decimal import Decimal, getcontext
+
+import numpy as np
+import pytest
+
+from oracle import (
+    attention_backward,
+    attention_forward,
+    dropout_keep,
+    dropout_threshold,
+    head_backward,
+    philox4x32_10,
+    philox_block,
+    safe_softmax,
+    valid_mask,
+    weyl_constants,
+)
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+# (causal, kv_len, block-mask kind) combinations used throughout
+MASK_MODES = [
+    dict(),
+    dict(causal=True),
+    dict(kv_len=True),
+    dict(block=True),
+    dict(causal=True, kv_len=True, block=True),
+]
+
+
+def _mask_args(mode, B, N, rng):
+    causal = mode.get("causal", False)
+    seqlens = None
+    if mode.get("kv_len"):
+        seqlens = rng.integers(max(1, N // 2), N + 1, size=B).astype(np.int32)
+    block = None
+    if mode.get("block"):
+        nb = (N + 127) // 128
+        block = (rng.random((nb, nb)) < 0.5).astype(np.uint8)
+        np.fill_diagonal(block, 1)
+    return causal, seqlens, block
+
+
+def _rand(shape, rng):
+    return rng.standard_normal(shape)
+
+
+# ---------------------------------------------------------------------------
+# Philox
+# ---------------------------------------------------------------------------
+
+def test_philox_round_structure_matches_numpy_philox4x64():
+    """numpy.random.Philox is an independent Philox4x64-10.  The generic round
+    function of the oracle at width 64 must reproduce its raw output (numpy
+    increments the 256-bit counter before producing each 4-word block).  Catches
+    a wrong permutation of the words, a wrong key schedule or round count."""
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        ctr = [int(x) for x in rng.integers(0, 2**63, size=4, dtype=np.uint64)]
+        ctr[1] = ctr[1] % 1000  # keep the carry into word 1 simple
+        key = [int(x) for x in rng.integers(0, 2**63, size=2, dtype=np.uint64)]
+        bg = np.random.Philox(counter=np.array(ctr, dtype=np.uint64),
+                              key=np.array(key, dtype=np.uint64))
+        got = [int(x) for x in bg.random_raw(4)]
+        nxt = list(ctr)
+        nxt[0] = (nxt[0] + 1) % 2**64
+        if nxt[0] == 0:
+            nxt[1] += 1
+        want = list(philox_block(nxt, key, width=64, rounds=10))
+        assert got == want
+
+
+def test_weyl_constants_from_high_precision_arithmetic():
+    """Key increments are floor(2^w (phi-1)) and floor(2^w (sqrt3-1)); recompute
+    them with 60-digit decimal arithmetic (an independent route from isqrt)."""
+    getcontext().prec = 60
+    for w in (32, 64):
+        s = Decimal(2) ** w
+        phi1 = (Decimal(5).sqrt() - 1) / 2
+        s31 = Decimal(3).sqrt() - 1
+        assert weyl_constants(w) == (int(s * phi1), int(s * s31))
+
+
+def test_philox4x32_vectorised_equals_scalar_definition():
+    rng = np.random.default_rng(7)
+    c = rng.integers(0, 2**32, size=(4, 64), dtype=np.uint64)
+    k = rng.integers(0, 2**32, size=(2, 64), dtype=np.uint64)
+    vec = philox4x32_10(c[0], c[1], c[2], c[3], k[0], k[1])
+    for n in range(64):
+        want = philox_block([c[i, n] for i in range(4)], [k[0, n], k[1, n]], 32, 10)
+        assert tuple(int(v[n]) for v in vec) == want
+
+
+def test_philox4x32_words_are_uniform():
+    """Chi-square of byte values and the mean of 2^20 words: a generator with a
+    dropped round or a wrong multiplier on a structured counter sequence fails."""
+    n = 1 << 18
+    ctr = np.arange(n, dtype=np.uint64)
+    words = np.stack(philox4x32_10(ctr, 0, 0, 0, 0x12345678, 0x9ABCDEF0)).ravel()
+    assert abs(words.astype(np.float64).mean() / 2**32 - 0.5) < 5 * math.sqrt(1 / 12 / words.size)
+    counts = np.bincount((words & 0xFF).astype(np.int64), minlength=256)
+    e = words.size / 256
+    chi2 = ((counts - e) ** 2 / e).sum()
+    # 255 degrees of freedom: mean 255, sd ~22.6; allow 6 sd
+    assert chi2 < 255 + 6 * math.sqrt(2 * 255)
+    # successive counters must decorrelate: lag-1 correlation of the words
+    x = words[::4].astype(np.float64)
+    r = np.corrcoef(x[:-1], x[1:])[0, 1]
+    assert abs(r) < 5 / math.sqrt(x.size)
+
+
+# ---------------------------------------------------------------------------
+# dropout bits
+# ---------------------------------------------------------------------------
+
+def test_dropout_threshold_is_exact_integer_of_float32_p():
+    # 0.1 as float32 is 13421773 * 2^-27, so p * 2^32 = 429496736 exactly
+    assert dropout_threshold(0.1) == 429496736
+    assert dropout_threshold(0.0) == 0
+    assert dropout_threshold(0.5) == 2**31
+    assert dropout_threshold(np.nextafter(np.float32(1), np.float32(0))) == 2**32 - 2**8
+    for bad in (-0.1, 1.0, 1.5, float("nan")):
+        with pytest.raises(ValueError):
+            dropout_threshold(bad)
+
+
+def test_dropout_keep_uses_the_stated_counter_mapping():
+    """keep(b,h,i,j) = word (j & 3) of Philox4x32-10(counter=(j>>2, i, h, b),
+    key=(seed lo, seed hi)) >= t, checked element by element by brute force."""
+    seed = 0x0123456789ABCDEF
+    p = 0.3
+    t = dropout_threshold(p)
+    rows = np.array([0, 1, 5, 130])
+    keep = dropout_keep(seed, p, 3, 2, rows, 11)
+    for a, i in enumerate(rows):
+        for j in range(11):
+            w = philox_block([j >> 2, int(i), 2, 3], [seed & 0xFFFFFFFF, seed >> 32])[j & 3]
+            assert keep[a, j] == (w >= t)
+
+
+def test_dropout_keep_rate_within_5_sigma():
+    """Over ~10^7 draws the keep fraction is 1 - p within 5 sigma (binomial)."""
+    for p in (0.1, 0.5):
+        keep = dropout_keep(77, p, 1, 4, np.arange(2500), 4000)
+        n = keep.size
+        q = 1 - float(np.float32(p))
+        assert abs(keep.mean() - q) < 5 * math.sqrt(q * (1 - q) / n)
+
+
+def test_dropout_p_zero_keeps_everything():
+    assert dropout_keep(1, 0.0, 0, 0, np.arange(4), 9).all()
+
+
+# ---------------------------------------------------------------------------
+# softmax
+# ---------------------------------------------------------------------------
+
+def test_safe_softmax_pages_constant_rows():
+    """The pages' overflow/underflow example: every score equal to c = +-20000.
+    The safe softmax must give the uniform row with no inf/nan."""
+    with open(os.path.join(GOLDEN, "safe_softmax_constant_rows.json")) as f:
+        gold = json.load(f)
+    for case in gold["cases"]:
+        s = np.full((3, case["n"]), case["c"])
+        p, lse, _, _ = safe_softmax(s, np.ones_like(s, dtype=bool))
+        assert np.isfinite(p).all() and np.isfinite(lse).all()
+        assert np.array_equal(p, np.full_like(p, case["p"]))
+        assert np.allclose(lse, case["c"] + math.log(case["n"]), rtol=0, atol=1e-9)
+
+
+def test_softmax_shift_invariance_at_plus_minus_20000():
+    rng = np.random.default_rng(1)
+    s = rng.standard_normal((16, 40))
+    valid = rng.random((16, 40)) < 0.7
+    valid[:, 0] = True
+    p0, lse0, _, _ = safe_softmax(s, valid)
+    for c in (20000.0, -20000.0):
+        p, lse, _, _ = safe_softmax(s + c, valid)
+        assert np.isfinite(p).all()
+        assert np.abs(p - p0).max() < 1e-12
+        assert np.abs(lse - (lse0 + c)).max() < 1e-9
+
+
+def test_softmax_rows_sum_to_one_and_vanish_off_mask():
+    rng = np.random.default_rng(2)
+    for mode in MASK_MODES:
+        B, N = 2, 300
+        causal, seqlens, block = _mask_args(mode, B, N, rng)
+        for b in range(B):
+            kv = None if seqlens is None else seqlens[b]
+            rows = np.arange(N)
+            valid = valid_mask(N, rows, causal, kv, block)
+            s = 3 * rng.standard_normal((N, N))
+            p, _, _, _ = safe_softmax(s, valid)
+            has = valid.any(axis=1)
+            assert (p >= 0).all()
+            assert np.abs(p.sum(axis=1)[has] - 1).max() < 1e-12
+            assert (p[~valid] == 0).all()
+
+
+def test_valid_mask_brute_force():
+    rng = np.random.default_rng(3)
+    N = 260
+    block = (rng.random((3, 3)) < 0.5).astype(np.uint8)
+    rows = np.arange(N)
+    m = valid_mask(N, rows, True, 200, block)
+    for i in range(0, N, 7):
+        for j in range(0, N, 5):
+            want = (j <= i) and (j < 200) and bool(block[i // 128, j // 128])
+            assert m[i, j] == want
+
+
+# ---------------------------------------------------------------------------
+# forward: closed forms
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", MASK_MODES)
+def test_constant_v_rows_give_that_constant(mode):
+    """V_j = v for every j gives O_i = v on every row with a valid key."""
+    rng = np.random.default_rng(11)
+    B, H, N, d = 2, 2, 200, 8
+    causal, seqlens, block = _mask_args(mode, B, N, rng)
+    q, k = _rand((B, H, N, d), rng), _rand((B, H, N, d), rng)
+    vrow = rng.standard_normal((B, H, 1, d))
+    v = np.broadcast_to(vrow, (B, H, N, d)).copy()
+    o, lse = attention_forward(q, k, v, 0.3, causal, seqlens, block_mask=block)
+    for b in range(B):
+        kv = None if seqlens is None else seqlens[b]
+        has = valid_mask(N, np.arange(N), causal, kv, block).any(axis=1)
+        for h in range(H):
+            assert np.abs(o[b, h][has] - vrow[b, h]).max() < 1e-12
+            assert (o[b, h][~has] == 0).all()
+            assert np.isneginf(lse[b, h][~has]).all()
+
+
+@pytest.mark.parametrize("mode", MASK_MODES)
+def test_zero_q_gives_masked_mean_and_log_count(mode):
+    """Q = 0 makes every valid score 0: O_i is the mean of V over the valid keys
+    of row i and LSE_i = ln(number of valid keys)."""
+    rng = np.random.default_rng(12)
+    B, H, N, d = 2, 1, 260, 4
+    causal, seqlens, block = _mask_args(mode, B, N, rng)
+    q = np.zeros((B, H, N, d))
+    k, v = _rand((B, H, N, d), rng), _rand((B, H, N, d), rng)
+    o, lse = attention_forward(q, k, v, 0.125, causal, seqlens, block_mask=block)
+    for b in range(B):
+        kv = None if seqlens is None else seqlens[b]
+        valid = valid_mask(N, np.arange(N), causal, kv, block)
+        for i in range(N):
+            cnt = valid[i].sum()
+            if cnt == 0:
+                assert (o[b, 0, i] == 0).all() and np.isneginf(lse[b, 0, i])
+                continue
+            assert np.abs(o[b, 0, i] - v[b, 0][valid[i]].mean(axis=0)).max() < 1e-12
+            assert abs(lse[b, 0, i] - math.log(cnt)) < 1e-12
+
+
+def test_huge_scores_do_not_overflow_in_attention():
+    """Scores of +-20000 through the whole forward: q = c e_0, every key e_0."""
+    B, H, N, d = 1, 1, 6, 4
+    k = np.zeros((B, H, N, d))
+    k[..., 0] = 1.0
+    v = np.arange(N * d, dtype=np.float64).reshape(1, 1, N, d)
+    for c in (20000.0, -20000.0):
+        q = np.zeros((B, H, N, d))
+        q[..., 0] = c
+        o, lse = attention_forward(q, k, v, 1.0)
+        assert np.isfinite(o).all() and np.isfinite(lse).all()
+        assert np.abs(o[0, 0] - v[0, 0].mean(axis=0)).max() < 1e-9
+        assert np.abs(lse - (c + math.log(N))).max() < 1e-9
+
+
+def test_slab_size_does_not_change_any_value():
+    """Rows are independent: slabs of 1 row and of 256 rows agree to rounding
+    (BLAS may sum in another order for another shape); the row-subset interface
+    returns the same rows."""
+    rng = np.random.default_rng(13)
+    q, k, v = (_rand((1, 2, 300, 8), rng) for _ in range(3))
+    a = attention_forward(q, k, v, 0.2, True, dropout_p=0.2, seed=9, slab=1)
+    b = attention_forward(q, k, v, 0.2, True, dropout_p=0.2, seed=9, slab=256)
+    assert np.abs(a[0] - b[0]).max() < 1e-13 and np.abs(a[1] - b[1]).max() < 1e-13
+    rows = np.array([0, 131, 299])
+    c = attention_forward(q, k, v, 0.2, True, dropout_p=0.2, seed=9, rows=rows)
+    assert np.allclose(c[0], a[0][:, :, rows], rtol=0, atol=1e-14)
+
+
+def test_dropout_is_unbiased_on_average():
+    """E[Z/(1-p)] = 1: averaged over many seeds, dropped attention approaches
+    the undropped output (inverted dropout)."""
+    rng = np.random.default_rng(14)
+    q, k, v = (_rand((1, 1, 16, 4), rng) for _ in range(3))
+    o0, lse0 = attention_forward(q, k, v, 0.5)
+    acc = np.zeros_like(o0)
+    n = 400
+    for s in range(n):
+        o, lse = attention_forward(q, k, v, 0.5, dropout_p=0.25, seed=1000 + s)
+        assert np.array_equal(lse, lse0)  # LSE is that of the undropped softmax
+        acc += o
+    err = np.abs(acc / n - o0).max()
+    assert err < 0.15
+
+
+# ---------------------------------------------------------------------------
+# forward + backward against an independent library routine
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", MASK_MODES)
+def test_matches_torch_sdpa_and_autograd_without_dropout(mode):
+    """torch.nn.functional.scaled_dot_product_attention (CPU, float64, boolean
+    mask) and torch.autograd compute the same definition independently."""
+    import torch
+
+    rng = np.random.default_rng(15)
+    B, H, N, d = 2, 2, 150, 16
+    causal, seqlens, block = _mask_args(mode, B, N, rng)
+    q, k, v, do = (_rand((B, H, N, d), rng) for _ in range(4))
+    scale = 0.2
+    o, lse = attention_forward(q, k, v, scale, causal, seqlens, block_mask=block)
+    dq, dk, dv = attention_backward(q, k, v, do, scale, causal, seqlens, block_mask=block)
+
+    mask = np.stack([valid_mask(N, np.arange(N), causal,
+                                None if seqlens is None else seqlens[b], block)
+                     for b in range(B)])[:, None]
+    has = mask.any(axis=-1)  # rows with at least one valid key
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=torch.tensor(mask), scale=scale)
+    # fully masked rows give NaN in SDPA; compare only rows that have keys
+    to = torch.where(torch.tensor(has)[..., None], to, torch.zeros_like(to))
+    (to * torch.tensor(do)).sum().backward()
+    assert np.abs(o - to.detach().numpy()).max() < 1e-12
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.abs(mine - ref.numpy()).max() < 1e-10
+    # the LSE against a direct logsumexp of the masked scores
+    s = scale * np.einsum("bhid,bhjd->bhij", q, k)
+    s = np.where(mask, s, -np.inf)
+    with np.errstate(divide="ignore"):
+        ref_lse = np.log(np.exp(s - s.max(-1, keepdims=True, initial=-1e300)).sum(-1)) \
+            + s.max(-1, initial=-1e300)
+    assert np.abs(np.where(has, lse - ref_lse, 0)).max() < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# backward: finite differences and identities
+# ---------------------------------------------------------------------------
+
+FD_CASES = [
+    (5, 4, dict(), 0.0),
+    (8, 8, dict(causal=True), 0.0),
+    (16, 4, dict(kv_len=True), 0.0),
+    (16, 8, dict(causal=True, kv_len=True), 0.3),
+    (8, 4, dict(), 0.5),
+]
+
+
+@pytest.mark.parametrize("N,d,mode,p", FD_CASES)
+def test_backward_matches_central_finite_differences(N, d, mode, p):
+    """dL/dx for L = sum(O * dO) by central differences in float64, dropout bits
+    held fixed by the seed: catches a dropped term, sign or transposition."""
+    rng = np.random.default_rng(100 + N + d)
+    B, H = 1, 1
+    causal = mode.get("causal", False)
+    seqlens = np.array([max(1, N - 3)], dtype=np.int32) if mode.get("kv_len") else None
+    q, k, v, do = (_rand((B, H, N, d), rng) for _ in range(4))
+    scale, seed = 0.7, 4242
+
+    def loss(q_, k_, v_):
+        o, _ = attention_forward(q_, k_, v_, scale, causal, seqlens, p, seed)
+        return float((o * do).sum())
+
+    dq, dk, dv = attention_backward(q, k, v, do, scale, causal, seqlens, p, seed)
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        err = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+        assert err < 1e-6, (name, err)
+
+
+@pytest.mark.parametrize("p", [0.0, 0.2])
+def test_backward_identities(p):
+    """(i) sum_j dK_j = 0 per (b,h); (ii) D_i = sum_j P_ij dP_ij equals
+    sum_c dO_ic O_ic; (iii) constant key rows give dQ = 0."""
+    rng = np.random.default_rng(21)
+    N, d = 200, 8
+    q, k, v, do = (_rand((N, d), rng) for _ in range(4))
+    keep = dropout_keep(5, p, 0, 0, np.arange(N), N) if p > 0 else None
+    dq, dk, dv, dsum = head_backward(q, k, v, do, 0.4, True, None, None, keep, p)
+    assert np.abs(dk.sum(axis=0)).max() < 1e-10
+    o, _ = attention_forward(q[None, None], k[None, None], v[None, None], 0.4, True,
+                             dropout_p=p, seed=5)
+    assert np.abs(dsum - (do * o[0, 0]).sum(axis=1)).max() < 1e-10
+    kc = np.broadcast_to(k[:1], k.shape).copy()
+    dq2, _, _, _ = head_backward(q, kc, v, do, 0.4, True, None, None, keep, p)
+    assert np.abs(dq2).max() < 1e-12
+
+
+def test_zero_q_gives_closed_form_dv():
+    """Q = 0, no dropout: P_ij = 1/n_i on the valid keys, so
+    dV_j = sum over rows i where j is valid of dO_i / n_i."""
+    rng = np.random.default_rng(22)
+    N, d = 140, 4
+    q = np.zeros((N, d))
+    k, v, do = (_rand((N, d), rng) for _ in range(3))
+    _, _, dv, _ = head_backward(q, k, v, do, 1.0, True, 100)
+    valid = valid_mask(N, np.arange(N), True, 100)
+    n = valid.sum(axis=1)
+    want = np.zeros((N, d))
+    for i in range(N):
+        for j in np.nonzero(valid[i])[0]:
+            want[j] += do[i] / n[i]
+    assert np.abs(dv - want).max() < 1e-12
