@@ -1,0 +1,455 @@
+// Forward pass of exact attention on sm_100a.
+//
+// Work unit: one (b, h) and 256 query rows, held as two 128-row Q tiles that
+// share every K/V tile the CTA loads.  The CTA walks the K/V tiles of its head
+// that at least one of its Q tiles needs (tiles that are fully masked by the
+// causal mask, the key lengths or the block mask are neither loaded nor
+// computed).  Per K/V tile and per active Q tile t:
+//
+//   S_t = Q_t K^T           tcgen05.mma, bf16 x bf16 -> fp32 in TMEM
+//   P_t = exp2(S_t * scale * log2e - m_t)   online softmax, one thread per row
+//   O_t += P_t V            tcgen05.mma with P_t read from TMEM
+//
+// Roles (384 threads):
+//   warp 0       TMA producer: Q tiles once, then K/V tiles into a ring
+//   warp 1       TMEM allocator and single-thread MMA issuer
+//   warps 2-3    idle
+//   warps 4-7    softmax for Q tile 0   (thread = row, TMEM lanes 0..127)
+//   warps 8-11   softmax for Q tile 1
+//
+// The running maximum m is only moved when a new block raises it by more than
+// 8 (in log2 units); until then exp2 values may reach 2^8, and O and the row
+// sum l keep using the same stale maximum, so the final O / l and
+// LSE = ln2 * (m + log2 l) are unchanged (the online-softmax rescaling of the
+// tiling section of the pages, applied lazily).
+//
+// TMEM columns: S/P of tile t at [128 t, 128 t + 128) (P packed as bf16 pairs in
+// the first 64 columns), O of tile t at [256 + D t, 256 + D t + D).
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "philox.cuh"
+#include "ptx.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kFwdThreads = 384;
+constexpr float kLn2 = 0.693147180559945309f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdLayout {
+  static constexpr int PANELS = D / 64;                 // 64-column, 128-byte-swizzled panels
+  static constexpr uint32_t PANEL = 128u * 128u;        // bytes of one [128 rows][64 cols] panel
+  static constexpr uint32_t TILE = PANEL * PANELS;      // bytes of one 128-row tile
+  static constexpr int STAGES = (D == 64) ? 4 : 2;      // K/V ring depth
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_KV = 2 * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_KV + STAGES * 2 * TILE;
+  static constexpr int B_QFULL = 0;
+  static constexpr int B_KFULL = 2;
+  static constexpr int B_VFULL = B_KFULL + STAGES;
+  static constexpr int B_KVEMPTY = B_VFULL + STAGES;
+  static constexpr int B_SFULL = B_KVEMPTY + STAGES;
+  static constexpr int B_PFULL = B_SFULL + 2;
+  static constexpr int B_ODONE = B_PFULL + 2;
+  static constexpr int B_DRAIN = B_ODONE + 2;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t SMEM = OFF_MISC + 16;
+  static constexpr uint32_t O_COL = 256;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(O_COL + 2 * D <= 512, "TMEM budget");
+};
+
+// Which (Q tile, K/V tile) pairs of this CTA take part.
+struct FwdWork {
+  int b, h, bh, q0, qb0, kv_len, n_kb, kb_end, nblk;
+  bool exists1, causal;
+  const uint8_t* bm;
+
+  __device__ __forceinline__ bool act(int t, int kb) const {
+    if (t == 1 && !exists1) return false;
+    if (kb >= n_kb) return false;
+    const int qb = qb0 + t;
+    if (causal && kb > qb) return false;
+    if (bm != nullptr && bm[static_cast<size_t>(qb) * nblk + kb] == 0) return false;
+    return true;
+  }
+  __device__ __forceinline__ bool any(int kb) const { return act(0, kb) || act(1, kb); }
+  __device__ __forceinline__ int next(int kb) const {
+    while (kb < kb_end && !any(kb)) ++kb;
+    return kb;
+  }
+};
+
+template <int D, bool DROPOUT>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {  // the swizzled layouts need 1024-byte alignment
+    if (threadIdx.x == 0 && p.status) atomicExch(p.status, kStatusInternal);
+    return;
+  }
+  auto bar = [&](int i) -> uint32_t { return sbase + L::OFF_BAR + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC + 4);
+  const WaitGuard g{abort_flag, p.status, p.timeout_ns};
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  FwdWork w;
+  {
+    const int nqp = (p.N + 255) / 256;
+    const int qp = nqp - 1 - static_cast<int>(blockIdx.x);  // heaviest causal rows first
+    w.q0 = qp * 256;
+    w.qb0 = qp * 2;
+    w.bh = blockIdx.y;
+    w.b = w.bh / p.H;
+    w.h = w.bh % p.H;
+    w.exists1 = (w.q0 + 128) < p.N;
+    int kv = p.N;
+    if (p.seqlens != nullptr) kv = max(0, min(p.seqlens[w.b], p.N));
+    w.kv_len = kv;
+    w.n_kb = (kv + 127) / 128;
+    w.causal = p.causal != 0;
+    w.kb_end = w.causal ? min(w.n_kb, w.qb0 + (w.exists1 ? 2 : 1)) : w.n_kb;
+    w.nblk = p.nblk;
+    w.bm = p.block_mask;
+  }
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0u;
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::B_QFULL + t), 1);
+      mbar_init(bar(L::B_SFULL + t), 1);
+      mbar_init(bar(L::B_PFULL + t), 128);
+      mbar_init(bar(L::B_ODONE + t), 1);
+    }
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(bar(L::B_KFULL + s), 1);
+      mbar_init(bar(L::B_VFULL + s), 1);
+      mbar_init(bar(L::B_KVEMPTY + s), 1);
+    }
+    mbar_init(bar(L::B_DRAIN), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      for (int t = 0; t < 2; ++t) {
+        if (t == 1 && !w.exists1) break;
+        mbar_arrive_expect_tx(bar(L::B_QFULL + t), L::TILE);
+        for (int pn = 0; pn < L::PANELS; ++pn)
+          tma_load_3d(sbase + L::OFF_Q + t * L::TILE + pn * L::PANEL, &tm_q, bar(L::B_QFULL + t),
+                      64 * pn, w.q0 + 128 * t, w.bh);
+      }
+      int it = 0;
+      for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1), ++it) {
+        const int s = it % L::STAGES;
+        const uint32_t ph = (it / L::STAGES) & 1u;
+        if (it >= L::STAGES && !mbar_wait(bar(L::B_KVEMPTY + s), ph ^ 1u, g)) break;
+        const uint32_t kdst = sbase + L::OFF_KV + s * 2 * L::TILE;
+        const uint32_t vdst = kdst + L::TILE;
+        mbar_arrive_expect_tx(bar(L::B_KFULL + s), L::TILE);
+        for (int pn = 0; pn < L::PANELS; ++pn)
+          tma_load_3d(kdst + pn * L::PANEL, &tm_k, bar(L::B_KFULL + s), 64 * pn, kb * 128, w.bh);
+        mbar_arrive_expect_tx(bar(L::B_VFULL + s), L::TILE);
+        for (int pn = 0; pn < L::PANELS; ++pn)
+          tma_load_3d(vdst + pn * L::PANEL, &tm_v, bar(L::B_VFULL + s), 64 * pn, kb * 128, w.bh);
+      }
+      if (*abort_flag) {  // let the copies already issued land before the CTA exits
+        for (int j = max(0, it - L::STAGES); j < it; ++j) {
+          const int s = j % L::STAGES;
+          const uint32_t ph = (j / L::STAGES) & 1u;
+          mbar_wait_drain(bar(L::B_KFULL + s), ph, 100000000ull);
+          mbar_wait_drain(bar(L::B_VFULL + s), ph, 100000000ull);
+        }
+        mbar_wait_drain(bar(L::B_QFULL + 0), 0, 100000000ull);
+        if (w.exists1) mbar_wait_drain(bar(L::B_QFULL + 1), 0, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);
+      bool q_ready[2] = {false, false};
+      bool o_init[2] = {false, false};
+      uint32_t p_cnt[2] = {0u, 0u};
+      bool ok = true;
+
+      auto issue_s = [&](int t, uint32_t kaddr) {
+        const uint32_t qaddr = sbase + L::OFF_Q + t * L::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::PANEL + (kk & 3) * 32;
+          mma_ss(tmem + 128 * t, sdesc_sw128(qaddr + off, 16, 1024),
+                 sdesc_sw128(kaddr + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(L::B_SFULL + t));
+      };
+      auto ensure_q = [&](int t) -> bool {
+        if (q_ready[t]) return true;
+        if (!mbar_wait(bar(L::B_QFULL + t), 0, g)) return false;
+        q_ready[t] = true;
+        return true;
+      };
+
+      int kb = w.next(0);
+      int it = 0;
+      if (kb < w.kb_end) {
+        ok = mbar_wait(bar(L::B_KFULL + 0), 0, g);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!w.act(t, kb)) continue;
+          ok = ensure_q(t);
+          if (ok) {
+            tc_fence_after();
+            issue_s(t, sbase + L::OFF_KV);
+          }
+        }
+      }
+      while (ok && kb < w.kb_end) {
+        const int s = it % L::STAGES;
+        const uint32_t ph = (it / L::STAGES) & 1u;
+        const int kbn = w.next(kb + 1);
+        const int sn = (it + 1) % L::STAGES;
+        const uint32_t phn = ((it + 1) / L::STAGES) & 1u;
+        bool kn_ready = false;
+        if (!mbar_wait(bar(L::B_VFULL + s), ph, g)) break;
+        const uint32_t vaddr = sbase + L::OFF_KV + s * 2 * L::TILE + L::TILE;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (w.act(t, kb)) {
+            if (!mbar_wait(bar(L::B_PFULL + t), p_cnt[t] & 1u, g)) {
+              ok = false;
+              break;
+            }
+            ++p_cnt[t];
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + L::O_COL + D * t, tmem + 128 * t + 8 * kk,
+                     sdesc_sw128(vaddr + kk * 2048, L::PANEL, 1024), kIdPV,
+                     (o_init[t] || kk > 0) ? 1u : 0u);
+            o_init[t] = true;
+            mma_commit(bar(L::B_ODONE + t));
+          }
+          if (kbn < w.kb_end && w.act(t, kbn)) {
+            if (!kn_ready) {
+              if (!mbar_wait(bar(L::B_KFULL + sn), phn, g)) {
+                ok = false;
+                break;
+              }
+              kn_ready = true;
+            }
+            if (!ensure_q(t)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(t, sbase + L::OFF_KV + sn * 2 * L::TILE);
+          }
+        }
+        if (!ok) break;
+        mma_commit(bar(L::B_KVEMPTY + s));
+        kb = kbn;
+        ++it;
+      }
+      // every MMA issued above has completed once this commit arrives
+      mma_commit(bar(L::B_DRAIN));
+      mbar_wait_drain(bar(L::B_DRAIN), 0, 1000000000ull);
+      for (int t = 0; t < 2; ++t)
+        if ((t == 0 || w.exists1) && !q_ready[t]) mbar_wait_drain(bar(L::B_QFULL + t), 0, 100000000ull);
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- softmax
+    const int t = (warp - 4) >> 2;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const int i = w.q0 + 128 * t + r;
+    if (t == 0 || w.exists1) {
+      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+      const uint32_t s_addr = lane_addr + 128 * t;
+      const uint32_t o_addr = lane_addr + L::O_COL + D * t;
+      float m = -INFINITY;  // reference maximum, log2 units of scaled scores
+      float l = 0.f;        // row sum of exp2(x - m)
+      uint32_t cnt = 0;     // active K/V tiles processed so far
+      bool ok = true;
+      for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1)) {
+        if (!w.act(t, kb)) continue;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + t), cnt & 1u, g));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32<0>(s_addr + 0, sr);
+        tmem_ld32<32>(s_addr + 32, sr);
+        tmem_ld32<64>(s_addr + 64, sr);
+        tmem_ld32<96>(s_addr + 96, sr);
+        tmem_wait_ld32<0>(sr);
+        tmem_wait_ld32<32>(sr);
+        tmem_wait_ld32<64>(sr);
+        tmem_wait_ld32<96>(sr);
+
+        const int j0 = kb * 128;
+        const bool need_mask = (w.causal && kb == w.qb0 + t) || (j0 + 128 > w.kv_len);
+        float mx = -INFINITY;
+        if (need_mask) {
+          const int lim = w.causal ? min(w.kv_len - j0, i - j0 + 1) : (w.kv_len - j0);
+#pragma unroll
+          for (int j = 0; j < 128; ++j) {
+            const float v = (j < lim) ? __uint_as_float(sr[j]) : -INFINITY;
+            sr[j] = __float_as_uint(v);
+            mx = fmaxf(mx, v);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 128; ++j) mx = fmaxf(mx, __uint_as_float(sr[j]));
+        }
+        mx *= p.scale_log2;
+        const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = fast_exp2(m - m_use);  // 0 on the first tile, 1 if unchanged
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 128; j += 2) {
+          const float e0 = fast_exp2(fmaf(__uint_as_float(sr[j]), p.scale_log2, -m_use));
+          const float e1 = fast_exp2(fmaf(__uint_as_float(sr[j + 1]), p.scale_log2, -m_use));
+          rs0 += e0;
+          rs1 += e1;
+          sr[j] = __float_as_uint(e0);
+          sr[j + 1] = __float_as_uint(e1);
+        }
+        l = l * alpha + (rs0 + rs1);
+        m = m_new;
+
+        if constexpr (DROPOUT) {
+          const uint32_t thr = p.drop_threshold;
+#pragma unroll
+          for (int gq = 0; gq < 32; ++gq) {
+            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(kb * 32 + gq),
+                                              static_cast<uint32_t>(i), static_cast<uint32_t>(w.h),
+                                              static_cast<uint32_t>(w.b), p.seed_lo, p.seed_hi);
+            if (rnd.w0 < thr) sr[4 * gq + 0] = 0u;
+            if (rnd.w1 < thr) sr[4 * gq + 1] = 0u;
+            if (rnd.w2 < thr) sr[4 * gq + 2] = 0u;
+            if (rnd.w3 < thr) sr[4 * gq + 3] = 0u;
+          }
+        }
+
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          pk[c] = pack_bf16(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]));
+        tmem_st32<0>(s_addr + 0, pk);
+        tmem_st32<32>(s_addr + 32, pk);
+
+        if (cnt > 0) {
+          // previous O += P V is complete (it precedes the S MMA just consumed)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ODONE + t), (cnt - 1) & 1u, g));
+          if (!ok) break;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t orr[32];
+              tmem_ld32<0>(o_addr + 32 * c, orr);
+              tmem_wait_ld32<0>(orr);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) orr[k] = __float_as_uint(__uint_as_float(orr[k]) * alpha);
+              tmem_st32<0>(o_addr + 32 * c, orr);
+            }
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::B_PFULL + t));
+        ++cnt;
+      }
+
+      // ------------------------------------------------------------ epilogue
+      if (ok && cnt > 0)
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ODONE + t), (cnt - 1) & 1u, g));
+      if (ok) {
+        tc_fence_after();
+        const bool row_ok = i < p.N;
+        const float inv = (l > 0.f) ? p.drop_rscale / l : 0.f;
+        __nv_bfloat16* orow =
+            reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(w.bh) * p.N + i) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          if (cnt > 0) {
+            tmem_ld32<0>(o_addr + 32 * c, orr);
+            tmem_wait_ld32<0>(orr);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) orr[k] = 0u;
+          }
+          uint32_t ob[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            ob[k] = pack_bf16(__uint_as_float(orr[2 * k]) * inv, __uint_as_float(orr[2 * k + 1]) * inv);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              dst[k] = make_uint4(ob[4 * k], ob[4 * k + 1], ob[4 * k + 2], ob[4 * k + 3]);
+          }
+        }
+        if (row_ok)
+          p.lse[static_cast<size_t>(w.bh) * p.N + i] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool DROPOUT>
+cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const FwdParams& p, cudaStream_t stream) {
+  using L = FwdLayout<D>;
+  auto kern = fwd_kernel<D, DROPOUT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::SMEM));
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.N + 255) / 256, p.B * p.H);
+  kern<<<grid, kFwdThreads, L::SMEM, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const FwdParams& p, cudaStream_t stream) {
+  if (d == 64) return dropout ? launch_fwd_t<64, true>(tq, tk, tv, p, stream)
+                              : launch_fwd_t<64, false>(tq, tk, tv, p, stream);
+  if (d == 128) return dropout ? launch_fwd_t<128, true>(tq, tk, tv, p, stream)
+                               : launch_fwd_t<128, false>(tq, tk, tv, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fa

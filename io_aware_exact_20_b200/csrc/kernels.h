@@ -1,0 +1,64 @@
+// Internal interface between the C ABI (fa_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace fa {
+
+// Device status codes written to the per-device status word.
+enum : int { kStatusOk = 0, kStatusInternal = 3, kStatusTimeout = 4 };
+
+struct FwdParams {
+  void* o;                    // bf16 [B,H,N,d]
+  float* lse;                 // fp32 [B,H,N]
+  const int32_t* seqlens;     // int32 [B] or null
+  const uint8_t* block_mask;  // uint8 [nblk][nblk] or null
+  int* status;                // device status word
+  int B, H, N, nblk;
+  float scale_log2;           // softmax_scale * log2(e)
+  int causal;
+  uint32_t drop_threshold;    // keep iff word >= threshold
+  float drop_rscale;          // 1 / (1 - p)
+  uint32_t seed_lo, seed_hi;
+  uint64_t timeout_ns;
+};
+
+struct BwdParams {
+  const void* o;              // bf16 [B,H,N,d]  (forward output)
+  const void* dout;           // bf16 [B,H,N,d]
+  const float* lse;           // fp32 [B,H,N]
+  void* dq;                   // bf16 [B,H,N,d]
+  void* dk;                   // bf16 [B,H,N,d]
+  void* dv;                   // bf16 [B,H,N,d]
+  float* ws_lse2;             // fp32 [B*H][Npad]  LSE * log2(e), +inf where no key
+  float* ws_delta;            // fp32 [B*H][Npad]  sum_c dO_ic O_ic
+  float* ws_dq;               // fp32 [B*H][Npad][d] dQ accumulators (unscaled)
+  const int32_t* seqlens;
+  const uint8_t* block_mask;
+  int* status;
+  int B, H, N, Npad, nblk;
+  float scale;                // softmax_scale
+  float scale_log2;           // softmax_scale * log2(e)
+  int causal;
+  uint32_t drop_threshold;
+  float drop_rscale;
+  uint32_t seed_lo, seed_hi;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_fwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const FwdParams& p, cudaStream_t stream);
+
+cudaError_t launch_bwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p,
+                       cudaStream_t stream);
+
+cudaError_t launch_dropout_mask(uint8_t* keep, int B, int H, int N, uint32_t threshold,
+                                uint32_t seed_lo, uint32_t seed_hi, cudaStream_t stream);
+
+cudaError_t launch_wait_timeout_probe(int* status, uint64_t timeout_ns, cudaStream_t stream);
+
+}  // namespace fa

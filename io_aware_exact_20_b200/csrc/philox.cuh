@@ -1,0 +1,42 @@
+// Philox4x32-10 counter-based generator on the device, written from its
+// published definition (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers:
+// As Easy as 1, 2, 3", SC'11): ten rounds, each multiplying words 0 and 2 by
+// fixed odd multipliers, swapping high/low halves with the other two words
+// and the key, the key advanced between rounds by the Weyl constants
+// floor(2^32 (phi - 1)) and floor(2^32 (sqrt(3) - 1)).
+//
+// Dropout keep bit of (b, h, i, j): word (j & 3) of the block at counter
+// (j >> 2, i, h, b) with key (seed lo, seed hi); kept iff word >= threshold.
+#pragma once
+
+#include <cstdint>
+
+namespace fa {
+
+struct Philox4 {
+  uint32_t w0, w1, w2, w3;
+};
+
+__device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                 uint32_t c3, uint32_t k0, uint32_t k1) {
+  constexpr uint32_t kMul0 = 0xD2511F53u, kMul1 = 0xCD9E8D57u;
+  constexpr uint32_t kWeyl0 = 0x9E3779B9u, kWeyl1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += kWeyl0;
+      k1 += kWeyl1;
+    }
+    const uint32_t hi0 = __umulhi(kMul0, c0), lo0 = kMul0 * c0;
+    const uint32_t hi1 = __umulhi(kMul1, c2), lo1 = kMul1 * c2;
+    const uint32_t n0 = hi1 ^ c1 ^ k0;
+    const uint32_t n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return Philox4{c0, c1, c2, c3};
+}
+
+}  // namespace fa
