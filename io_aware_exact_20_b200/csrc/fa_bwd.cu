@@ -1,7 +1,548 @@
+// Backward pass of exact attention on sm_100a.
+//
+// The probabilities are not stored by the forward pass: they are rebuilt here
+// from the saved log-sum-exp (the recomputation of the pages: keep the softmax
+// statistics, recompute the attention blocks in the backward).  With
+// P = exp(S - LSE), dP = dO V^T (times the dropout keep / (1 - p)),
+// D_i = sum_c dO_ic O_ic and dS = P * (dP - D):
+//
+//   dV = P_drop^T dO,   dK = scale dS^T Q,   dQ = scale dS K.
+//
+// Three kernels:
+//   bwd_pre   D_i, LSE_i * log2(e) (+inf for rows without keys and padding
+//             rows, so that their P is exactly 0), zeroed dQ accumulators;
+//   bwd_main  one CTA per (b, h, 128-key tile), looping over the query tiles
+//             that tile meets; dK, dV stay in TMEM for the whole loop, dQ
+//             partial products are added into fp32 accumulators;
+//   bwd_post  dQ = bf16(scale * accumulator).
+//
+// bwd_main roles (512 threads):
+//   warp 0        TMA producer: K, V once; per query tile Q, dO and the
+//                 128-row slices of LSE*log2e and D into a ring
+//   warp 1        TMEM allocator and single-thread MMA issuer
+//   warps 4-11    two warpgroups, thread = key row; warpgroup w handles the
+//                 query columns [64 w, 64 w + 64): P from S^T, dS from dP^T,
+//                 P (bf16) back to TMEM, dS (bf16) to swizzled shared memory
+//   warps 12-15   dQ warpgroup, thread = query row: TMEM -> red.global.add
+//
+// TMEM columns: S^T [0,128) with P packed into [64 w, 64 w + 32) per
+// warpgroup; dP^T [128,256), reused for the dQ tile once dP^T is consumed;
+// dV [256, 256 + D); dK [256 + D, 256 + 2 D).
+#include <cuda_bf16.h>
+
 #include "kernels.h"
+#include "philox.cuh"
+#include "ptx.cuh"
+
 namespace fa {
-cudaError_t launch_bwd(int, bool, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                       const CUtensorMap&, const BwdParams&, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kBwdThreads = 512;
+constexpr float kLog2e = 1.44269504088896340736f;
+
+template <int D>
+struct BwdLayout {
+  static constexpr int PANELS = D / 64;
+  static constexpr uint32_t PANEL = 128u * 128u;
+  static constexpr uint32_t TILE = PANEL * PANELS;
+  static constexpr int STAGES = (D == 64) ? 3 : 2;
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_V = TILE;
+  static constexpr uint32_t OFF_Q = 2 * TILE;
+  static constexpr uint32_t OFF_DO = OFF_Q + STAGES * TILE;
+  static constexpr uint32_t OFF_DS = OFF_DO + STAGES * TILE;  // [128 keys][128 queries] bf16
+  static constexpr uint32_t OFF_LD = OFF_DS + 2 * PANEL;      // per stage: lse2[128], delta[128]
+  static constexpr uint32_t OFF_BAR = OFF_LD + STAGES * 1024;
+  static constexpr int B_KV = 0;
+  static constexpr int B_QFULL = 1;
+  static constexpr int B_QEMPTY = B_QFULL + STAGES;
+  static constexpr int B_SFULL = B_QEMPTY + STAGES;
+  static constexpr int B_DPFULL = B_SFULL + 1;
+  static constexpr int B_PFULL = B_DPFULL + 1;
+  static constexpr int B_DSEMPTY = B_PFULL + 1;
+  static constexpr int B_DQFULL = B_DSEMPTY + 1;
+  static constexpr int B_DQEMPTY = B_DQFULL + 1;
+  static constexpr int B_KVDONE = B_DQEMPTY + 1;
+  static constexpr int NBAR = B_KVDONE + 1;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t SMEM = OFF_MISC + 16;
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(COL_DK + D <= 512, "TMEM budget");
+};
+
+struct BwdWork {
+  int b, h, bh, kb, kv_len, nqb, qb_begin, nblk;
+  bool alive, causal;
+  const uint8_t* bm;
+
+  __device__ __forceinline__ bool act(int qb) const {
+    if (!alive) return false;
+    if (bm != nullptr && bm[static_cast<size_t>(qb) * nblk + kb] == 0) return false;
+    return true;
+  }
+  __device__ __forceinline__ int next(int qb) const {
+    while (qb < nqb && !act(qb)) ++qb;
+    return qb;
+  }
+};
+
+// ---------------------------------------------------------------------------
+// pre / post kernels
+// ---------------------------------------------------------------------------
+
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
+  constexpr int G = D / 8;  // threads per row, 8 elements each
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = tid / G;
+  const int part = static_cast<int>(tid % G);
+  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Npad;
+  if (row >= rows) return;  // whole warps: rows is a multiple of 128
+  const int64_t bh = row / p.Npad;
+  const int i = static_cast<int>(row % p.Npad);
+  float acc = 0.f;
+  if (i < p.N) {
+    const size_t off = (static_cast<size_t>(bh) * p.N + i) * D + part * 8;
+    const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + off);
+    const uint4 gv =
+        *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + off);
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 a = __bfloat1622float2(o2[k]);
+      const float2 c = __bfloat1622float2(g2[k]);
+      acc = fmaf(a.x, c.x, acc);
+      acc = fmaf(a.y, c.y, acc);
+    }
+  }
+#pragma unroll
+  for (int m = G / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (part == 0) {
+    p.ws_delta[row] = (i < p.N) ? acc : 0.f;
+    float l2 = INFINITY;
+    if (i < p.N) {
+      const float l = p.lse[static_cast<size_t>(bh) * p.N + i];
+      if (l != -INFINITY) l2 = l * kLog2e;
+    }
+    p.ws_lse2[row] = l2;
+  }
+  float4* dq = reinterpret_cast<float4*>(p.ws_dq + row * D + part * 8);
+  dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+  dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
+
+template <int D>
+__global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(p.B) * p.H * p.N * (D / 8);
+  if (tid >= total) return;
+  const int64_t row = tid / (D / 8);  // bh * N + i
+  const int part = static_cast<int>(tid % (D / 8));
+  const int64_t bh = row / p.N;
+  const int64_t i = row % p.N;
+  const float4* src = reinterpret_cast<const float4*>(p.ws_dq + (bh * p.Npad + i) * D + part * 8);
+  const float4 a = src[0], c = src[1];
+  const float s = p.scale;
+  uint4 out;
+  out.x = pack_bf16(a.x * s, a.y * s);
+  out.y = pack_bf16(a.z * s, a.w * s);
+  out.z = pack_bf16(c.x * s, c.y * s);
+  out.w = pack_bf16(c.z * s, c.w * s);
+  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dq) + row * D + part * 8) = out;
+}
+
+// ---------------------------------------------------------------------------
+// main kernel
+// ---------------------------------------------------------------------------
+
+template <int D, bool DROPOUT>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using L = BwdLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0 && p.status) atomicExch(p.status, kStatusInternal);
+    return;
+  }
+  auto bar = [&](int i) -> uint32_t { return sbase + L::OFF_BAR + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC + 4);
+  const WaitGuard g{abort_flag, p.status, p.timeout_ns};
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  BwdWork w;
+  w.kb = blockIdx.x;
+  w.bh = blockIdx.y;
+  w.b = w.bh / p.H;
+  w.h = w.bh % p.H;
+  {
+    int kv = p.N;
+    if (p.seqlens != nullptr) kv = max(0, min(p.seqlens[w.b], p.N));
+    w.kv_len = kv;
+  }
+  w.alive = w.kb * 128 < w.kv_len;
+  w.nqb = (p.N + 127) / 128;
+  w.causal = p.causal != 0;
+  w.qb_begin = w.causal ? w.kb : 0;
+  w.nblk = p.nblk;
+  w.bm = p.block_mask;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0u;
+    mbar_init(bar(L::B_KV), 1);
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(bar(L::B_QFULL + s), 1);
+      mbar_init(bar(L::B_QEMPTY + s), 1);
+    }
+    mbar_init(bar(L::B_SFULL), 1);
+    mbar_init(bar(L::B_DPFULL), 1);
+    mbar_init(bar(L::B_PFULL), 256);
+    mbar_init(bar(L::B_DSEMPTY), 1);
+    mbar_init(bar(L::B_DQFULL), 1);
+    mbar_init(bar(L::B_DQEMPTY), 128);
+    mbar_init(bar(L::B_KVDONE), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int q_first = w.next(w.qb_begin);
+  const bool any_work = q_first < w.nqb;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0 && any_work) {
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      tma_prefetch_map(&tm_do);
+      mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::TILE);
+      for (int pn = 0; pn < L::PANELS; ++pn) {
+        tma_load_3d(sbase + L::OFF_K + pn * L::PANEL, &tm_k, bar(L::B_KV), 64 * pn, w.kb * 128, w.bh);
+        tma_load_3d(sbase + L::OFF_V + pn * L::PANEL, &tm_v, bar(L::B_KV), 64 * pn, w.kb * 128, w.bh);
+      }
+      int it = 0;
+      for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
+        const int s = it % L::STAGES;
+        const uint32_t ph = (it / L::STAGES) & 1u;
+        if (it >= L::STAGES && !mbar_wait(bar(L::B_QEMPTY + s), ph ^ 1u, g)) break;
+        mbar_arrive_expect_tx(bar(L::B_QFULL + s), 2 * L::TILE + 1024);
+        for (int pn = 0; pn < L::PANELS; ++pn) {
+          tma_load_3d(sbase + L::OFF_Q + s * L::TILE + pn * L::PANEL, &tm_q, bar(L::B_QFULL + s),
+                      64 * pn, qb * 128, w.bh);
+          tma_load_3d(sbase + L::OFF_DO + s * L::TILE + pn * L::PANEL, &tm_do, bar(L::B_QFULL + s),
+                      64 * pn, qb * 128, w.bh);
+        }
+        const size_t roff = static_cast<size_t>(w.bh) * p.Npad + static_cast<size_t>(qb) * 128;
+        bulk_load(sbase + L::OFF_LD + s * 1024, p.ws_lse2 + roff, 512, bar(L::B_QFULL + s));
+        bulk_load(sbase + L::OFF_LD + s * 1024 + 512, p.ws_delta + roff, 512, bar(L::B_QFULL + s));
+      }
+      if (*abort_flag) {
+        for (int j = max(0, it - L::STAGES); j < it; ++j)
+          mbar_wait_drain(bar(L::B_QFULL + j % L::STAGES), (j / L::STAGES) & 1u, 100000000ull);
+        mbar_wait_drain(bar(L::B_KV), 0, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0 && any_work) {
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t kIdKQ = idesc_bf16(128, D, false, true);  // dV, dK
+      constexpr uint32_t kIdQ = idesc_bf16(128, D, true, true);    // dQ
+      const uint32_t k_addr = sbase + L::OFF_K, v_addr = sbase + L::OFF_V;
+      const uint32_t ds_addr = sbase + L::OFF_DS;
+      bool ok = mbar_wait(bar(L::B_KV), 0, g);
+
+      auto issue_sdp = [&](int s, bool dp_only) {
+        const uint32_t q_addr = sbase + L::OFF_Q + s * L::TILE;
+        const uint32_t do_addr = sbase + L::OFF_DO + s * L::TILE;
+        if (!dp_only) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::PANEL + (kk & 3) * 32;
+            mma_ss(tmem + L::COL_S, sdesc_sw128(k_addr + off, 16, 1024),
+                   sdesc_sw128(q_addr + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::B_SFULL));
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::PANEL + (kk & 3) * 32;
+            mma_ss(tmem + L::COL_DP, sdesc_sw128(v_addr + off, 16, 1024),
+                   sdesc_sw128(do_addr + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::B_DPFULL));
+        }
+      };
+
+      int it = 0;
+      if (ok) ok = mbar_wait(bar(L::B_QFULL + 0), 0, g);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(0, false);
+        issue_sdp(0, true);
+      }
+      for (int qb = q_first; ok && qb < w.nqb; ++it) {
+        const int s = it % L::STAGES;
+        const int qbn = w.next(qb + 1);
+        if (!mbar_wait(bar(L::B_PFULL), it & 1u, g)) break;
+        tc_fence_after();
+        const uint32_t q_addr = sbase + L::OFF_Q + s * L::TILE;
+        const uint32_t do_addr = sbase + L::OFF_DO + s * L::TILE;
+        // dV += P^T dO   (A = P from TMEM, B = dO MN-major)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + L::COL_DV, tmem + L::COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
+                 sdesc_sw128(do_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q   (A = dS^T K-major in shared memory, B = Q MN-major)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::COL_DK, sdesc_sw128(ds_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(q_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        // dQ_tile = dS K   (A = dS MN-major, B = K MN-major), into the dP^T columns
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::COL_DP, sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024),
+                 sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024), kIdQ, kk > 0 ? 1u : 0u);
+        mma_commit(bar(L::B_DQFULL));
+        mma_commit(bar(L::B_DSEMPTY));
+        mma_commit(bar(L::B_QEMPTY + s));
+        if (qbn < w.nqb) {
+          const int sn = (it + 1) % L::STAGES;
+          if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
+          tc_fence_after();
+          issue_sdp(sn, false);
+          if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
+          tc_fence_after();
+          issue_sdp(sn, true);
+        }
+        qb = qbn;
+      }
+      mma_commit(bar(L::B_KVDONE));
+      mbar_wait_drain(bar(L::B_KVDONE), 0, 1000000000ull);
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------ P / dS warpgroups
+    const int wg = (warp - 4) >> 2;
+    const int wq = warp & 3;
+    const int j = wq * 32 + lane;  // key row within the tile
+    const int jg = w.kb * 128 + j;
+    const bool key_live = jg < w.kv_len;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    bool ok = true;
+    int it = 0;
+    for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
+      const int s = it % L::STAGES;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + s), (it / L::STAGES) & 1u, g));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL), it & 1u, g));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DPFULL), it & 1u, g));
+      if (ok && it > 0)
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DSEMPTY), (it - 1) & 1u, g));
+      if (!ok) break;
+      tc_fence_after();
+      const float* lse2 = reinterpret_cast<const float*>(smem + L::OFF_LD + s * 1024);
+      const float* dlt = lse2 + 128;
+      const bool diag = w.causal && qb == w.kb;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int qoff = 64 * wg + 32 * c;  // query offset within the tile
+        uint32_t sv[32], dv[32];
+        tmem_ld32<0>(lane_addr + L::COL_S + qoff, sv);
+        tmem_ld32<0>(lane_addr + L::COL_DP + qoff, dv);
+        tmem_wait_ld32<0>(sv);
+        tmem_wait_ld32<0>(dv);
+        uint32_t kw[4] = {0u, 0u, 0u, 0u};
+        if constexpr (DROPOUT) {
+          // Lane r of each group of four computes the block of query
+          // qoff + 4 g + r (four keys each); the four 32-bit masks are then
+          // exchanged so every lane holds the bits of its own key.
+          uint32_t own = 0u;
+          const uint32_t thr = p.drop_threshold;
+#pragma unroll
+          for (int gq = 0; gq < 8; ++gq) {
+            const uint32_t qg = static_cast<uint32_t>(qb * 128 + qoff + 4 * gq + (lane & 3));
+            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(jg >> 2), qg,
+                                              static_cast<uint32_t>(w.h), static_cast<uint32_t>(w.b),
+                                              p.seed_lo, p.seed_hi);
+            const uint32_t nib = (rnd.w0 >= thr ? 1u : 0u) | (rnd.w1 >= thr ? 2u : 0u) |
+                                 (rnd.w2 >= thr ? 4u : 0u) | (rnd.w3 >= thr ? 8u : 0u);
+            own |= nib << (4 * gq);
+          }
+#pragma unroll
+          for (int r = 0; r < 4; ++r) kw[r] = __shfl_sync(0xffffffffu, own, (lane & ~3) | r);
+        }
+        const float4* l4 = reinterpret_cast<const float4*>(lse2 + qoff);
+        const float4* d4 = reinterpret_cast<const float4*>(dlt + qoff);
+        uint32_t ppk[16], dpk[16];
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 lv = l4[k4];
+          const float4 dl = d4[k4];
+          const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+          const float dq[4] = {dl.x, dl.y, dl.z, dl.w};
+          float pe[4], ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = 4 * k4 + e;
+            float pv = fast_exp2(fmaf(__uint_as_float(sv[k]), p.scale_log2, -lq[e]));
+            if (!key_live || (diag && qoff + k < j)) pv = 0.f;
+            float dpv = __uint_as_float(dv[k]);
+            float pd = pv;
+            if constexpr (DROPOUT) {
+              // query qoff + k = qoff + 4 k4 + e: group k4, lane e of the quad
+              const bool keep = (kw[e] >> (4 * k4 + (lane & 3))) & 1u;
+              pd = keep ? pv : 0.f;
+              dpv = keep ? dpv * p.drop_rscale : 0.f;
+            }
+            pe[e] = pd;
+            ds[e] = pv * (dpv - dq[e]);
+          }
+          ppk[2 * k4] = pack_bf16(pe[0], pe[1]);
+          ppk[2 * k4 + 1] = pack_bf16(pe[2], pe[3]);
+          dpk[2 * k4] = pack_bf16(ds[0], ds[1]);
+          dpk[2 * k4 + 1] = pack_bf16(ds[2], ds[3]);
+        }
+        // P^T (bf16 pairs) into TMEM: queries [64 wg, 64 wg + 64) -> columns [64 wg, 64 wg + 32)
+        tmem_st16<0>(lane_addr + L::COL_S + 64 * wg + 16 * c, ppk);
+        // dS^T row j into the 128-byte-swizzled [keys][queries] buffer, panel wg
+        const uint32_t row_addr = sbase + L::OFF_DS + wg * L::PANEL + j * 128;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const uint32_t chunk = static_cast<uint32_t>(4 * c + ch) ^ static_cast<uint32_t>(j & 7);
+          st_shared_v4(row_addr + chunk * 16, dpk[4 * ch], dpk[4 * ch + 1], dpk[4 * ch + 2],
+                       dpk[4 * ch + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_PFULL));
+    }
+
+    // -------------------------------------------------- dK, dV epilogue
+    const int n_it = it;
+    if (ok && any_work) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_KVDONE), 0, g));
+    if (ok) {
+      tc_fence_after();
+      const bool row_ok = jg < p.N;
+      const size_t roff = (static_cast<size_t>(w.bh) * p.N + jg) * D;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = wg * (D / 2) + 32 * c;
+        uint32_t a[32], bk[32];
+        if (any_work && n_it > 0) {
+          tmem_ld32<0>(lane_addr + L::COL_DV + col, a);
+          tmem_ld32<0>(lane_addr + L::COL_DK + col, bk);
+          tmem_wait_ld32<0>(a);
+          tmem_wait_ld32<0>(bk);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) a[k] = bk[k] = 0u;
+        }
+        if (row_ok) {
+          uint4* dvp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + roff + col);
+          uint4* dkp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + roff + col);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint32_t vv[4], kk4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int x = 8 * k + 2 * e;
+              vv[e] = pack_bf16(__uint_as_float(a[x]) * p.drop_rscale,
+                                __uint_as_float(a[x + 1]) * p.drop_rscale);
+              kk4[e] = pack_bf16(__uint_as_float(bk[x]) * p.scale, __uint_as_float(bk[x + 1]) * p.scale);
+            }
+            dvp[k] = make_uint4(vv[0], vv[1], vv[2], vv[3]);
+            dkp[k] = make_uint4(kk4[0], kk4[1], kk4[2], kk4[3]);
+          }
+        }
+      }
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------- dQ reduction
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // query row within the tile
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    int it = 0;
+    for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL), it & 1u, g))) break;
+      tc_fence_after();
+      float* dst = p.ws_dq + (static_cast<size_t>(w.bh) * p.Npad + qb * 128 + r) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32<0>(lane_addr + L::COL_DP + 32 * c, a);
+        tmem_wait_ld32<0>(a);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          red_add_v4(dst + 32 * c + 4 * k, __uint_as_float(a[4 * k]), __uint_as_float(a[4 * k + 1]),
+                     __uint_as_float(a[4 * k + 2]), __uint_as_float(a[4 * k + 3]));
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::B_DQEMPTY));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool DROPOUT>
+cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+  using L = BwdLayout<D>;
+  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Npad;
+  {
+    const int64_t threads = rows * (D / 8);
+    bwd_pre_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    auto kern = bwd_main_kernel<D, DROPOUT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(L::SMEM));
+    if (e != cudaSuccess) return e;
+    dim3 grid((p.N + 127) / 128, p.B * p.H);
+    kern<<<grid, kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    const int64_t threads = static_cast<int64_t>(p.B) * p.H * p.N * (D / 8);
+    bwd_post_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+    return cudaGetLastError();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p,
+                       cudaStream_t stream) {
+  if (d == 64) return dropout ? launch_bwd_t<64, true>(tq, tk, tv, tdo, p, stream)
+                              : launch_bwd_t<64, false>(tq, tk, tv, tdo, p, stream);
+  if (d == 128) return dropout ? launch_bwd_t<128, true>(tq, tk, tv, tdo, p, stream)
+                               : launch_bwd_t<128, false>(tq, tk, tv, tdo, p, stream);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace fa

@@ -270,6 +270,19 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[NR
                : "memory");
 }
 
+#define FA_R16(p, a, o) FA_R8(p, a, o), FA_R8(p, a, o + 8)
+#define FA_REGLIST16_1 \
+  "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16}"
+
+// Issue a 16-column store from r[o .. o+15].
+template <int O, int NREG>
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[NREG]) {
+  static_assert(O + 16 <= NREG, "register window");
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], " FA_REGLIST16_1 ";" ::"r"(taddr),
+               FA_R16(FA_IN, r, O)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -285,6 +298,13 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
 }
 
 // Vector fp32 reduction-add into global memory (sm_90+).
