@@ -96,6 +96,26 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
                    uint64_t seed, const uint8_t* block_mask, void* workspace,
                    size_t workspace_bytes, void* stream);
 
+/* The three launches fa_bwd makes, exposed so that each can be timed or
+ * scheduled on its own.  Called in this order on one stream with the same
+ * workspace they are exactly fa_bwd.
+ *  fa_bwd_prepare: from o, lse, dout fills the workspace with D_i, the
+ *    log2-domain LSE (+inf where a row has no key, so its P is 0) and zeroed
+ *    dQ accumulators.  Reads the softmax statistics the forward saved.
+ *  fa_bwd_main: recomputes P block by block from those statistics (the
+ *    recomputation of the pages) and writes dk, dv (bf16) and the fp32 dQ
+ *    accumulators in the workspace.
+ *  fa_bwd_finish: dq = bf16(softmax_scale * accumulator). */
+fa_status_t fa_bwd_prepare(const void* o, const float* lse, const void* dout, int B, int H, int N,
+                           int d, void* workspace, size_t workspace_bytes, void* stream);
+fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dk,
+                        void* dv, int B, int H, int N, int d, float softmax_scale, int causal,
+                        const int32_t* seqlens, float dropout_p, uint64_t seed,
+                        const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
+                        void* stream);
+fa_status_t fa_bwd_finish(void* dq, int B, int H, int N, int d, float softmax_scale,
+                          const void* workspace, size_t workspace_bytes, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* fa_status_string(fa_status_t status);
 

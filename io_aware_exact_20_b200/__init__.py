@@ -20,7 +20,7 @@ import os
 from .build import LIB_PATH
 
 __all__ = [
-    "FaError", "library", "forward", "backward", "bwd_workspace_size",
+    "FaError", "library", "forward", "backward", "backward_phases", "bwd_workspace_size",
     "dropout_mask", "last_device_status", "set_wait_timeout_ns",
     "wait_timeout_probe", "STATUS",
 ]
@@ -51,6 +51,10 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
     "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _f, _u64, _vp, _vp, _sz, _vp]),
+    "fa_bwd_prepare": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "fa_bwd_main": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _f, _u64,
+                         _vp, _vp, _sz, _vp]),
+    "fa_bwd_finish": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_last_device_status": (_i, [_vp]),
     "fa_set_wait_timeout_ns": (None, [_u64]),
@@ -163,6 +167,44 @@ def backward(q, k, v, o, lse, dout, scale=None, causal=False, seqlens=None, drop
                             _stream_ptr(q.device))
     _check(code, "fa_bwd")
     return dq, dk, dv
+
+
+def backward_phases(q, k, v, o, lse, dout, scale=None, causal=False, seqlens=None,
+                    dropout_p=0.0, seed=0, block_mask=None, workspace=None, dq=None, dk=None,
+                    dv=None):
+    """The three launches of ``backward`` as three callables (prepare, main,
+    finish) bound to the same buffers, plus the outputs: lets a caller put
+    events or other work between them."""
+    import torch
+    _check_qkv(q, k, v, o, dout)
+    B, H, N, d = q.shape
+    scale = d ** -0.5 if scale is None else scale
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_size(B, H, N, d), dtype=torch.uint8,
+                                device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    sl, bm = _masks(seqlens, block_mask, q.device)
+    ws, nws = _ptr(workspace), workspace.numel() * workspace.element_size()
+    lib = library()
+    seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+
+    def prepare():
+        _check(lib.fa_bwd_prepare(_ptr(o), _ptr(lse), _ptr(dout), B, H, N, d, ws, nws,
+                                  _stream_ptr(q.device)), "fa_bwd_prepare")
+
+    def main():
+        _check(lib.fa_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dk), _ptr(dv), B, H,
+                               N, d, float(scale), int(bool(causal)), _ptr(sl),
+                               float(dropout_p), seed, _ptr(bm), ws, nws,
+                               _stream_ptr(q.device)), "fa_bwd_main")
+
+    def finish():
+        _check(lib.fa_bwd_finish(_ptr(dq), B, H, N, d, float(scale), ws, nws,
+                                 _stream_ptr(q.device)), "fa_bwd_finish")
+
+    return (prepare, main, finish), (dq, dk, dv), (sl, bm, workspace)
 
 
 def dropout_mask(B, H, N, dropout_p, seed, device="cuda"):

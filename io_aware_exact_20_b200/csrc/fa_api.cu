@@ -141,61 +141,122 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return static_cast<size_t>((bytes + 255) / 256 * 256);
 }
 
-fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                   const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-                   float softmax_scale, int causal, const int32_t* seqlens, float dropout_p,
-                   uint64_t seed, const uint8_t* block_mask, void* workspace,
-                   size_t workspace_bytes, void* stream) {
-  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(o) || !tensor_ok(dout) ||
-      !tensor_ok(dq) || !tensor_ok(dk) || !tensor_ok(dv))
-    return FA_ERR_INVALID_ARG;
-  if (lse == nullptr || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
-  if (seqlens != nullptr && !aligned(seqlens, 4)) return FA_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// Workspace views and scalar parameters shared by the three backward phases.
+fa_status_t bwd_params(fa::BwdParams* p, int B, int H, int N, int d, float softmax_scale,
+                       float dropout_p, const void* workspace, size_t workspace_bytes) {
   fa_status_t st = check_shape(B, H, N, d, softmax_scale, dropout_p);
   if (st != FA_OK) return st;
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need)
     return FA_ERR_WORKSPACE;
-
   int* status = status_word();
   if (status == nullptr) return FA_ERR_CUDA;
+  const Dropout dr = dropout_params(dropout_p);
+  const int64_t npad = padded_rows(N);
+  const uint64_t bh = static_cast<uint64_t>(B) * H;
+  *p = fa::BwdParams{};
+  p->ws_lse2 = static_cast<float*>(const_cast<void*>(workspace));
+  p->ws_delta = p->ws_lse2 + bh * npad;
+  p->ws_dq = p->ws_delta + bh * npad;
+  p->status = status;
+  p->B = B;
+  p->H = H;
+  p->N = N;
+  p->Npad = static_cast<int>(npad);
+  p->nblk = (N + 127) / 128;
+  p->scale = softmax_scale;
+  p->scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * kLog2e);
+  p->drop_threshold = dr.threshold;
+  p->drop_rscale = dr.rscale;
+  p->timeout_ns = g_timeout_ns;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status_t fa_bwd_prepare(const void* o, const float* lse, const void* dout, int B, int H, int N,
+                           int d, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!tensor_ok(o) || !tensor_ok(dout)) return FA_ERR_INVALID_ARG;
+  if (lse == nullptr || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  fa::BwdParams p;
+  // scale and dropout do not enter this phase: validate with neutral values
+  fa_status_t st = bwd_params(&p, B, H, N, d, 1.f, 0.f, workspace, workspace_bytes);
+  if (st != FA_OK) return st;
+  p.o = o;
+  p.lse = lse;
+  p.dout = dout;
+  return fa::launch_bwd_pre(d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK
+                                                                                     : FA_ERR_CUDA;
+}
+
+fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dk,
+                        void* dv, int B, int H, int N, int d, float softmax_scale, int causal,
+                        const int32_t* seqlens, float dropout_p, uint64_t seed,
+                        const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(dout) || !tensor_ok(dk) ||
+      !tensor_ok(dv))
+    return FA_ERR_INVALID_ARG;
+  if (seqlens != nullptr && !aligned(seqlens, 4)) return FA_ERR_INVALID_ARG;
+  fa::BwdParams p;
+  fa_status_t st =
+      bwd_params(&p, B, H, N, d, softmax_scale, dropout_p, workspace, workspace_bytes);
+  if (st != FA_OK) return st;
   CUtensorMap tq, tk, tv, tdo;
   const uint64_t bh = static_cast<uint64_t>(B) * H;
   if (!fa::make_tmap_bf16(&tq, q, d, N, bh, 128) || !fa::make_tmap_bf16(&tk, k, d, N, bh, 128) ||
       !fa::make_tmap_bf16(&tv, v, d, N, bh, 128) || !fa::make_tmap_bf16(&tdo, dout, d, N, bh, 128))
     return FA_ERR_CUDA;
-
-  const Dropout dr = dropout_params(dropout_p);
-  const int64_t npad = padded_rows(N);
-  fa::BwdParams p{};
-  p.o = o;
-  p.dout = dout;
-  p.lse = lse;
-  p.dq = dq;
   p.dk = dk;
   p.dv = dv;
-  p.ws_lse2 = static_cast<float*>(workspace);
-  p.ws_delta = p.ws_lse2 + bh * npad;
-  p.ws_dq = p.ws_delta + bh * npad;
   p.seqlens = seqlens;
   p.block_mask = block_mask;
-  p.status = status;
-  p.B = B;
-  p.H = H;
-  p.N = N;
-  p.Npad = static_cast<int>(npad);
-  p.nblk = (N + 127) / 128;
-  p.scale = softmax_scale;
-  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * kLog2e);
   p.causal = causal != 0;
-  p.drop_threshold = dr.threshold;
-  p.drop_rscale = dr.rscale;
   p.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
   p.seed_hi = static_cast<uint32_t>(seed >> 32);
-  p.timeout_ns = g_timeout_ns;
-  const cudaError_t e = fa::launch_bwd(d, dr.threshold != 0, tq, tk, tv, tdo, p,
-                                       static_cast<cudaStream_t>(stream));
+  const cudaError_t e = fa::launch_bwd_main(d, p.drop_threshold != 0, tq, tk, tv, tdo, p,
+                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status_t fa_bwd_finish(void* dq, int B, int H, int N, int d, float softmax_scale,
+                          const void* workspace, size_t workspace_bytes, void* stream) {
+  if (!tensor_ok(dq)) return FA_ERR_INVALID_ARG;
+  fa::BwdParams p;
+  fa_status_t st = bwd_params(&p, B, H, N, d, softmax_scale, 0.f, workspace, workspace_bytes);
+  if (st != FA_OK) return st;
+  p.dq = dq;
+  return fa::launch_bwd_post(d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK
+                                                                                     : FA_ERR_CUDA;
+}
+
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                   float softmax_scale, int causal, const int32_t* seqlens, float dropout_p,
+                   uint64_t seed, const uint8_t* block_mask, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  // validate everything before the first launch
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(o) || !tensor_ok(dout) ||
+      !tensor_ok(dq) || !tensor_ok(dk) || !tensor_ok(dv))
+    return FA_ERR_INVALID_ARG;
+  if (lse == nullptr || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  if (seqlens != nullptr && !aligned(seqlens, 4)) return FA_ERR_INVALID_ARG;
+  fa::BwdParams chk;
+  fa_status_t st =
+      bwd_params(&chk, B, H, N, d, softmax_scale, dropout_p, workspace, workspace_bytes);
+  if (st != FA_OK) return st;
+  st = fa_bwd_prepare(o, lse, dout, B, H, N, d, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  st = fa_bwd_main(q, k, v, dout, dk, dv, B, H, N, d, softmax_scale, causal, seqlens, dropout_p,
+                   seed, block_mask, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  return fa_bwd_finish(dq, B, H, N, d, softmax_scale, workspace, workspace_bytes, stream);
 }
 
 fa_status_t fa_debug_dropout_mask(uint8_t* keep, int B, int H, int N, float dropout_p,

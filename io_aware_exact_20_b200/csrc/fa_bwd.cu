@@ -505,43 +505,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+template <int D>
+cudaError_t launch_pre_t(const BwdParams& p, cudaStream_t stream) {
+  const int64_t threads = static_cast<int64_t>(p.B) * p.H * p.Npad * (D / 8);
+  bwd_pre_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <int D, bool DROPOUT>
-cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
   using L = BwdLayout<D>;
-  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Npad;
-  {
-    const int64_t threads = rows * (D / 8);
-    bwd_pre_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  {
-    auto kern = bwd_main_kernel<D, DROPOUT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(L::SMEM));
-    if (e != cudaSuccess) return e;
-    dim3 grid((p.N + 127) / 128, p.B * p.H);
-    kern<<<grid, kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  {
-    const int64_t threads = static_cast<int64_t>(p.B) * p.H * p.N * (D / 8);
-    bwd_post_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
-    return cudaGetLastError();
-  }
+  auto kern = bwd_main_kernel<D, DROPOUT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::SMEM));
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.N + 127) / 128, p.B * p.H);
+  kern<<<grid, kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_post_t(const BwdParams& p, cudaStream_t stream) {
+  const int64_t threads = static_cast<int64_t>(p.B) * p.H * p.N * (D / 8);
+  bwd_post_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_bwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
-                       const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p,
-                       cudaStream_t stream) {
-  if (d == 64) return dropout ? launch_bwd_t<64, true>(tq, tk, tv, tdo, p, stream)
-                              : launch_bwd_t<64, false>(tq, tk, tv, tdo, p, stream);
-  if (d == 128) return dropout ? launch_bwd_t<128, true>(tq, tk, tv, tdo, p, stream)
-                               : launch_bwd_t<128, false>(tq, tk, tv, tdo, p, stream);
+cudaError_t launch_bwd_pre(int d, const BwdParams& p, cudaStream_t stream) {
+  if (d == 64) return launch_pre_t<64>(p, stream);
+  if (d == 128) return launch_pre_t<128>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p,
+                            cudaStream_t stream) {
+  if (d == 64) return dropout ? launch_main_t<64, true>(tq, tk, tv, tdo, p, stream)
+                              : launch_main_t<64, false>(tq, tk, tv, tdo, p, stream);
+  if (d == 128) return dropout ? launch_main_t<128, true>(tq, tk, tv, tdo, p, stream)
+                               : launch_main_t<128, false>(tq, tk, tv, tdo, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_post(int d, const BwdParams& p, cudaStream_t stream) {
+  if (d == 64) return launch_post_t<64>(p, stream);
+  if (d == 128) return launch_post_t<128>(p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -52,9 +52,13 @@ struct BwdParams {
 cudaError_t launch_fwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, cudaStream_t stream);
 
-cudaError_t launch_bwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
-                       const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p,
-                       cudaStream_t stream);
+// Backward in three launches: D / log2-LSE / zeroed dQ accumulators, the main
+// kernel (dK, dV, dQ accumulators), and the dQ conversion.
+cudaError_t launch_bwd_pre(int d, const BwdParams& p, cudaStream_t stream);
+cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p,
+                            cudaStream_t stream);
+cudaError_t launch_bwd_post(int d, const BwdParams& p, cudaStream_t stream);
 
 cudaError_t launch_dropout_mask(uint8_t* keep, int B, int H, int N, uint32_t threshold,
                                 uint32_t seed_lo, uint32_t seed_hi, cudaStream_t stream);
