@@ -116,6 +116,28 @@ fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void*
 fa_status_t fa_bwd_finish(void* dq, int B, int H, int N, int d, float softmax_scale,
                           const void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward pass that allocates nothing (no counterpart in the paper: an
+ * interface convenience of this library).  For callers that cannot allocate
+ * device memory, for example code inside an allocator or memory-pool callback
+ * that must not re-enter the allocator, or a host application that reserves
+ * all device memory up front: same arguments and results as fa_bwd without
+ * the workspace, which instead lives in a fixed 64 MiB device array inside
+ * the library (held on every device that loads it until the process exits).
+ *  - Returns FA_ERR_WORKSPACE, launching nothing, when
+ *    fa_bwd_workspace_size(B,H,N,d) exceeds 64 MiB (67108864 bytes).
+ *  - The first call on a device looks the array's address up with
+ *    cudaGetSymbolAddress; make that first call before any stream capture.
+ *  - All calls on a device share the array and it keeps the last call's
+ *    contents; each call rewrites everything that must start at zero before
+ *    using it.  Calls whose kernels overlap on the GPU (unordered streams)
+ *    race on the array: issue them on one stream or otherwise serialise them.
+ *  - Calls no cudaMalloc, cudaFree or other allocating routine. */
+fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                           int H, int N, int d, float softmax_scale, int causal,
+                           const int32_t* seqlens, float dropout_p, uint64_t seed,
+                           const uint8_t* block_mask, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* fa_status_string(fa_status_t status);
 

@@ -55,6 +55,8 @@ SIGNATURES = {
     "fa_bwd_main": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _f, _u64,
                          _vp, _vp, _sz, _vp]),
     "fa_bwd_finish": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
+    "fa_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
+                            _vp, _f, _u64, _vp, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_last_device_status": (_i, [_vp]),
     "fa_set_wait_timeout_ns": (None, [_u64]),
