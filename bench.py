@@ -53,6 +53,10 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt2")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (profiling / scaling studies)")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="override the workload's sequence length (profiling / scaling studies)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="bound on the CPU-oracle sample timed beside the GPU run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -229,11 +233,47 @@ def time_oracle_heads(w, inp, seconds=None, heads=None):
 # reference arm: the oracle as it stands, on the host cores
 # ---------------------------------------------------------------------------
 
+def selected_workload(args):
+    from dataclasses import replace
+    w = WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = replace(w, B=args.batch)
+    if args.seqlen is not None:
+        lens = w.seqlen_range
+        if lens is not None:
+            lens = (min(lens[0], args.seqlen), min(lens[1], args.seqlen))
+        w = replace(w, N=args.seqlen, seqlen_range=lens)
+    return w
+
+
+def rank_workload(w, rank):
+    """The workload one rank runs: the same shape, its own batch of data (the
+    data seed is shifted by the rank), so ranks share no (b, h) problem."""
+    from dataclasses import replace
+    return replace(w, data_seed=w.data_seed + 7919 * rank)
+
+
+def max_over_ranks(x, world, device):
+    """Largest value of x over all ranks (the whole job ends with the slowest)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, flops_per_step, steps, total_ms):
+    """Whole-job TFLOP/s: every rank ran `steps` steps of `flops_per_step`."""
+    return world * flops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = WORKLOADS[args.workload]
+    w = selected_workload(args)
     inp = make_inputs(w, B=1)
     heads = [(0, h % w.H) for h in range(max(1, args.warmup + args.steps))]
     for i in range(args.warmup):
@@ -278,11 +318,8 @@ def run_ours(args):
 
     import io_aware_exact_20_b200 as fa
 
-    w = WORKLOADS[args.workload]
-    # each rank gets its own batch: the data seed is shifted by the rank
-    from dataclasses import replace
-    wr = replace(w, data_seed=w.data_seed + 7919 * rank)
-    inp = make_inputs(wr)
+    w = selected_workload(args)
+    inp = make_inputs(rank_workload(w, rank))
     q, k, v, do = (inp[x].to(dev) for x in ("q", "k", "v", "do"))
     B, H, N, d = q.shape
     kw = dict(scale=w.scale, causal=w.causal, seqlens=inp["seqlens"], dropout_p=w.dropout_p,
@@ -337,14 +374,10 @@ def run_ours(args):
     pre_ms = [e[1].elapsed_time(e[2]) for e in events]
     main_ms = [e[2].elapsed_time(e[3]) for e in events]
     post_ms = [e[3].elapsed_time(e[4]) for e in events]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
 
     f_fwd, f_bwd = attention_flops(B, H, N, d, w.causal)
-    value = world * (f_fwd + f_bwd) * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput(world, f_fwd + f_bwd, args.steps, total_ms)
     peaks, peak_src = read_peaks()
     peak = float(peaks["bf16_tflops"])
     fwd_avg, main_avg = statistics.mean(fwd_ms), statistics.mean(main_ms)
@@ -400,13 +433,9 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-        e_ms = sum(a.elapsed_time(b) for a, b in ev)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dev)
         nb = q.numel() * q.element_size()
-        e2e = {"value": world * (f_fwd + f_bwd) * n_e2e / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_throughput(world, f_fwd + f_bwd, n_e2e, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": 4 * nb,
                "d2h_bytes_per_step": 4 * nb + lse.numel() * lse.element_size(),
                "steps": n_e2e, "ms_per_step": e_ms / n_e2e}

@@ -128,6 +128,7 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
   p.drop_rscale = dr.rscale;
   p.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
   p.seed_hi = static_cast<uint32_t>(seed >> 32);
+  p.rk = fa::philox_round_keys(seed);
   p.timeout_ns = g_timeout_ns;
   const cudaError_t e =
       fa::launch_fwd(d, dr.threshold != 0, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
@@ -220,6 +221,7 @@ fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void*
   p.causal = causal != 0;
   p.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
   p.seed_hi = static_cast<uint32_t>(seed >> 32);
+  p.rk = fa::philox_round_keys(seed);
   const cudaError_t e = fa::launch_bwd_main(d, p.drop_threshold != 0, tq, tk, tv, tdo, p,
                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;

@@ -26,8 +26,9 @@
 //   warps 12-15   dQ warpgroup, thread = query row: TMEM -> red.global.add
 //
 // TMEM columns: S^T [0,128) with P packed into [64 w, 64 w + 32) per
-// warpgroup; dP^T [128,256), reused for the dQ tile once dP^T is consumed;
-// dV [256, 256 + D); dK [256 + D, 256 + 2 D).
+// warpgroup; dP^T [128,256); dV [256, 256 + D); dK [256 + D, 256 + 2 D); the
+// dQ tile in [384, 448) for d = 64, in the dP^T columns for d = 128 (after
+// dP^T has been consumed).
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -67,6 +68,10 @@ struct BwdLayout {
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+  // d = 64 leaves room for a dQ tile of its own; d = 128 reuses the dP^T
+  // columns once dP^T has been consumed.
+  static constexpr bool SEPARATE_DQ = (COL_DK + D + D <= 512);
+  static constexpr uint32_t COL_DQ = SEPARATE_DQ ? COL_DK + D : COL_DP;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(COL_DK + D <= 512, "TMEM budget");
 };
@@ -312,10 +317,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_ss(tmem + L::COL_DK, sdesc_sw128(ds_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024),
                  sdesc_sw128(q_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
                  (it > 0 || kk > 0) ? 1u : 0u);
-        // dQ_tile = dS K   (A = dS MN-major, B = K MN-major), into the dP^T columns
+        // dQ_tile = dS K   (A = dS MN-major, B = K MN-major)
+        if (L::SEPARATE_DQ && it > 0) {
+          // the dQ columns must have been drained by the previous iteration
+          if (!mbar_wait(bar(L::B_DQEMPTY), (it - 1) & 1u, g)) break;
+          tc_fence_after();
+        }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::COL_DP, sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024),
+          mma_ss(tmem + L::COL_DQ, sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024),
                  sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024), kIdQ, kk > 0 ? 1u : 0u);
         mma_commit(bar(L::B_DQFULL));
         mma_commit(bar(L::B_DSEMPTY));
@@ -325,8 +335,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
           tc_fence_after();
           issue_sdp(sn, false);
-          if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
-          tc_fence_after();
+          if (!L::SEPARATE_DQ) {
+            if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
+            tc_fence_after();
+          }
           issue_sdp(sn, true);
         }
         qb = qbn;
@@ -346,6 +358,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     int it = 0;
     for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
       const int s = it % L::STAGES;
+      // Dropout keep bits of this key for the warpgroup's 64 queries, drawn
+      // before the waits (they do not depend on S or dP).  Lane r of each group
+      // of four computes the block of query q0 + 4 g + r (four keys each); the
+      // four masks are then exchanged so every lane holds its own key's bits:
+      // keep(query qoff + 4 g + r) = bit (4 g + lane % 4) of kw[c][r].
+      uint32_t kw[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+      if constexpr (DROPOUT) {
+        const uint32_t thr = p.drop_threshold;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int qoff = 64 * wg + 32 * c;
+          uint32_t own = 0u;
+#pragma unroll
+          for (int gq = 0; gq < 8; ++gq) {
+            const uint32_t qg = static_cast<uint32_t>(qb * 128 + qoff + 4 * gq + (lane & 3));
+            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(jg >> 2), qg,
+                                              static_cast<uint32_t>(w.h), static_cast<uint32_t>(w.b),
+                                              p.rk);
+            const uint32_t nib = (rnd.w0 >= thr ? 1u : 0u) | (rnd.w1 >= thr ? 2u : 0u) |
+                                 (rnd.w2 >= thr ? 4u : 0u) | (rnd.w3 >= thr ? 8u : 0u);
+            own |= nib << (4 * gq);
+          }
+#pragma unroll
+          for (int r = 0; r < 4; ++r) kw[c][r] = __shfl_sync(0xffffffffu, own, (lane & ~3) | r);
+        }
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + s), (it / L::STAGES) & 1u, g));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL), it & 1u, g));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DPFULL), it & 1u, g));
@@ -364,26 +402,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32<0>(lane_addr + L::COL_DP + qoff, dv);
         tmem_wait_ld32<0>(sv);
         tmem_wait_ld32<0>(dv);
-        uint32_t kw[4] = {0u, 0u, 0u, 0u};
-        if constexpr (DROPOUT) {
-          // Lane r of each group of four computes the block of query
-          // qoff + 4 g + r (four keys each); the four 32-bit masks are then
-          // exchanged so every lane holds the bits of its own key.
-          uint32_t own = 0u;
-          const uint32_t thr = p.drop_threshold;
-#pragma unroll
-          for (int gq = 0; gq < 8; ++gq) {
-            const uint32_t qg = static_cast<uint32_t>(qb * 128 + qoff + 4 * gq + (lane & 3));
-            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(jg >> 2), qg,
-                                              static_cast<uint32_t>(w.h), static_cast<uint32_t>(w.b),
-                                              p.seed_lo, p.seed_hi);
-            const uint32_t nib = (rnd.w0 >= thr ? 1u : 0u) | (rnd.w1 >= thr ? 2u : 0u) |
-                                 (rnd.w2 >= thr ? 4u : 0u) | (rnd.w3 >= thr ? 8u : 0u);
-            own |= nib << (4 * gq);
-          }
-#pragma unroll
-          for (int r = 0; r < 4; ++r) kw[r] = __shfl_sync(0xffffffffu, own, (lane & ~3) | r);
-        }
         const float4* l4 = reinterpret_cast<const float4*>(lse2 + qoff);
         const float4* d4 = reinterpret_cast<const float4*>(dlt + qoff);
         uint32_t ppk[16], dpk[16];
@@ -403,7 +421,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             float pd = pv;
             if constexpr (DROPOUT) {
               // query qoff + k = qoff + 4 k4 + e: group k4, lane e of the quad
-              const bool keep = (kw[e] >> (4 * k4 + (lane & 3))) & 1u;
+              const bool keep = (kw[c][e] >> (4 * k4 + (lane & 3))) & 1u;
               pd = keep ? pv : 0.f;
               dpv = keep ? dpv * p.drop_rscale : 0.f;
             }
@@ -484,7 +502,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t a[32];
-        tmem_ld32<0>(lane_addr + L::COL_DP + 32 * c, a);
+        tmem_ld32<0>(lane_addr + L::COL_DQ + 32 * c, a);
         tmem_wait_ld32<0>(a);
 #pragma unroll
         for (int k = 0; k < 8; ++k)

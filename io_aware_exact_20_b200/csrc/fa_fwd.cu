@@ -294,6 +294,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = true;
       for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1)) {
         if (!w.act(t, kb)) continue;
+        // Dropout keep bits of this row for keys [128 kb, 128 kb + 128): they do
+        // not depend on S, so they are drawn while the Q K^T MMA runs.
+        uint32_t keepw[4] = {0u, 0u, 0u, 0u};
+        if constexpr (DROPOUT) {
+          const uint32_t thr = p.drop_threshold;
+#pragma unroll
+          for (int gq = 0; gq < 32; ++gq) {
+            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(kb * 32 + gq),
+                                              static_cast<uint32_t>(i), static_cast<uint32_t>(w.h),
+                                              static_cast<uint32_t>(w.b), p.rk);
+            const uint32_t nib = (rnd.w0 >= thr ? 1u : 0u) | (rnd.w1 >= thr ? 2u : 0u) |
+                                 (rnd.w2 >= thr ? 4u : 0u) | (rnd.w3 >= thr ? 8u : 0u);
+            keepw[gq >> 3] |= nib << (4 * (gq & 7));
+          }
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + t), cnt & 1u, g));
         if (!ok) break;
         tc_fence_after();
@@ -340,17 +355,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m = m_new;
 
         if constexpr (DROPOUT) {
-          const uint32_t thr = p.drop_threshold;
 #pragma unroll
-          for (int gq = 0; gq < 32; ++gq) {
-            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(kb * 32 + gq),
-                                              static_cast<uint32_t>(i), static_cast<uint32_t>(w.h),
-                                              static_cast<uint32_t>(w.b), p.seed_lo, p.seed_hi);
-            if (rnd.w0 < thr) sr[4 * gq + 0] = 0u;
-            if (rnd.w1 < thr) sr[4 * gq + 1] = 0u;
-            if (rnd.w2 < thr) sr[4 * gq + 2] = 0u;
-            if (rnd.w3 < thr) sr[4 * gq + 3] = 0u;
-          }
+          for (int j = 0; j < 128; ++j)
+            if (((keepw[j >> 5] >> (j & 31)) & 1u) == 0u) sr[j] = 0u;
         }
 
         uint32_t pk[64];

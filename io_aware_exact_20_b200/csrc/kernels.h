@@ -6,6 +6,8 @@
 
 #include <cstdint>
 
+#include "philox.cuh"
+
 namespace fa {
 
 // Device status codes written to the per-device status word.
@@ -23,6 +25,7 @@ struct FwdParams {
   uint32_t drop_threshold;    // keep iff word >= threshold
   float drop_rscale;          // 1 / (1 - p)
   uint32_t seed_lo, seed_hi;
+  PhiloxRoundKeys rk;         // round keys of the dropout generator
   uint64_t timeout_ns;
 };
 
@@ -46,6 +49,7 @@ struct BwdParams {
   uint32_t drop_threshold;
   float drop_rscale;
   uint32_t seed_lo, seed_hi;
+  PhiloxRoundKeys rk;
   uint64_t timeout_ns;
 };
 

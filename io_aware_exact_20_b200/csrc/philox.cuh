@@ -39,4 +39,44 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
   return Philox4{c0, c1, c2, c3};
 }
 
+// Round keys (k0 + r W0, k1 + r W1) for r = 0..9, computed once on the host
+// and read from the kernel parameters, so that each round is two 32x32->64
+// multiplies and two three-input xors.
+struct PhiloxRoundKeys {
+  uint32_t k0[10];
+  uint32_t k1[10];
+};
+
+__device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                 uint32_t c3, const PhiloxRoundKeys& rk) {
+  constexpr uint32_t kMul0 = 0xD2511F53u, kMul1 = 0xCD9E8D57u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = static_cast<uint64_t>(c0) * kMul0;
+    const uint64_t p1 = static_cast<uint64_t>(c2) * kMul1;
+    const uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+    const uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
+    const uint32_t n0 = hi1 ^ c1 ^ rk.k0[r];
+    const uint32_t n2 = hi0 ^ c3 ^ rk.k1[r];
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return Philox4{c0, c1, c2, c3};
+}
+
+// Host-side round keys for a 64-bit seed.
+inline PhiloxRoundKeys philox_round_keys(uint64_t seed) {
+  PhiloxRoundKeys rk;
+  uint32_t k0 = static_cast<uint32_t>(seed & 0xFFFFFFFFull), k1 = static_cast<uint32_t>(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    rk.k0[r] = k0;
+    rk.k1[r] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return rk;
+}
+
 }  // namespace fa

@@ -12,6 +12,9 @@ from .attention_ref import (  # noqa: F401
     dropout_keep,
     dropout_threshold,
     head_backward,
+    head_backward_cols,
+    head_backward_rows,
+    head_forward_rows,
     safe_softmax,
     valid_mask,
 )

@@ -222,3 +222,74 @@ def attention_backward(q, k, v, dout, scale, causal=False, seqlens=None,
         dq[b, h], dk[b, h], dv[b, h] = g[0], g[1], g[2]
     return dq, dk, dv
 
+
+
+# ----------------------------------------------------------------------------
+# sampled backward, for checking full-size runs output by output
+# ----------------------------------------------------------------------------
+
+def _row_terms(q, k, v, dout, scale, rows, causal, kv_len, block_mask, keep, dropout_p):
+    """P, the dropped P, and dS of the given query rows (each row needs only its
+    own row of S, of dP = dO V^T and its own D_i)."""
+    n = k.shape[0]
+    s = scale * (q[rows] @ k.T)
+    valid = valid_mask(n, rows, causal, kv_len, block_mask)
+    p, _, _, _ = safe_softmax(s, valid)
+    p32 = float(np.float32(dropout_p))
+    if keep is None or p32 == 0:
+        z, rscale = 1.0, 1.0
+    else:
+        z, rscale = keep.astype(np.float64), 1.0 / (1.0 - p32)
+    pd = p * z * rscale
+    dp = (dout[rows] @ v.T) * z * rscale
+    dsum = (p * dp).sum(axis=1)
+    ds = p * (dp - dsum[:, None])
+    return pd, ds
+
+
+def head_forward_rows(q, k, v, scale, rows, causal=False, kv_len=None, block_mask=None,
+                      dropout_p=0.0, seed=0, b=0, h=0):
+    """O and LSE of the given query rows of one (b, h) (q, k, v: [N, d])."""
+    rows = np.asarray(rows, dtype=np.int64)
+    p32 = float(np.float32(dropout_p))
+    keep, rscale = None, 1.0
+    if p32 > 0:
+        keep = dropout_keep(seed, p32, b, h, rows, k.shape[0])
+        rscale = 1.0 / (1.0 - p32)
+    return _head_forward(q, k, v, scale, rows, causal, kv_len, block_mask, keep, rscale)
+
+
+def head_backward_rows(q, k, v, dout, scale, rows, causal=False, kv_len=None,
+                       block_mask=None, dropout_p=0.0, seed=0, b=0, h=0):
+    """dQ of the given query rows of one (b, h): scale * dS[rows] K."""
+    rows = np.asarray(rows, dtype=np.int64)
+    p32 = float(np.float32(dropout_p))
+    keep = dropout_keep(seed, p32, b, h, rows, k.shape[0]) if p32 > 0 else None
+    _, ds = _row_terms(q, k, v, dout, scale, rows, causal, kv_len, block_mask, keep, p32)
+    return scale * (ds @ k)
+
+
+def head_backward_cols(q, k, v, dout, scale, cols, causal=False, kv_len=None,
+                       block_mask=None, dropout_p=0.0, seed=0, b=0, h=0, slab=256,
+                       rows=None):
+    """dK and dV of the given key columns of one (b, h).
+
+    Both are sums over query rows (dV_j = sum_i Pdrop_ij dO_i,
+    dK_j = scale sum_i dS_ij Q_i); the rows are visited in slabs of ``slab``
+    only to bound memory.  ``rows`` (default: all) limits the sum to a subset
+    of query rows; it is only correct when every left-out row has P_ij = 0 for
+    all the requested columns (e.g. rows whose blocks the block mask removes).
+    """
+    cols = np.asarray(cols, dtype=np.int64)
+    n, d = k.shape
+    p32 = float(np.float32(dropout_p))
+    dk = np.zeros((cols.size, d))
+    dv = np.zeros((cols.size, d))
+    all_rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
+    for r0 in range(0, all_rows.size, slab):
+        rows = all_rows[r0:r0 + slab]
+        keep = dropout_keep(seed, p32, b, h, rows, n) if p32 > 0 else None
+        pd, ds = _row_terms(q, k, v, dout, scale, rows, causal, kv_len, block_mask, keep, p32)
+        dv += pd[:, cols].T @ dout[rows]
+        dk += scale * (ds[:, cols].T @ q[rows])
+    return dk, dv

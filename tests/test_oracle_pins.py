@@ -428,3 +428,81 @@ def test_zero_q_gives_closed_form_dv():
         for j in np.nonzero(valid[i])[0]:
             want[j] += do[i] / n[i]
     assert np.abs(dv - want).max() < 1e-12
+
+
+@pytest.mark.parametrize("mode", MASK_MODES)
+def test_sampled_backward_matches_torch_autograd(mode):
+    """The row- and column-sampled backward (used to check full-size runs)
+    against torch autograd through SDPA, with the same masks, no dropout."""
+    import torch
+
+    from oracle import head_backward_cols, head_backward_rows, head_forward_rows
+
+    rng = np.random.default_rng(31)
+    B, N, d = 1, 300, 8
+    causal, seqlens, block = _mask_args(mode, B, N, rng)
+    kv = None if seqlens is None else int(seqlens[0])
+    q, k, v, do = (_rand((N, d), rng) for _ in range(4))
+    mask = valid_mask(N, np.arange(N), causal, kv, block)
+    has = mask.any(axis=1)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(
+        tq[None], tk[None], tv[None], attn_mask=torch.tensor(mask)[None], scale=0.3)[0]
+    to = torch.where(torch.tensor(has)[:, None], to, torch.zeros_like(to))
+    (to * torch.tensor(do)).sum().backward()
+    rows = np.array([0, 5, 127, 128, 299])
+    cols = np.array([0, 3, 128, 250, 299])
+    dq = head_backward_rows(q, k, v, do, 0.3, rows, causal, kv, block)
+    dk, dv = head_backward_cols(q, k, v, do, 0.3, cols, causal, kv, block, slab=64)
+    o_rows, _ = head_forward_rows(q, k, v, 0.3, rows, causal, kv, block)
+    assert np.abs(o_rows - to.detach().numpy()[rows]).max() < 1e-12
+    assert np.abs(dq - tq.grad.numpy()[rows]).max() < 1e-10
+    assert np.abs(dk - tk.grad.numpy()[cols]).max() < 1e-10
+    assert np.abs(dv - tv.grad.numpy()[cols]).max() < 1e-10
+
+
+def test_sampled_forward_rows_use_the_head_own_dropout_bits():
+    """head_forward_rows(b, h) equals the (b, h) slice of the batched forward."""
+    from oracle import head_forward_rows
+
+    rng = np.random.default_rng(33)
+    q, k, v = (_rand((2, 3, 140, 4), rng) for _ in range(3))
+    o, lse = attention_forward(q, k, v, 0.4, True, dropout_p=0.2, seed=5)
+    rows = np.array([0, 64, 139])
+    for b, h in ((0, 0), (1, 2)):
+        ro, rl = head_forward_rows(q[b, h], k[b, h], v[b, h], 0.4, rows, True,
+                                   dropout_p=0.2, seed=5, b=b, h=h)
+        assert np.abs(ro - o[b, h][rows]).max() < 1e-12
+        assert np.abs(rl - lse[b, h][rows]).max() < 1e-12
+
+
+def test_sampled_backward_with_dropout_matches_finite_differences():
+    """With dropout (bits fixed by the seed), sampled dQ rows and dK / dV
+    columns against central differences of L = sum(O * dO)."""
+    from oracle import head_backward_cols, head_backward_rows
+
+    rng = np.random.default_rng(32)
+    N, d, p, seed = 12, 4, 0.3, 77
+    q, k, v, do = (_rand((1, 1, N, d), rng) for _ in range(4))
+
+    def loss(q_, k_, v_):
+        o, _ = attention_forward(q_, k_, v_, 0.5, True, None, p, seed)
+        return float((o * do).sum())
+
+    eps = 1e-6
+    rows, cols = np.array([1, 7, 11]), np.array([0, 6, 10])
+    dq = head_backward_rows(q[0, 0], k[0, 0], v[0, 0], do[0, 0], 0.5, rows, True,
+                            dropout_p=p, seed=seed)
+    dk, dv = head_backward_cols(q[0, 0], k[0, 0], v[0, 0], do[0, 0], 0.5, cols, True,
+                                dropout_p=p, seed=seed, slab=5)
+    for name, x, sel, g in (("q", q, rows, dq), ("k", k, cols, dk), ("v", v, cols, dv)):
+        num = np.zeros((sel.size, d))
+        for a, r in enumerate(sel):
+            for c in range(d):
+                xp, xm = x.copy(), x.copy()
+                xp[0, 0, r, c] += eps
+                xm[0, 0, r, c] -= eps
+                args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+                args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+                num[a, c] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        assert np.linalg.norm(num - g) / np.linalg.norm(num) < 1e-6, name
