@@ -27,8 +27,8 @@
 //
 // TMEM columns: S^T [0,128) with P packed into [64 w, 64 w + 32) per
 // warpgroup; dP^T [128,256); dV [256, 256 + D); dK [256 + D, 256 + 2 D); the
-// dQ tile in [384, 448) for d = 64, in the dP^T columns for d = 128 (after
-// dP^T has been consumed).
+// dQ tile in [384, 448) for d = 64; for d = 128 its transpose dQ^T (lane =
+// feature, column = query) in the dP^T columns once dP^T has been consumed.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -72,6 +72,10 @@ struct BwdLayout {
   // columns once dP^T has been consumed.
   static constexpr bool SEPARATE_DQ = (COL_DK + D + D <= 512);
   static constexpr uint32_t COL_DQ = SEPARATE_DQ ? COL_DK + D : COL_DP;
+  // d = 128: the dQ tile is computed transposed (dQ^T = K^T dS^T, TMEM lane =
+  // feature c, column = query) so that each warp's reduction into the fp32
+  // accumulators covers 32 consecutive floats of one row: one 128-byte line.
+  static constexpr bool DQ_T = (D == 128);
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(COL_DK + D <= 512, "TMEM budget");
 };
@@ -182,8 +186,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
 
   BwdWork w;
-  w.kb = blockIdx.x;
-  w.bh = blockIdx.y;
+  w.kb = static_cast<int>(p.tiles_major ? blockIdx.y : blockIdx.x);  // key tile 0 is heaviest
+  w.bh = static_cast<int>(p.tiles_major ? blockIdx.x : blockIdx.y);
   w.b = w.bh / p.H;
   w.h = w.bh % p.H;
   {
@@ -264,7 +268,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0 && any_work) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t kIdKQ = idesc_bf16(128, D, false, true);  // dV, dK
-      constexpr uint32_t kIdQ = idesc_bf16(128, D, true, true);    // dQ
+      constexpr uint32_t kIdQ = L::DQ_T ? idesc_bf16(D, 128, true, true)   // dQ^T
+                                        : idesc_bf16(128, D, true, true);  // dQ
       const uint32_t k_addr = sbase + L::OFF_K, v_addr = sbase + L::OFF_V;
       const uint32_t ds_addr = sbase + L::OFF_DS;
       bool ok = mbar_wait(bar(L::B_KV), 0, g);
@@ -324,9 +329,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
         }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::COL_DQ, sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024),
-                 sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024), kIdQ, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ds_desc = sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024);
+          const uint64_t k_desc = sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024);
+          if constexpr (L::DQ_T)  // dQ^T = K^T dS^T: A = K^T (MN-major), B = dS^T (MN-major)
+            mma_ss(tmem + L::COL_DQ, k_desc, ds_desc, kIdQ, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tmem + L::COL_DQ, ds_desc, k_desc, kIdQ, kk > 0 ? 1u : 0u);
+        }
         mma_commit(bar(L::B_DQFULL));
         mma_commit(bar(L::B_DSEMPTY));
         mma_commit(bar(L::B_QEMPTY + s));
@@ -498,16 +508,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL), it & 1u, g))) break;
       tc_fence_after();
-      float* dst = p.ws_dq + (static_cast<size_t>(w.bh) * p.Npad + qb * 128 + r) * D;
+      if constexpr (L::DQ_T) {
+        // lane r = feature r; column c = query qb * 128 + c
+        float* dst = p.ws_dq + (static_cast<size_t>(w.bh) * p.Npad + qb * 128) * D + r;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t a[32];
-        tmem_ld32<0>(lane_addr + L::COL_DQ + 32 * c, a);
-        tmem_wait_ld32<0>(a);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t a[32];
+          tmem_ld32<0>(lane_addr + L::COL_DQ + 32 * c, a);
+          tmem_wait_ld32<0>(a);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          red_add_v4(dst + 32 * c + 4 * k, __uint_as_float(a[4 * k]), __uint_as_float(a[4 * k + 1]),
-                     __uint_as_float(a[4 * k + 2]), __uint_as_float(a[4 * k + 3]));
+          for (int k = 0; k < 32; ++k) red_add_f32(dst + (32 * c + k) * D, __uint_as_float(a[k]));
+        }
+      } else {
+        float* dst = p.ws_dq + (static_cast<size_t>(w.bh) * p.Npad + qb * 128 + r) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32<0>(lane_addr + L::COL_DQ + 32 * c, a);
+          tmem_wait_ld32<0>(a);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            red_add_v4(dst + 32 * c + 4 * k, __uint_as_float(a[4 * k]), __uint_as_float(a[4 * k + 1]),
+                       __uint_as_float(a[4 * k + 2]), __uint_as_float(a[4 * k + 3]));
+        }
       }
       tc_fence_before();
       mbar_arrive(bar(L::B_DQEMPTY));
@@ -538,7 +561,8 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::SMEM));
   if (e != cudaSuccess) return e;
-  dim3 grid((p.N + 127) / 128, p.B * p.H);
+  const unsigned tiles = static_cast<unsigned>((p.N + 127) / 128), bh = static_cast<unsigned>(p.B * p.H);
+  const dim3 grid = p.tiles_major ? dim3(bh, tiles) : dim3(tiles, bh);
   kern<<<grid, kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError();
 }

@@ -106,10 +106,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   FwdWork w;
   {
     const int nqp = (p.N + 255) / 256;
-    const int qp = nqp - 1 - static_cast<int>(blockIdx.x);  // heaviest causal rows first
+    const int tile = static_cast<int>(p.tiles_major ? blockIdx.y : blockIdx.x);
+    const int qp = nqp - 1 - tile;  // heaviest causal rows first
     w.q0 = qp * 256;
     w.qb0 = qp * 2;
-    w.bh = blockIdx.y;
+    w.bh = static_cast<int>(p.tiles_major ? blockIdx.x : blockIdx.y);
     w.b = w.bh / p.H;
     w.h = w.bh % p.H;
     w.exists1 = (w.q0 + 128) < p.N;
@@ -443,7 +444,8 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::SMEM));
   if (e != cudaSuccess) return e;
-  dim3 grid((p.N + 255) / 256, p.B * p.H);
+  const unsigned tiles = static_cast<unsigned>((p.N + 255) / 256), bh = static_cast<unsigned>(p.B * p.H);
+  const dim3 grid = p.tiles_major ? dim3(bh, tiles) : dim3(tiles, bh);
   kern<<<grid, kFwdThreads, L::SMEM, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }

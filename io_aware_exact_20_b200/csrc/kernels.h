@@ -10,6 +10,16 @@
 
 namespace fa {
 
+// Grid order.  When every head's K and V fit in L2 many times over, the grid
+// puts the tile index slowest so that all heads' heaviest tiles (most K/V
+// tiles under a causal mask) start first (longest-processing-time order);
+// otherwise it is head-major so that the CTAs resident at one time share few
+// heads and each head's K/V stays in L2.
+inline bool tiles_major_order(int B, int H, int N, int d) {
+  const double kv_bytes = 4.0 * B * H * static_cast<double>(N) * d;  // K and V, bf16
+  return kv_bytes <= 48.0 * 1024 * 1024;
+}
+
 // Device status codes written to the per-device status word.
 enum : int { kStatusOk = 0, kStatusInternal = 3, kStatusTimeout = 4 };
 
@@ -22,6 +32,7 @@ struct FwdParams {
   int B, H, N, nblk;
   float scale_log2;           // softmax_scale * log2(e)
   int causal;
+  int tiles_major;            // grid is (B*H, tiles) instead of (tiles, B*H)
   uint32_t drop_threshold;    // keep iff word >= threshold
   float drop_rscale;          // 1 / (1 - p)
   uint32_t seed_lo, seed_hi;
@@ -46,6 +57,7 @@ struct BwdParams {
   float scale;                // softmax_scale
   float scale_log2;           // softmax_scale * log2(e)
   int causal;
+  int tiles_major;            // grid is (B*H, tiles) instead of (tiles, B*H)
   uint32_t drop_threshold;
   float drop_rscale;
   uint32_t seed_lo, seed_hi;
