@@ -57,6 +57,8 @@ def parse_args():
                     help="override the workload's batch size (profiling / scaling studies)")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="override the workload's sequence length (profiling / scaling studies)")
+    ap.add_argument("--dropout", type=float, default=None,
+                    help="override the workload's dropout probability (ablation studies)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="bound on the CPU-oracle sample timed beside the GPU run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -243,6 +245,8 @@ def selected_workload(args):
         if lens is not None:
             lens = (min(lens[0], args.seqlen), min(lens[1], args.seqlen))
         w = replace(w, N=args.seqlen, seqlen_range=lens)
+    if args.dropout is not None:
+        w = replace(w, dropout_p=args.dropout)
     return w
 
 

@@ -34,10 +34,12 @@
  *  - seqlens: NULL, or device int32[B]; keys j >= seqlens[b] are masked for
  *    batch entry b (values are clamped to [0, N]).  Query rows are not masked.
  *  - dropout_p in [0, 1): inverted dropout on the normalised probabilities.
- *    Keep bit of (b, h, i, j): word (j & 3) of Philox4x32-10 with key
- *    (seed & 0xffffffff, seed >> 32) and counter (j >> 2, i, h, b), kept iff
- *    word >= min(floor(dropout_p * 2^32), 2^32 - 1).  dropout_p == 0 draws no
- *    random numbers.
+ *    Keep bit of (b, h, i, j): Philox4x32-10 with key (seed & 0xffffffff,
+ *    seed >> 32) and counter (j >> 3, i, h, b); key j takes the 16-bit half
+ *    (j & 1) (0 = low) of output word ((j >> 1) & 3) and is kept iff that
+ *    value >= t = min(floor(dropout_p * 2^16), 2^16 - 1).  The drop
+ *    probability in force is t / 2^16 (0.0999908 for 0.1) and kept values are
+ *    divided by 1 - t / 2^16.  dropout_p == 0 draws no random numbers.
  *  - block_mask: NULL, or device uint8[nb][nb] with nb = ceil(N / 128),
  *    shared by all (b, h); entry [r][c] == 0 masks every (query, key) pair with
  *    i / 128 == r and j / 128 == c, and such blocks are neither loaded nor

@@ -51,11 +51,13 @@ struct Dropout {
   float rscale;
 };
 
+// Keep test: a 16-bit uniform >= threshold = min(floor(p 2^16), 2^16 - 1);
+// kept values are divided by the keep probability 1 - threshold / 2^16.
 Dropout dropout_params(float p) {
-  const double t = std::floor(static_cast<double>(p) * 4294967296.0);
+  const double t = std::floor(static_cast<double>(p) * 65536.0);
   Dropout d;
-  d.threshold = t >= 4294967295.0 ? 0xFFFFFFFFu : static_cast<uint32_t>(t);
-  d.rscale = p > 0.f ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p))) : 1.f;
+  d.threshold = t >= 65535.0 ? 65535u : static_cast<uint32_t>(t);
+  d.rscale = static_cast<float>(65536.0 / (65536.0 - static_cast<double>(d.threshold)));
   return d;
 }
 

@@ -369,11 +369,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
       const int s = it % L::STAGES;
       // Dropout keep bits of this key for the warpgroup's 64 queries, drawn
-      // before the waits (they do not depend on S or dP).  Lane r of each group
-      // of four computes the block of query q0 + 4 g + r (four keys each); the
-      // four masks are then exchanged so every lane holds its own key's bits:
-      // keep(query qoff + 4 g + r) = bit (4 g + lane % 4) of kw[c][r].
-      uint32_t kw[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+      // before the waits (they do not depend on S or dP).  A block covers
+      // eight keys, which are the eight lanes of an aligned group: lane r of
+      // the group computes the block of query q0 + 8 g + r, then the eight
+      // 32-bit masks are exchanged so every lane holds its own key's bits:
+      // keep(query qoff + 8 g + r) = bit (8 g + lane % 8) of kw[c][r].
+      uint32_t kw[2][8];
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int r = 0; r < 8; ++r) kw[c][r] = 0u;
       if constexpr (DROPOUT) {
         const uint32_t thr = p.drop_threshold;
 #pragma unroll
@@ -381,17 +386,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int qoff = 64 * wg + 32 * c;
           uint32_t own = 0u;
 #pragma unroll
-          for (int gq = 0; gq < 8; ++gq) {
-            const uint32_t qg = static_cast<uint32_t>(qb * 128 + qoff + 4 * gq + (lane & 3));
-            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(jg >> 2), qg,
+          for (int gq = 0; gq < 4; ++gq) {
+            const uint32_t qg = static_cast<uint32_t>(qb * 128 + qoff + 8 * gq + (lane & 7));
+            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(jg >> 3), qg,
                                               static_cast<uint32_t>(w.h), static_cast<uint32_t>(w.b),
                                               p.rk);
-            const uint32_t nib = (rnd.w0 >= thr ? 1u : 0u) | (rnd.w1 >= thr ? 2u : 0u) |
-                                 (rnd.w2 >= thr ? 4u : 0u) | (rnd.w3 >= thr ? 8u : 0u);
-            own |= nib << (4 * gq);
+            own |= keep_byte(rnd, thr) << (8 * gq);
           }
 #pragma unroll
-          for (int r = 0; r < 4; ++r) kw[c][r] = __shfl_sync(0xffffffffu, own, (lane & ~3) | r);
+          for (int r = 0; r < 8; ++r) kw[c][r] = __shfl_sync(0xffffffffu, own, (lane & ~7) | r);
         }
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + s), (it / L::STAGES) & 1u, g));
@@ -430,8 +433,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             float dpv = __uint_as_float(dv[k]);
             float pd = pv;
             if constexpr (DROPOUT) {
-              // query qoff + k = qoff + 4 k4 + e: group k4, lane e of the quad
-              const bool keep = (kw[c][e] >> (4 * k4 + (lane & 3))) & 1u;
+              // query qoff + k, k = 4 k4 + e = 8 g + r with g = k4 / 2, r = 4 (k4 % 2) + e
+              const bool keep = (kw[c][4 * (k4 & 1) + e] >> (8 * (k4 >> 1) + (lane & 7))) & 1u;
               pd = keep ? pv : 0.f;
               dpv = keep ? dpv * p.drop_rscale : 0.f;
             }

@@ -10,7 +10,7 @@ namespace {
 
 __global__ void dropout_mask_kernel(uint8_t* keep, int B, int H, int N, uint32_t threshold,
                                     uint32_t seed_lo, uint32_t seed_hi) {
-  const int64_t groups = (N + 3) / 4;
+  const int64_t groups = (N + 7) / 8;
   const int64_t total = static_cast<int64_t>(B) * H * N * groups;
   for (int64_t x = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; x < total;
        x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -25,9 +25,10 @@ __global__ void dropout_mask_kernel(uint8_t* keep, int B, int H, int N, uint32_t
                                     seed_hi);
     const uint32_t wv[4] = {r.w0, r.w1, r.w2, r.w3};
     uint8_t* dst = keep + row * N;
-    for (int k = 0; k < 4; ++k) {
-      const int64_t j = 4 * g + k;
-      if (j < N) dst[j] = wv[k] >= threshold ? 1 : 0;
+    for (int k = 0; k < 8; ++k) {
+      const int64_t j = 8 * g + k;
+      const uint32_t u = (wv[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+      if (j < N) dst[j] = u >= threshold ? 1 : 0;
     }
   }
 }
@@ -53,7 +54,7 @@ __global__ void wait_timeout_kernel(int* status, uint64_t timeout_ns) {
 
 cudaError_t launch_dropout_mask(uint8_t* keep, int B, int H, int N, uint32_t threshold,
                                 uint32_t seed_lo, uint32_t seed_hi, cudaStream_t stream) {
-  const int64_t total = static_cast<int64_t>(B) * H * N * ((N + 3) / 4);
+  const int64_t total = static_cast<int64_t>(B) * H * N * ((N + 7) / 8);
   const int threads = 256;
   const int64_t blocks = (total + threads - 1) / threads;
   const int grid = static_cast<int>(blocks < 148 * 64 ? blocks : 148 * 64);

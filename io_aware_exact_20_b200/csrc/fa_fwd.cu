@@ -301,13 +301,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if constexpr (DROPOUT) {
           const uint32_t thr = p.drop_threshold;
 #pragma unroll
-          for (int gq = 0; gq < 32; ++gq) {
-            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(kb * 32 + gq),
+          for (int gq = 0; gq < 16; ++gq) {  // keys 8 gq .. 8 gq + 7 of the tile
+            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(kb * 16 + gq),
                                               static_cast<uint32_t>(i), static_cast<uint32_t>(w.h),
                                               static_cast<uint32_t>(w.b), p.rk);
-            const uint32_t nib = (rnd.w0 >= thr ? 1u : 0u) | (rnd.w1 >= thr ? 2u : 0u) |
-                                 (rnd.w2 >= thr ? 4u : 0u) | (rnd.w3 >= thr ? 8u : 0u);
-            keepw[gq >> 3] |= nib << (4 * (gq & 7));
+            keepw[gq >> 2] |= keep_byte(rnd, thr) << (8 * (gq & 3));
           }
         }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + t), cnt & 1u, g));

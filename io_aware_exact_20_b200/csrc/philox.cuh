@@ -5,8 +5,9 @@
 // and the key, the key advanced between rounds by the Weyl constants
 // floor(2^32 (phi - 1)) and floor(2^32 (sqrt(3) - 1)).
 //
-// Dropout keep bit of (b, h, i, j): word (j & 3) of the block at counter
-// (j >> 2, i, h, b) with key (seed lo, seed hi); kept iff word >= threshold.
+// Dropout keep bit of (b, h, i, j): one block at counter (j >> 3, i, h, b) with
+// key (seed lo, seed hi) serves eight keys; key j takes the 16-bit half (j & 1)
+// (0 = low) of word ((j >> 1) & 3) and is kept iff that value >= threshold.
 #pragma once
 
 #include <cstdint>
@@ -64,6 +65,14 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
     c3 = lo0;
   }
   return Philox4{c0, c1, c2, c3};
+}
+
+// The eight keep bits of one block: bit k for key 8 g + k.
+__device__ __forceinline__ uint32_t keep_byte(const Philox4& r, uint32_t thr) {
+  return ((r.w0 & 0xFFFFu) >= thr ? 1u : 0u) | ((r.w0 >> 16) >= thr ? 2u : 0u) |
+         ((r.w1 & 0xFFFFu) >= thr ? 4u : 0u) | ((r.w1 >> 16) >= thr ? 8u : 0u) |
+         ((r.w2 & 0xFFFFu) >= thr ? 16u : 0u) | ((r.w2 >> 16) >= thr ? 32u : 0u) |
+         ((r.w3 & 0xFFFFu) >= thr ? 64u : 0u) | ((r.w3 >> 16) >= thr ? 128u : 0u);
 }
 
 // Host-side round keys for a 64-bit seed.

@@ -110,6 +110,20 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, u
   }
 }
 
+// Per-warpgroup register budget changes (all four warps of a warpgroup execute
+// them).  An increase waits until the registers released by decreases elsewhere
+// in the CTA are available, so the sum over warpgroups must not exceed the
+// CTA's launch allocation (threads x registers per thread); the launcher checks
+// the kernel's register count before the first launch.
+template <uint32_t kRegs>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 // ----------------------------------------------------------------------------
 // TMA (bulk tensor / bulk copies), proxy fences
 // ----------------------------------------------------------------------------

@@ -10,6 +10,7 @@ from .attention_ref import (  # noqa: F401
     attention_backward,
     attention_forward,
     dropout_keep,
+    dropout_scale,
     dropout_threshold,
     head_backward,
     head_backward_cols,

@@ -36,11 +36,15 @@ Readings taken where the pages are silent (all are repeated in the design doc):
     whole 128 x 128 block of (query, key) pairs;
   * all masks combine by logical AND;
   * a row with no valid key has P = 0, O = 0 and LSE = -inf;
-  * dropout is inverted dropout on the normalised P: P_drop = P * Z / (1 - p),
-    Z the keep bit; LSE is that of the undropped softmax;
-  * keep bit Z(b,h,i,j): Philox4x32-10 with key (seed mod 2^32, seed >> 32),
-    counter (j >> 2, i, h, b), output word (j & 3); keep iff word >= t with
-    t = min(floor(p * 2^32), 2^32 - 1), p the float32 value the library receives.
+  * dropout is inverted dropout on the normalised P: P_drop = P * Z / q with
+    q = 1 - t / 2^16 the keep probability of the generator below, Z the keep
+    bit; LSE is that of the undropped softmax;
+  * keep bit Z(b,h,i,j): one Philox4x32-10 block serves eight consecutive
+    keys: key (seed mod 2^32, seed >> 32), counter (j >> 3, i, h, b); key j
+    takes the 16-bit half (j & 1) (0 = low) of output word ((j >> 1) & 3);
+    keep iff that 16-bit value >= t with t = min(floor(p * 2^16), 2^16 - 1),
+    p the float32 value the library receives.  The realised drop probability
+    is therefore t / 2^16 (0.0999908 for p = 0.1).
 
 Parity pins for every function here live in ``tests/test_oracle_pins.py``.
 """
@@ -81,11 +85,17 @@ def valid_mask(n, rows, causal=False, kv_len=None, block_mask=None):
 
 
 def dropout_threshold(p):
-    """Integer threshold t for keep-iff-word >= t, from the float32 value of p."""
+    """Integer threshold t for keep-iff-u16 >= t, from the float32 value of p."""
     p32 = float(np.float32(p))
     if not (0.0 <= p32 < 1.0):
         raise ValueError("dropout probability must lie in [0, 1)")
-    return min(int(math.floor(p32 * 4294967296.0)), 4294967295)
+    return min(int(math.floor(p32 * 65536.0)), 65535)
+
+
+def dropout_scale(p):
+    """1 / keep probability = 2^16 / (2^16 - t): kept values are divided by it."""
+    t = dropout_threshold(p)
+    return 65536.0 / (65536.0 - t)
 
 
 def dropout_keep(seed, p, b, h, rows, n):
@@ -96,11 +106,15 @@ def dropout_keep(seed, p, b, h, rows, n):
     seed = int(seed) & 0xFFFFFFFFFFFFFFFF
     k0, k1 = seed & 0xFFFFFFFF, seed >> 32
     rows = np.asarray(rows, dtype=np.uint64)[:, None]
-    groups = np.arange((n + 3) // 4, dtype=np.uint64)[None, :]
+    groups = np.arange((n + 7) // 8, dtype=np.uint64)[None, :]
     words = philox4x32_10(groups, rows, np.uint64(h), np.uint64(b), k0, k1)
-    # words[w][r, g] is the word for key 4 g + w
-    w = np.stack(words, axis=-1).reshape(len(rows), -1)[:, :n]
-    return w >= np.uint32(t)
+    # key 8 g + 2 m + s takes half s of word m of block g
+    halves = []
+    for w in words:
+        halves.append(w & np.uint32(0xFFFF))
+        halves.append(w >> np.uint32(16))
+    u = np.stack(halves, axis=-1).reshape(len(rows), -1)[:, :n]
+    return u >= np.uint32(t)
 
 
 # ----------------------------------------------------------------------------
@@ -153,7 +167,7 @@ def attention_forward(q, k, v, scale, causal=False, seqlens=None, dropout_p=0.0,
     lse = np.full((B, H, rows.size), np.nan)
     pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
     p32 = float(np.float32(dropout_p))
-    rscale = 1.0 / (1.0 - p32) if p32 > 0 else 1.0
+    rscale = dropout_scale(p32)
     for b, h in pairs:
         kv_len = None if seqlens is None else int(seqlens[b])
         for r0 in range(0, rows.size, slab):
@@ -192,7 +206,7 @@ def head_backward(q, k, v, dout, scale, causal=False, kv_len=None, block_mask=No
         rscale = 1.0
     else:
         z = keep.astype(np.float64)
-        rscale = 1.0 / (1.0 - p32)
+        rscale = dropout_scale(p32)
     pd = p * z * rscale                 # dropped, rescaled P that multiplies V
     dv = pd.T @ dout                    # O = Pd V  ->  dV = Pd^T dO
     dpd = dout @ v.T                    # gradient w.r.t. Pd
@@ -239,7 +253,7 @@ def _row_terms(q, k, v, dout, scale, rows, causal, kv_len, block_mask, keep, dro
     if keep is None or p32 == 0:
         z, rscale = 1.0, 1.0
     else:
-        z, rscale = keep.astype(np.float64), 1.0 / (1.0 - p32)
+        z, rscale = keep.astype(np.float64), dropout_scale(p32)
     pd = p * z * rscale
     dp = (dout[rows] @ v.T) * z * rscale
     dsum = (p * dp).sum(axis=1)
@@ -255,7 +269,7 @@ def head_forward_rows(q, k, v, scale, rows, causal=False, kv_len=None, block_mas
     keep, rscale = None, 1.0
     if p32 > 0:
         keep = dropout_keep(seed, p32, b, h, rows, k.shape[0])
-        rscale = 1.0 / (1.0 - p32)
+        rscale = dropout_scale(p32)
     return _head_forward(q, k, v, scale, rows, causal, kv_len, block_mask, keep, rscale)
 
 

@@ -9,7 +9,7 @@ read back exactly through one-hot dO rows.
 import numpy as np
 import pytest
 
-from oracle import attention_backward, dropout_keep
+from oracle import attention_backward, dropout_keep, dropout_scale
 from io_aware_exact_20_b200.workloads import make_block_mask, make_qkvdo, make_seqlens
 
 pytestmark = pytest.mark.gpu
@@ -84,7 +84,7 @@ def test_backward_is_repeatable_for_dk_dv(lib):
 @pytest.mark.parametrize("d", [64, 128])
 def test_backward_kernel_dropout_bits_exact(lib, d):
     """Q = 0 gives P = 1/N; dO rows one-hot over a window of d queries give
-    dV[j, c] = keep(i0 + c, j) / (N (1 - p)): every keep bit the backward
+    dV[j, c] = keep(i0 + c, j) / (N q), q the keep probability: every keep bit the backward
     kernel used for dV is read back and compared with the oracle's."""
     import torch
     B, H, N, p, seed = 1, 2, 256, 0.1, 0x5EED0003
@@ -93,7 +93,7 @@ def test_backward_kernel_dropout_bits_exact(lib, d):
     k = torch.randn(B, H, N, d, generator=gen).to(torch.bfloat16).cuda()
     v = torch.randn(B, H, N, d, generator=gen).to(torch.bfloat16).cuda()
     o, lse = lib.forward(q, k, v, dropout_p=p, seed=seed)
-    level = 1.0 / (N * (1 - np.float32(p)))
+    level = dropout_scale(p) / N
     for i0 in range(0, N, d):
         do = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
         for c in range(d):

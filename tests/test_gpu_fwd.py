@@ -4,7 +4,7 @@ Tolerances: O max-abs <= 1e-2 and LSE max-abs <= 1e-3 (bf16 inputs, fp32
 accumulation, P rounded to bf16 before the P V product).  O is stored as
 bf16, whose round-to-nearest adds up to 2^-8 |O| on top of the computed
 value's error (half a bf16 ulp, 0.0156 once |O| >= 4, which dropout's
-1 / (1 - p) and rows with few keys reach), so the O bound is
+1 / (keep probability) and rows with few keys reach), so the O bound is
 1e-2 + 2^-8 |O_ref|.  Rows without a valid key must give O = 0 and
 LSE = -inf exactly; dropout keep bits are bit-exact.
 """
@@ -12,7 +12,7 @@ LSE = -inf exactly; dropout keep bits are bit-exact.
 import numpy as np
 import pytest
 
-from oracle import attention_forward, dropout_keep
+from oracle import attention_forward, dropout_keep, dropout_scale
 from io_aware_exact_20_b200.workloads import make_block_mask, make_qkvdo, make_seqlens
 
 pytestmark = pytest.mark.gpu
@@ -127,13 +127,13 @@ def test_dropout_mask_bits_match_oracle(lib):
 @pytest.mark.parametrize("d", [64, 128])
 def test_forward_kernel_dropout_bits_exact(lib, d):
     """Q = 0 makes P uniform (1/N); V rows one-hot over a window of d keys then
-    give O[i, c] = keep(i, j0 + c) / (N (1 - p)): every keep bit the real
+    give O[i, c] = keep(i, j0 + c) / (N q), q the keep probability: every keep bit the real
     forward kernel used is read back and compared with the oracle's."""
     import torch
     B, H, N, p, seed = 1, 2, 256, 0.1, 0x5EED0002
     q = torch.zeros(B, H, N, d, dtype=torch.bfloat16, device="cuda")
     k = torch.randn(B, H, N, d, generator=torch.Generator().manual_seed(0)).to(torch.bfloat16).cuda()
-    level = 1.0 / (N * (1 - np.float32(p)))
+    level = dropout_scale(p) / N
     for j0 in range(0, N, d):
         v = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
         for c in range(d):

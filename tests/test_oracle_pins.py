@@ -124,37 +124,47 @@ def test_philox4x32_words_are_uniform():
 # ---------------------------------------------------------------------------
 
 def test_dropout_threshold_is_exact_integer_of_float32_p():
-    # 0.1 as float32 is 13421773 * 2^-27, so p * 2^32 = 429496736 exactly
-    assert dropout_threshold(0.1) == 429496736
+    # 0.1 as float32 is 13421773 * 2^-27, so p * 2^16 = 6553.6000976... -> 6553
+    assert dropout_threshold(0.1) == 6553
     assert dropout_threshold(0.0) == 0
-    assert dropout_threshold(0.5) == 2**31
-    assert dropout_threshold(np.nextafter(np.float32(1), np.float32(0))) == 2**32 - 2**8
+    assert dropout_threshold(0.5) == 2**15
+    assert dropout_threshold(np.nextafter(np.float32(1), np.float32(0))) == 2**16 - 1
     for bad in (-0.1, 1.0, 1.5, float("nan")):
         with pytest.raises(ValueError):
             dropout_threshold(bad)
 
 
 def test_dropout_keep_uses_the_stated_counter_mapping():
-    """keep(b,h,i,j) = word (j & 3) of Philox4x32-10(counter=(j>>2, i, h, b),
-    key=(seed lo, seed hi)) >= t, checked element by element by brute force."""
+    """keep(b,h,i,j) = 16-bit half (j & 1) of word ((j >> 1) & 3) of
+    Philox4x32-10(counter=(j>>3, i, h, b), key=(seed lo, seed hi)) >= t,
+    checked element by element by brute force."""
     seed = 0x0123456789ABCDEF
     p = 0.3
     t = dropout_threshold(p)
     rows = np.array([0, 1, 5, 130])
-    keep = dropout_keep(seed, p, 3, 2, rows, 11)
+    keep = dropout_keep(seed, p, 3, 2, rows, 19)
     for a, i in enumerate(rows):
-        for j in range(11):
-            w = philox_block([j >> 2, int(i), 2, 3], [seed & 0xFFFFFFFF, seed >> 32])[j & 3]
-            assert keep[a, j] == (w >= t)
+        for j in range(19):
+            w = philox_block([j >> 3, int(i), 2, 3], [seed & 0xFFFFFFFF, seed >> 32])[(j >> 1) & 3]
+            u = (w >> (16 * (j & 1))) & 0xFFFF
+            assert keep[a, j] == (u >= t)
 
 
 def test_dropout_keep_rate_within_5_sigma():
-    """Over ~10^7 draws the keep fraction is 1 - p within 5 sigma (binomial)."""
+    """Over ~10^7 draws the keep fraction is 1 - t / 2^16 within 5 sigma
+    (binomial), t = floor(p 2^16)."""
     for p in (0.1, 0.5):
         keep = dropout_keep(77, p, 1, 4, np.arange(2500), 4000)
         n = keep.size
-        q = 1 - float(np.float32(p))
+        q = 1 - dropout_threshold(p) / 65536.0
         assert abs(keep.mean() - q) < 5 * math.sqrt(q * (1 - q) / n)
+
+
+def test_dropout_scale_is_the_inverse_keep_probability():
+    from oracle import dropout_scale
+    assert dropout_scale(0.0) == 1.0
+    assert dropout_scale(0.5) == 2.0
+    assert dropout_scale(0.1) == 65536.0 / (65536.0 - 6553.0)
 
 
 def test_dropout_p_zero_keeps_everything():
