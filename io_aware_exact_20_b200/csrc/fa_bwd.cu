@@ -21,8 +21,13 @@
 //                 128-row slices of LSE*log2e and D into a ring
 //   warp 1        TMEM allocator and single-thread MMA issuer
 //   warps 4-11    two warpgroups, thread = key row; warpgroup w handles the
-//                 query columns [64 w, 64 w + 64): P from S^T, dS from dP^T,
-//                 P (bf16) back to TMEM, dS (bf16) to swizzled shared memory
+//                 query columns [64 w, 64 w + 64) in two phases per query
+//                 tile: P from S^T (bf16 back to TMEM), then dS from dP^T
+//                 (bf16 to swizzled shared memory)
+//
+// Per query tile the MMA warp issues dV as soon as P is in TMEM and the next
+// tile's S^T right behind it, both while the dS phase runs; dK and dQ follow
+// the dS phase and overlap the next tile's P phase.
 //   warps 12-15   dQ warpgroup, thread = query row: TMEM -> red.global.add
 //
 // TMEM columns: S^T [0,128) with P packed into [64 w, 64 w + 32) per
@@ -59,8 +64,9 @@ struct BwdLayout {
   static constexpr int B_QEMPTY = B_QFULL + STAGES;
   static constexpr int B_SFULL = B_QEMPTY + STAGES;
   static constexpr int B_DPFULL = B_SFULL + 1;
-  static constexpr int B_PFULL = B_DPFULL + 1;
-  static constexpr int B_DSEMPTY = B_PFULL + 1;
+  static constexpr int B_PFULL = B_DPFULL + 1;   // P of the tile is in TMEM
+  static constexpr int B_DSFULL = B_PFULL + 1;   // dS of the tile is in shared memory
+  static constexpr int B_DSEMPTY = B_DSFULL + 1;
   static constexpr int B_DQFULL = B_DSEMPTY + 1;
   static constexpr int B_DQEMPTY = B_DQFULL + 1;
   static constexpr int B_KVDONE = B_DQEMPTY + 1;
@@ -172,6 +178,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
   using L = BwdLayout<D>;
+  // Without dropout the P / dS work is split into two phases so that it
+  // overlaps the MMAs of neighbouring tiles; with dropout the compute warps
+  // are the bottleneck and the serialized order lets the keep-bit generation
+  // of the next tile hide under that tile's MMAs instead.
+  constexpr bool kTwoPhase = !DROPOUT;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {
@@ -211,10 +222,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(bar(L::B_SFULL), 1);
     mbar_init(bar(L::B_DPFULL), 1);
-    mbar_init(bar(L::B_PFULL), 256);
+    mbar_init(bar(L::B_PFULL), 8);     // one arrival per P / dS warp
+    mbar_init(bar(L::B_DSFULL), 8);
     mbar_init(bar(L::B_DSEMPTY), 1);
     mbar_init(bar(L::B_DQFULL), 1);
-    mbar_init(bar(L::B_DQEMPTY), 128);
+    mbar_init(bar(L::B_DQEMPTY), 4);   // one arrival per dQ warp
     mbar_init(bar(L::B_KVDONE), 1);
     fence_mbar_init();
   }
@@ -303,55 +315,117 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_sdp(0, false);
         issue_sdp(0, true);
       }
-      for (int qb = q_first; ok && qb < w.nqb; ++it) {
-        const int s = it % L::STAGES;
-        const int qbn = w.next(qb + 1);
-        if (!mbar_wait(bar(L::B_PFULL), it & 1u, g)) break;
-        tc_fence_after();
-        const uint32_t q_addr = sbase + L::OFF_Q + s * L::TILE;
-        const uint32_t do_addr = sbase + L::OFF_DO + s * L::TILE;
-        // dV += P^T dO   (A = P from TMEM, B = dO MN-major)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::COL_DV, tmem + L::COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
-                 sdesc_sw128(do_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q   (A = dS^T K-major in shared memory, B = Q MN-major)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::COL_DK, sdesc_sw128(ds_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(q_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        // dQ_tile = dS K   (A = dS MN-major, B = K MN-major)
-        if (L::SEPARATE_DQ && it > 0) {
-          // the dQ columns must have been drained by the previous iteration
-          if (!mbar_wait(bar(L::B_DQEMPTY), (it - 1) & 1u, g)) break;
-          tc_fence_after();
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ds_desc = sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024);
-          const uint64_t k_desc = sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024);
-          if constexpr (L::DQ_T)  // dQ^T = K^T dS^T: A = K^T (MN-major), B = dS^T (MN-major)
-            mma_ss(tmem + L::COL_DQ, k_desc, ds_desc, kIdQ, kk > 0 ? 1u : 0u);
-          else
-            mma_ss(tmem + L::COL_DQ, ds_desc, k_desc, kIdQ, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(L::B_DQFULL));
-        mma_commit(bar(L::B_DSEMPTY));
-        mma_commit(bar(L::B_QEMPTY + s));
-        if (qbn < w.nqb) {
+      if constexpr (kTwoPhase) {
+        for (int qb = q_first; ok && qb < w.nqb; ++it) {
+          const int s = it % L::STAGES;
+          const int qbn = w.next(qb + 1);
           const int sn = (it + 1) % L::STAGES;
-          if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
+          const uint32_t q_addr = sbase + L::OFF_Q + s * L::TILE;
+          const uint32_t do_addr = sbase + L::OFF_DO + s * L::TILE;
+          // P of this tile is in TMEM: dV += P^T dO   (A = P from TMEM, B = dO MN-major)
+          if (!mbar_wait(bar(L::B_PFULL), it & 1u, g)) break;
           tc_fence_after();
-          issue_sdp(sn, false);
-          if (!L::SEPARATE_DQ) {
-            if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + L::COL_DV, tmem + L::COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
+                   sdesc_sw128(do_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          // the next tile's S^T overwrites S^T / P only after the dV MMAs above
+          if (qbn < w.nqb) {
+            if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
+            tc_fence_after();
+            issue_sdp(sn, false);
+          }
+          // dS of this tile is in shared memory: dK += dS^T Q  (A = dS^T K-major, B = Q MN-major)
+          if (!mbar_wait(bar(L::B_DSFULL), it & 1u, g)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + L::COL_DK, sdesc_sw128(ds_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(q_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          // dQ_tile = dS K   (A = dS MN-major, B = K MN-major)
+          if (L::SEPARATE_DQ && it > 0) {
+            // the dQ columns must have been drained by the previous iteration
+            if (!mbar_wait(bar(L::B_DQEMPTY), (it - 1) & 1u, g)) break;
             tc_fence_after();
           }
-          issue_sdp(sn, true);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ds_desc = sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024);
+            const uint64_t k_desc = sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024);
+            if constexpr (L::DQ_T)  // dQ^T = K^T dS^T: A = K^T (MN-major), B = dS^T (MN-major)
+              mma_ss(tmem + L::COL_DQ, k_desc, ds_desc, kIdQ, kk > 0 ? 1u : 0u);
+            else
+              mma_ss(tmem + L::COL_DQ, ds_desc, k_desc, kIdQ, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::B_DQFULL));
+          mma_commit(bar(L::B_DSEMPTY));
+          mma_commit(bar(L::B_QEMPTY + s));
+          if (qbn < w.nqb) {
+            // dP^T of the next tile: its columns were read by this tile's dS
+            // phase, and (d = 128) hold the dQ tile until it is drained
+            if (!L::SEPARATE_DQ) {
+              if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
+              tc_fence_after();
+            }
+            issue_sdp(sn, true);
+          }
+          qb = qbn;
         }
-        qb = qbn;
+      } else {
+        // serialized order: dV, dK, dQ once P and dS are both ready, then the
+        // next tile's S^T and dP^T
+        for (int qb = q_first; ok && qb < w.nqb; ++it) {
+          const int s = it % L::STAGES;
+          const int qbn = w.next(qb + 1);
+          if (!mbar_wait(bar(L::B_PFULL), it & 1u, g)) break;
+          tc_fence_after();
+          const uint32_t q_addr = sbase + L::OFF_Q + s * L::TILE;
+          const uint32_t do_addr = sbase + L::OFF_DO + s * L::TILE;
+          // dV += P^T dO   (A = P from TMEM, B = dO MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + L::COL_DV, tmem + L::COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
+                   sdesc_sw128(do_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          // dK += dS^T Q   (A = dS^T K-major in shared memory, B = Q MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + L::COL_DK, sdesc_sw128(ds_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(q_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          // dQ_tile = dS K   (A = dS MN-major, B = K MN-major)
+          if (L::SEPARATE_DQ && it > 0) {
+            // the dQ columns must have been drained by the previous iteration
+            if (!mbar_wait(bar(L::B_DQEMPTY), (it - 1) & 1u, g)) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ds_desc = sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024);
+            const uint64_t k_desc = sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024);
+            if constexpr (L::DQ_T)  // dQ^T = K^T dS^T: A = K^T (MN-major), B = dS^T (MN-major)
+              mma_ss(tmem + L::COL_DQ, k_desc, ds_desc, kIdQ, kk > 0 ? 1u : 0u);
+            else
+              mma_ss(tmem + L::COL_DQ, ds_desc, k_desc, kIdQ, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::B_DQFULL));
+          mma_commit(bar(L::B_DSEMPTY));
+          mma_commit(bar(L::B_QEMPTY + s));
+          if (qbn < w.nqb) {
+            const int sn = (it + 1) % L::STAGES;
+            if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
+            tc_fence_after();
+            issue_sdp(sn, false);
+            if (!L::SEPARATE_DQ) {
+              if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
+              tc_fence_after();
+            }
+            issue_sdp(sn, true);
+          }
+          qb = qbn;
+        }
       }
       mma_commit(bar(L::B_KVDONE));
       mbar_wait_drain(bar(L::B_KVDONE), 0, 1000000000ull);
@@ -399,68 +473,174 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + s), (it / L::STAGES) & 1u, g));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL), it & 1u, g));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DPFULL), it & 1u, g));
-      if (ok && it > 0)
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DSEMPTY), (it - 1) & 1u, g));
-      if (!ok) break;
-      tc_fence_after();
-      const float* lse2 = reinterpret_cast<const float*>(smem + L::OFF_LD + s * 1024);
-      const float* dlt = lse2 + 128;
-      const bool diag = w.causal && qb == w.kb;
+      if constexpr (kTwoPhase) {
+        if (!ok) break;
+        tc_fence_after();
+        const float* lse2 = reinterpret_cast<const float*>(smem + L::OFF_LD + s * 1024);
+        const float* dlt = lse2 + 128;
+        const bool diag = w.causal && qb == w.kb;
+
+        // ---- P phase: P = exp2(S^T scale log2e - LSE log2e), masked; the
+        // dropped P goes to TMEM for dV, the undropped P is kept as fp16 pairs
+        // (P <= 1 here) for the dS phase, negated where dropout drops the pair
+        // (P >= 0, and a P of 0 contributes nothing either way).
+        uint32_t pu[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int qoff = 64 * wg + 32 * c;  // query offset within the tile
-        uint32_t sv[32], dv[32];
-        tmem_ld32<0>(lane_addr + L::COL_S + qoff, sv);
-        tmem_ld32<0>(lane_addr + L::COL_DP + qoff, dv);
-        tmem_wait_ld32<0>(sv);
-        tmem_wait_ld32<0>(dv);
-        const float4* l4 = reinterpret_cast<const float4*>(lse2 + qoff);
-        const float4* d4 = reinterpret_cast<const float4*>(dlt + qoff);
-        uint32_t ppk[16], dpk[16];
+        for (int c = 0; c < 2; ++c) {
+          const int qoff = 64 * wg + 32 * c;  // query offset within the tile
+          uint32_t sv[32];
+          tmem_ld32<0>(lane_addr + L::COL_S + qoff, sv);
+          tmem_wait_ld32<0>(sv);
+          const float4* l4 = reinterpret_cast<const float4*>(lse2 + qoff);
+          uint32_t ppk[16];
 #pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const float4 lv = l4[k4];
-          const float4 dl = d4[k4];
-          const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
-          const float dq[4] = {dl.x, dl.y, dl.z, dl.w};
-          float pe[4], ds[4];
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 lv = l4[k4];
+            const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+            float pe[4], pv4[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k = 4 * k4 + e;
-            float pv = fast_exp2(fmaf(__uint_as_float(sv[k]), p.scale_log2, -lq[e]));
-            if (!key_live || (diag && qoff + k < j)) pv = 0.f;
-            float dpv = __uint_as_float(dv[k]);
-            float pd = pv;
-            if constexpr (DROPOUT) {
-              // query qoff + k, k = 4 k4 + e = 8 g + r with g = k4 / 2, r = 4 (k4 % 2) + e
-              const bool keep = (kw[c][4 * (k4 & 1) + e] >> (8 * (k4 >> 1) + (lane & 7))) & 1u;
-              pd = keep ? pv : 0.f;
-              dpv = keep ? dpv * p.drop_rscale : 0.f;
+            for (int e = 0; e < 4; ++e) {
+              const int k = 4 * k4 + e;
+              float pv = fast_exp2(fmaf(__uint_as_float(sv[k]), p.scale_log2, -lq[e]));
+              if (!key_live || (diag && qoff + k < j)) pv = 0.f;
+              float pd = pv, pkeep = pv;
+              if constexpr (DROPOUT) {
+                // query qoff + k, k = 4 k4 + e = 8 g + r with g = k4 / 2, r = 4 (k4 % 2) + e
+                const bool keep = (kw[c][4 * (k4 & 1) + e] >> (8 * (k4 >> 1) + (lane & 7))) & 1u;
+                pd = keep ? pv : 0.f;
+                pkeep = keep ? pv : -pv;
+              }
+              pe[e] = pd;
+              pv4[e] = pkeep;
             }
-            pe[e] = pd;
-            ds[e] = pv * (dpv - dq[e]);
+            ppk[2 * k4] = pack_bf16(pe[0], pe[1]);
+            ppk[2 * k4 + 1] = pack_bf16(pe[2], pe[3]);
+            pu[16 * c + 2 * k4] = pack_f16(pv4[0], pv4[1]);
+            pu[16 * c + 2 * k4 + 1] = pack_f16(pv4[2], pv4[3]);
           }
-          ppk[2 * k4] = pack_bf16(pe[0], pe[1]);
-          ppk[2 * k4 + 1] = pack_bf16(pe[2], pe[3]);
-          dpk[2 * k4] = pack_bf16(ds[0], ds[1]);
-          dpk[2 * k4 + 1] = pack_bf16(ds[2], ds[3]);
+          // P^T (bf16 pairs) into TMEM: queries [64 wg, 64 wg + 64) -> columns
+          // [64 wg, 64 wg + 32), inside this warpgroup's S^T columns already read
+          tmem_st16<0>(lane_addr + L::COL_S + 64 * wg + 16 * c, ppk);
         }
-        // P^T (bf16 pairs) into TMEM: queries [64 wg, 64 wg + 64) -> columns [64 wg, 64 wg + 32)
-        tmem_st16<0>(lane_addr + L::COL_S + 64 * wg + 16 * c, ppk);
-        // dS^T row j into the 128-byte-swizzled [keys][queries] buffer, panel wg
-        const uint32_t row_addr = sbase + L::OFF_DS + wg * L::PANEL + j * 128;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_PFULL));
+
+        // ---- dS phase: dS = P (dP - D), dP = dP_drop * keep / q under dropout
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DPFULL), it & 1u, g));
+        if (ok && it > 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DSEMPTY), (it - 1) & 1u, g));
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const uint32_t chunk = static_cast<uint32_t>(4 * c + ch) ^ static_cast<uint32_t>(j & 7);
-          st_shared_v4(row_addr + chunk * 16, dpk[4 * ch], dpk[4 * ch + 1], dpk[4 * ch + 2],
-                       dpk[4 * ch + 3]);
+        for (int c = 0; c < 2; ++c) {
+          const int qoff = 64 * wg + 32 * c;
+          uint32_t dv[32];
+          tmem_ld32<0>(lane_addr + L::COL_DP + qoff, dv);
+          tmem_wait_ld32<0>(dv);
+          const float4* d4 = reinterpret_cast<const float4*>(dlt + qoff);
+          uint32_t dpk[16];
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 dl = d4[k4];
+            const float dq[4] = {dl.x, dl.y, dl.z, dl.w};
+            const float2 p01 = unpack_f16(pu[16 * c + 2 * k4]);
+            const float2 p23 = unpack_f16(pu[16 * c + 2 * k4 + 1]);
+            const float pv4[4] = {p01.x, p01.y, p23.x, p23.y};
+            float ds[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int k = 4 * k4 + e;
+              float dpv = __uint_as_float(dv[k]);
+              float pv = pv4[e];
+              if constexpr (DROPOUT) {
+                dpv = (pv >= 0.f) ? dpv * p.drop_rscale : 0.f;  // negative: dropped
+                pv = fabsf(pv);
+              }
+              ds[e] = pv * (dpv - dq[e]);
+            }
+            dpk[2 * k4] = pack_bf16(ds[0], ds[1]);
+            dpk[2 * k4 + 1] = pack_bf16(ds[2], ds[3]);
+          }
+          // dS^T row j into the 128-byte-swizzled [keys][queries] buffer, panel wg
+          const uint32_t row_addr = sbase + L::OFF_DS + wg * L::PANEL + j * 128;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const uint32_t chunk = static_cast<uint32_t>(4 * c + ch) ^ static_cast<uint32_t>(j & 7);
+            st_shared_v4(row_addr + chunk * 16, dpk[4 * ch], dpk[4 * ch + 1], dpk[4 * ch + 2],
+                         dpk[4 * ch + 3]);
+          }
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_DSFULL));
+      } else {
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DPFULL), it & 1u, g));
+        if (ok && it > 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DSEMPTY), (it - 1) & 1u, g));
+        if (!ok) break;
+        tc_fence_after();
+        const float* lse2 = reinterpret_cast<const float*>(smem + L::OFF_LD + s * 1024);
+        const float* dlt = lse2 + 128;
+        const bool diag = w.causal && qb == w.kb;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int qoff = 64 * wg + 32 * c;  // query offset within the tile
+          uint32_t sv[32], dv[32];
+          tmem_ld32<0>(lane_addr + L::COL_S + qoff, sv);
+          tmem_ld32<0>(lane_addr + L::COL_DP + qoff, dv);
+          tmem_wait_ld32<0>(sv);
+          tmem_wait_ld32<0>(dv);
+          const float4* l4 = reinterpret_cast<const float4*>(lse2 + qoff);
+          const float4* d4 = reinterpret_cast<const float4*>(dlt + qoff);
+          uint32_t ppk[16], dpk[16];
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 lv = l4[k4];
+            const float4 dl = d4[k4];
+            const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+            const float dq[4] = {dl.x, dl.y, dl.z, dl.w};
+            float pe[4], ds[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int k = 4 * k4 + e;
+              float pv = fast_exp2(fmaf(__uint_as_float(sv[k]), p.scale_log2, -lq[e]));
+              if (!key_live || (diag && qoff + k < j)) pv = 0.f;
+              float dpv = __uint_as_float(dv[k]);
+              float pd = pv;
+              if constexpr (DROPOUT) {
+                // query qoff + k, k = 4 k4 + e = 8 g + r with g = k4 / 2, r = 4 (k4 % 2) + e
+                const bool keep = (kw[c][4 * (k4 & 1) + e] >> (8 * (k4 >> 1) + (lane & 7))) & 1u;
+                pd = keep ? pv : 0.f;
+                dpv = keep ? dpv * p.drop_rscale : 0.f;
+              }
+              pe[e] = pd;
+              ds[e] = pv * (dpv - dq[e]);
+            }
+            ppk[2 * k4] = pack_bf16(pe[0], pe[1]);
+            ppk[2 * k4 + 1] = pack_bf16(pe[2], pe[3]);
+            dpk[2 * k4] = pack_bf16(ds[0], ds[1]);
+            dpk[2 * k4 + 1] = pack_bf16(ds[2], ds[3]);
+          }
+          // P^T (bf16 pairs) into TMEM: queries [64 wg, 64 wg + 64) -> columns [64 wg, 64 wg + 32)
+          tmem_st16<0>(lane_addr + L::COL_S + 64 * wg + 16 * c, ppk);
+          // dS^T row j into the 128-byte-swizzled [keys][queries] buffer, panel wg
+          const uint32_t row_addr = sbase + L::OFF_DS + wg * L::PANEL + j * 128;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const uint32_t chunk = static_cast<uint32_t>(4 * c + ch) ^ static_cast<uint32_t>(j & 7);
+            st_shared_v4(row_addr + chunk * 16, dpk[4 * ch], dpk[4 * ch + 1], dpk[4 * ch + 2],
+                         dpk[4 * ch + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_PFULL));
       }
-      fence_proxy_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::B_PFULL));
     }
 
     // -------------------------------------------------- dK, dV epilogue
@@ -536,7 +716,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(L::B_DQEMPTY));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::B_DQEMPTY));
     }
   }
 

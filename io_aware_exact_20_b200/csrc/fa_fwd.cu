@@ -16,6 +16,8 @@
 //   warps 2-3    idle
 //   warps 4-7    softmax for Q tile 0   (thread = row, TMEM lanes 0..127)
 //   warps 8-11   softmax for Q tile 1
+// setmaxnreg moves registers from the first warpgroup (72 each) to the two
+// softmax warpgroups (216 each), within the 384 x 168 of the launch.
 //
 // The running maximum m is only moved when a new block raises it by more than
 // 8 (in log2 units); until then exp2 values may reach 2^8, and O and the row
@@ -35,6 +37,12 @@ namespace fa {
 namespace {
 
 constexpr int kFwdThreads = 384;
+constexpr int kLaunchRegs = 168;  // registers per thread at launch (checked)
+// Register budgets after setmaxnreg: the control warpgroup (producer, MMA, two
+// idle warps) gives registers to the two softmax warpgroups.
+constexpr uint32_t kRegsCtl = 72, kRegsSoftmax = 216;
+static_assert(4 * 32 * (kRegsCtl + 2 * kRegsSoftmax) <= kFwdThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -129,7 +137,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::B_QFULL + t), 1);
       mbar_init(bar(L::B_SFULL + t), 1);
-      mbar_init(bar(L::B_PFULL + t), 128);
+      mbar_init(bar(L::B_PFULL + t), 4);  // one arrival per softmax warp
       mbar_init(bar(L::B_ODONE + t), 1);
     }
     for (int s = 0; s < L::STAGES; ++s) {
@@ -149,6 +157,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Each role runs inside the branch that sets its register budget, so that
+  // the compiler allocates every role's code under its own limit.
+  if (warp < 4) {
+  setmaxnreg_dec<kRegsCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
@@ -279,7 +291,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int t = 0; t < 2; ++t)
         if ((t == 0 || w.exists1) && !q_ready[t]) mbar_wait_drain(bar(L::B_QFULL + t), 0, 100000000ull);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // -------------------------------------------------------------- softmax
     const int t = (warp - 4) >> 2;
     const int wq = warp & 3;
@@ -323,34 +337,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
         const int j0 = kb * 128;
         const bool need_mask = (w.causal && kb == w.qb0 + t) || (j0 + 128 > w.kv_len);
-        float mx = -INFINITY;
+        // row maximum with eight independent partial maxima (short dependency chains)
+        float mxp[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mxp[u] = -INFINITY;
         if (need_mask) {
           const int lim = w.causal ? min(w.kv_len - j0, i - j0 + 1) : (w.kv_len - j0);
 #pragma unroll
           for (int j = 0; j < 128; ++j) {
             const float v = (j < lim) ? __uint_as_float(sr[j]) : -INFINITY;
             sr[j] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
+            mxp[j & 7] = fmaxf(mxp[j & 7], v);
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 128; ++j) mx = fmaxf(mx, __uint_as_float(sr[j]));
+          for (int j = 0; j < 128; ++j) mxp[j & 7] = fmaxf(mxp[j & 7], __uint_as_float(sr[j]));
         }
+        float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                         fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
         mx *= p.scale_log2;
         const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         const float alpha = fast_exp2(m - m_use);  // 0 on the first tile, 1 if unchanged
-        float rs0 = 0.f, rs1 = 0.f;
+        float rsp[8];
 #pragma unroll
-        for (int j = 0; j < 128; j += 2) {
-          const float e0 = fast_exp2(fmaf(__uint_as_float(sr[j]), p.scale_log2, -m_use));
-          const float e1 = fast_exp2(fmaf(__uint_as_float(sr[j + 1]), p.scale_log2, -m_use));
-          rs0 += e0;
-          rs1 += e1;
-          sr[j] = __float_as_uint(e0);
-          sr[j + 1] = __float_as_uint(e1);
+        for (int u = 0; u < 8; ++u) rsp[u] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 128; ++j) {
+          const float e = fast_exp2(fmaf(__uint_as_float(sr[j]), p.scale_log2, -m_use));
+          rsp[j & 7] += e;
+          sr[j] = __float_as_uint(e);
         }
-        l = l * alpha + (rs0 + rs1);
+        const float rs = ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3])) + ((rsp[4] + rsp[5]) + (rsp[6] + rsp[7]));
+        l = l * alpha + rs;
         m = m_new;
 
         if constexpr (DROPOUT) {
@@ -385,7 +404,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(L::B_PFULL + t));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_PFULL + t));
         ++cnt;
       }
 
@@ -439,6 +459,16 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          const FwdParams& p, cudaStream_t stream) {
   using L = FwdLayout<D>;
   auto kern = fwd_kernel<D, DROPOUT>;
+  // The setmaxnreg split above is sized for exactly kLaunchRegs registers per
+  // thread at launch; with any other count an increase could wait forever.
+  static int regs_checked = 0;
+  if (!regs_checked) {
+    cudaFuncAttributes attr{};
+    cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+    if (e != cudaSuccess) return e;
+    if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    regs_checked = 1;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::SMEM));
   if (e != cudaSuccess) return e;
