@@ -10,14 +10,14 @@
 //   P_t = exp2(S_t * scale * log2e - m_t)   online softmax, one thread per row
 //   O_t += P_t V            tcgen05.mma with P_t read from TMEM
 //
-// Roles (384 threads):
+// Roles, two Q tiles per CTA (384 threads):
 //   warp 0       TMA producer: Q tiles once, then K/V tiles into a ring
 //   warp 1       TMEM allocator and single-thread MMA issuer
 //   warps 2-3    idle
 //   warps 4-7    softmax for Q tile 0   (thread = row, TMEM lanes 0..127)
 //   warps 8-11   softmax for Q tile 1
-// setmaxnreg moves registers from the first warpgroup (72 each) to the two
-// softmax warpgroups (216 each), within the 384 x 168 of the launch.
+// One Q tile per CTA (192 threads, two CTAs per SM): warps 0 and 1 as above,
+// warps 2-5 softmax.
 //
 // The running maximum m is only moved when a new block raises it by more than
 // 8 (in log2 units); until then exp2 values may reach 2^8, and O and the row
@@ -36,24 +36,35 @@
 namespace fa {
 namespace {
 
-constexpr int kFwdThreads = 384;
-constexpr int kLaunchRegs = 168;  // registers per thread at launch (checked)
-// Register budgets after setmaxnreg: the control warpgroup (producer, MMA, two
-// idle warps) gives registers to the two softmax warpgroups.
-constexpr uint32_t kRegsCtl = 72, kRegsSoftmax = 216;
-static_assert(4 * 32 * (kRegsCtl + 2 * kRegsSoftmax) <= kFwdThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int D>
+// Q tiles per CTA.  Two (the default) share every K/V tile between two 128-row
+// Q tiles, with the two softmax warpgroups ping-ponging on the tensor core.
+// One (d = 64, short sequences) halves the CTA so that two CTAs share an SM
+// and one CTA's set-up and epilogue hide under the other's main loop.
+template <int NQ>
+struct FwdRoles {
+  static constexpr int THREADS = NQ == 2 ? 384 : 192;
+  static constexpr int MIN_BLOCKS = NQ == 2 ? 1 : 2;
+  static constexpr int SOFTMAX_WARP0 = NQ == 2 ? 4 : 2;  // warps before it: producer, MMA, idle
+  static constexpr int LAUNCH_REGS = 168;                // registers per thread at launch (checked)
+  // NQ = 2: setmaxnreg moves registers from the first warpgroup (72 each) to
+  // the two softmax warpgroups (216 each), within the 384 x 168 of the launch.
+  static constexpr bool SPLIT_REGS = NQ == 2;
+  static constexpr uint32_t REGS_CTL = 72, REGS_SOFTMAX = 216;
+  static_assert(!SPLIT_REGS || 4 * 32 * (REGS_CTL + 2 * REGS_SOFTMAX) <= THREADS * LAUNCH_REGS,
+                "register split exceeds the launch allocation");
+};
+
+template <int D, int NQ>
 struct FwdLayout {
   static constexpr int PANELS = D / 64;                 // 64-column, 128-byte-swizzled panels
   static constexpr uint32_t PANEL = 128u * 128u;        // bytes of one [128 rows][64 cols] panel
   static constexpr uint32_t TILE = PANEL * PANELS;      // bytes of one 128-row tile
-  static constexpr int STAGES = (D == 64) ? 4 : 2;      // K/V ring depth
+  static constexpr int STAGES = NQ == 1 ? 2 : (D == 64 ? 4 : 2);  // K/V ring depth
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_KV = 2 * TILE;
+  static constexpr uint32_t OFF_KV = NQ * TILE;
   static constexpr uint32_t OFF_BAR = OFF_KV + STAGES * 2 * TILE;
   static constexpr int B_QFULL = 0;
   static constexpr int B_KFULL = 2;
@@ -66,9 +77,10 @@ struct FwdLayout {
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16;
-  static constexpr uint32_t O_COL = 256;
-  static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(O_COL + 2 * D <= 512, "TMEM budget");
+  static constexpr uint32_t O_COL = 128 * NQ;
+  static constexpr uint32_t TMEM_COLS = NQ == 2 ? 512 : 256;
+  static_assert(SMEM <= (NQ == 2 ? 232448u : 113u * 1024u), "shared memory budget");
+  static_assert(O_COL + NQ * D <= TMEM_COLS, "TMEM budget");
 };
 
 // Which (Q tile, K/V tile) pairs of this CTA take part.
@@ -92,11 +104,12 @@ struct FwdWork {
   }
 };
 
-template <int D, bool DROPOUT>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+template <int D, bool DROPOUT, int NQ>
+__global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCKS)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, NQ>;
+  using R = FwdRoles<NQ>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {  // the swizzled layouts need 1024-byte alignment
@@ -113,15 +126,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   FwdWork w;
   {
-    const int nqp = (p.N + 255) / 256;
+    const int nqp = (p.N + 128 * NQ - 1) / (128 * NQ);
     const int tile = static_cast<int>(p.tiles_major ? blockIdx.y : blockIdx.x);
     const int qp = nqp - 1 - tile;  // heaviest causal rows first
-    w.q0 = qp * 256;
-    w.qb0 = qp * 2;
+    w.q0 = qp * 128 * NQ;
+    w.qb0 = qp * NQ;
     w.bh = static_cast<int>(p.tiles_major ? blockIdx.x : blockIdx.y);
     w.b = w.bh / p.H;
     w.h = w.bh % p.H;
-    w.exists1 = (w.q0 + 128) < p.N;
+    w.exists1 = NQ == 2 && (w.q0 + 128) < p.N;
     int kv = p.N;
     if (p.seqlens != nullptr) kv = max(0, min(p.seqlens[w.b], p.N));
     w.kv_len = kv;
@@ -149,7 +162,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -159,8 +172,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   // Each role runs inside the branch that sets its register budget, so that
   // the compiler allocates every role's code under its own limit.
-  if (warp < 4) {
-  setmaxnreg_dec<kRegsCtl>();
+  if (warp < R::SOFTMAX_WARP0) {
+  if constexpr (R::SPLIT_REGS) setmaxnreg_dec<R::REGS_CTL>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
@@ -293,9 +306,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   }
   } else {
-    setmaxnreg_inc<kRegsSoftmax>();
+    if constexpr (R::SPLIT_REGS) setmaxnreg_inc<R::REGS_SOFTMAX>();
     // -------------------------------------------------------------- softmax
-    const int t = (warp - 4) >> 2;
+    const int t = (warp - R::SOFTMAX_WARP0) >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const int i = w.q0 + 128 * t + r;
@@ -337,38 +350,43 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
         const int j0 = kb * 128;
         const bool need_mask = (w.causal && kb == w.qb0 + t) || (j0 + 128 > w.kv_len);
-        // row maximum with eight independent partial maxima (short dependency chains)
-        float mxp[8];
+        // row maximum with independent partial maxima (short dependency chains;
+        // as many as the register budget allows)
+        constexpr int kParts = R::SPLIT_REGS ? 8 : 2;
+        float mxp[kParts];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mxp[u] = -INFINITY;
+        for (int u = 0; u < kParts; ++u) mxp[u] = -INFINITY;
         if (need_mask) {
           const int lim = w.causal ? min(w.kv_len - j0, i - j0 + 1) : (w.kv_len - j0);
 #pragma unroll
           for (int j = 0; j < 128; ++j) {
             const float v = (j < lim) ? __uint_as_float(sr[j]) : -INFINITY;
             sr[j] = __float_as_uint(v);
-            mxp[j & 7] = fmaxf(mxp[j & 7], v);
+            mxp[j % kParts] = fmaxf(mxp[j % kParts], v);
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 128; ++j) mxp[j & 7] = fmaxf(mxp[j & 7], __uint_as_float(sr[j]));
+          for (int j = 0; j < 128; ++j) mxp[j % kParts] = fmaxf(mxp[j % kParts], __uint_as_float(sr[j]));
         }
-        float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                         fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        float mx = mxp[0];
+#pragma unroll
+        for (int u = 1; u < kParts; ++u) mx = fmaxf(mx, mxp[u]);
         mx *= p.scale_log2;
         const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         const float alpha = fast_exp2(m - m_use);  // 0 on the first tile, 1 if unchanged
-        float rsp[8];
+        float rsp[kParts];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) rsp[u] = 0.f;
+        for (int u = 0; u < kParts; ++u) rsp[u] = 0.f;
 #pragma unroll
         for (int j = 0; j < 128; ++j) {
           const float e = fast_exp2(fmaf(__uint_as_float(sr[j]), p.scale_log2, -m_use));
-          rsp[j & 7] += e;
+          rsp[j % kParts] += e;
           sr[j] = __float_as_uint(e);
         }
-        const float rs = ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3])) + ((rsp[4] + rsp[5]) + (rsp[6] + rsp[7]));
+        float rs = rsp[0];
+#pragma unroll
+        for (int u = 1; u < kParts; ++u) rs += rsp[u];
         l = l * alpha + rs;
         m = m_new;
 
@@ -450,42 +468,51 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, L::TMEM_COLS);
   }
 }
 
-template <int D, bool DROPOUT>
+template <int D, bool DROPOUT, int NQ>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, cudaStream_t stream) {
-  using L = FwdLayout<D>;
-  auto kern = fwd_kernel<D, DROPOUT>;
-  // The setmaxnreg split above is sized for exactly kLaunchRegs registers per
-  // thread at launch; with any other count an increase could wait forever.
+  using L = FwdLayout<D, NQ>;
+  using R = FwdRoles<NQ>;
+  auto kern = fwd_kernel<D, DROPOUT, NQ>;
+  // The setmaxnreg split is sized for exactly LAUNCH_REGS registers per thread
+  // at launch; with any other count an increase could wait forever.
   static int regs_checked = 0;
   if (!regs_checked) {
     cudaFuncAttributes attr{};
     cudaError_t e = cudaFuncGetAttributes(&attr, kern);
     if (e != cudaSuccess) return e;
-    if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    if (R::SPLIT_REGS && attr.numRegs != R::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
     regs_checked = 1;
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::SMEM));
   if (e != cudaSuccess) return e;
-  const unsigned tiles = static_cast<unsigned>((p.N + 255) / 256), bh = static_cast<unsigned>(p.B * p.H);
+  const unsigned tiles = static_cast<unsigned>((p.N + 128 * NQ - 1) / (128 * NQ));
+  const unsigned bh = static_cast<unsigned>(p.B * p.H);
   const dim3 grid = p.tiles_major ? dim3(bh, tiles) : dim3(tiles, bh);
-  kern<<<grid, kFwdThreads, L::SMEM, stream>>>(tq, tk, tv, p);
+  kern<<<grid, R::THREADS, L::SMEM, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
+
+// One Q tile per CTA (two CTAs per SM) pays off when the sequences are short,
+// where each CTA has few K/V tiles to amortise its set-up and epilogue.
+inline bool one_tile_per_cta(int d, int N) { return d == 64 && N <= 4096; }
 
 }  // namespace
 
 cudaError_t launch_fwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, cudaStream_t stream) {
-  if (d == 64) return dropout ? launch_fwd_t<64, true>(tq, tk, tv, p, stream)
-                              : launch_fwd_t<64, false>(tq, tk, tv, p, stream);
-  if (d == 128) return dropout ? launch_fwd_t<128, true>(tq, tk, tv, p, stream)
-                               : launch_fwd_t<128, false>(tq, tk, tv, p, stream);
+  if (d == 64 && one_tile_per_cta(d, p.N))
+    return dropout ? launch_fwd_t<64, true, 1>(tq, tk, tv, p, stream)
+                   : launch_fwd_t<64, false, 1>(tq, tk, tv, p, stream);
+  if (d == 64) return dropout ? launch_fwd_t<64, true, 2>(tq, tk, tv, p, stream)
+                              : launch_fwd_t<64, false, 2>(tq, tk, tv, p, stream);
+  if (d == 128) return dropout ? launch_fwd_t<128, true, 2>(tq, tk, tv, p, stream)
+                               : launch_fwd_t<128, false, 2>(tq, tk, tv, p, stream);
   return cudaErrorInvalidValue;
 }
 
