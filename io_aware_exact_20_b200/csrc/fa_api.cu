@@ -212,10 +212,11 @@ fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void*
   fa_status_t st =
       bwd_params(&p, B, H, N, d, softmax_scale, dropout_p, workspace, workspace_bytes);
   if (st != FA_OK) return st;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   const uint64_t bh = static_cast<uint64_t>(B) * H;
   if (!fa::make_tmap_bf16(&tq, q, d, N, bh, 128) || !fa::make_tmap_bf16(&tk, k, d, N, bh, 128) ||
-      !fa::make_tmap_bf16(&tv, v, d, N, bh, 128) || !fa::make_tmap_bf16(&tdo, dout, d, N, bh, 128))
+      !fa::make_tmap_bf16(&tv, v, d, N, bh, 128) || !fa::make_tmap_bf16(&tdo, dout, d, N, bh, 128) ||
+      !fa::make_tmap_f32_2d(&tdq, p.ws_dq, d, bh * static_cast<uint64_t>(p.Npad), 128))
     return FA_ERR_CUDA;
   p.dk = dk;
   p.dv = dv;
@@ -226,7 +227,7 @@ fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void*
   p.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
   p.seed_hi = static_cast<uint32_t>(seed >> 32);
   p.rk = fa::philox_round_keys(seed);
-  const cudaError_t e = fa::launch_bwd_main(d, p.drop_threshold != 0, tq, tk, tv, tdo, p,
+  const cudaError_t e = fa::launch_bwd_main(d, p.drop_threshold != 0, tq, tk, tv, tdo, tdq, p,
                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -28,7 +28,12 @@
 // Per query tile the MMA warp issues dV as soon as P is in TMEM and the next
 // tile's S^T right behind it, both while the dS phase runs; dK and dQ follow
 // the dS phase and overlap the next tile's P phase.
-//   warps 12-15   dQ warpgroup, thread = query row: TMEM -> red.global.add
+//   warps 12-15   dQ warpgroup.  d = 64: TMEM -> the just-consumed Q / dO
+//                 stage (128-byte-swizzled fp32 boxes of 32 columns x 128
+//                 rows) -> TMA bulk reduce-add into the fp32 accumulators;
+//                 the stage goes back to the producer once the reduce has
+//                 read it.  d = 128: TMEM -> red.global.add of the transposed
+//                 tile, one coalesced 128-byte line per warp instruction
 //
 // TMEM columns: S^T [0,128) with P packed into [64 w, 64 w + 32) per
 // warpgroup; dP^T [128,256); dV [256, 256 + D); dK [256 + D, 256 + 2 D); the
@@ -70,7 +75,8 @@ struct BwdLayout {
   static constexpr int B_DQFULL = B_DSEMPTY + 1;
   static constexpr int B_DQEMPTY = B_DQFULL + 1;
   static constexpr int B_KVDONE = B_DQEMPTY + 1;
-  static constexpr int NBAR = B_KVDONE + 1;
+  static constexpr int B_STAGED = B_KVDONE + 1;   // dQ tile written to the staging boxes
+  static constexpr int NBAR = B_STAGED + 1;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
@@ -82,6 +88,12 @@ struct BwdLayout {
   // feature c, column = query) so that each warp's reduction into the fp32
   // accumulators covers 32 consecutive floats of one row: one 128-byte line.
   static constexpr bool DQ_T = (D == 128);
+  // d = 64: the dQ tile is staged in the just-consumed Q / dO stage and added
+  // into the accumulators by TMA bulk reduce-adds (the dQ warps then hand the
+  // stage back to the producer).  d = 128 keeps the transposed tile and its
+  // coalesced reductions: there a 64 KB stage of the two-deep Q / dO ring
+  // held until the reduce has read it costs more than it saves.
+  static constexpr bool TMA_REDUCE = !DQ_T;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(COL_DK + D <= 512, "TMEM budget");
 };
@@ -176,7 +188,7 @@ template <int D, bool DROPOUT>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdLayout<D>;
   // Without dropout the P / dS work is split into two phases so that it
   // overlaps the MMAs of neighbouring tiles; with dropout the compute warps
@@ -228,6 +240,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(L::B_DQFULL), 1);
     mbar_init(bar(L::B_DQEMPTY), 4);   // one arrival per dQ warp
     mbar_init(bar(L::B_KVDONE), 1);
+    mbar_init(bar(L::B_STAGED), 4);    // one arrival per dQ warp
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -361,7 +374,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           mma_commit(bar(L::B_DQFULL));
           mma_commit(bar(L::B_DSEMPTY));
-          mma_commit(bar(L::B_QEMPTY + s));
+          if constexpr (!L::TMA_REDUCE) mma_commit(bar(L::B_QEMPTY + s));
           if (qbn < w.nqb) {
             // dP^T of the next tile: its columns were read by this tile's dS
             // phase, and (d = 128) hold the dQ tile until it is drained
@@ -412,7 +425,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           mma_commit(bar(L::B_DQFULL));
           mma_commit(bar(L::B_DSEMPTY));
-          mma_commit(bar(L::B_QEMPTY + s));
+          if constexpr (!L::TMA_REDUCE) mma_commit(bar(L::B_QEMPTY + s));
           if (qbn < w.nqb) {
             const int sn = (it + 1) % L::STAGES;
             if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
@@ -688,37 +701,69 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int r = wq * 32 + lane;  // query row within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     int it = 0;
+    bool issued = false;
     for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
+      const int s = it % L::STAGES;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL), it & 1u, g))) break;
       tc_fence_after();
+      // box b (columns 32 b .. 32 b + 31) of the staging area: the Q buffer of
+      // stage s holds the first D / 64 boxes, its dO buffer the rest
+      auto box = [&](int b) -> uint32_t {
+        return b < L::PANELS ? sbase + L::OFF_Q + s * L::TILE + b * L::PANEL
+                             : sbase + L::OFF_DO + s * L::TILE + (b - L::PANELS) * L::PANEL;
+      };
       if constexpr (L::DQ_T) {
-        // lane r = feature r; column c = query qb * 128 + c
+        // lane r = feature r; column c = query qb * 128 + c: each warp's
+        // reduction covers 32 consecutive floats of one accumulator row
         float* dst = p.ws_dq + (static_cast<size_t>(w.bh) * p.Npad + qb * 128) * D + r;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c4 = 0; c4 < 4; ++c4) {
           uint32_t a[32];
-          tmem_ld32<0>(lane_addr + L::COL_DQ + 32 * c, a);
+          tmem_ld32<0>(lane_addr + L::COL_DQ + 32 * c4, a);
           tmem_wait_ld32<0>(a);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) red_add_f32(dst + (32 * c + k) * D, __uint_as_float(a[k]));
+          for (int k = 0; k < 32; ++k) red_add_f32(dst + (32 * c4 + k) * D, __uint_as_float(a[k]));
         }
       } else {
-        float* dst = p.ws_dq + (static_cast<size_t>(w.bh) * p.Npad + qb * 128 + r) * D;
+        // lane r = query r; columns 32 b .. 32 b + 31 = box b
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int b = 0; b < D / 32; ++b) {
           uint32_t a[32];
-          tmem_ld32<0>(lane_addr + L::COL_DQ + 32 * c, a);
+          tmem_ld32<0>(lane_addr + L::COL_DQ + 32 * b, a);
           tmem_wait_ld32<0>(a);
+          const uint32_t row = box(b) + r * 128;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            red_add_v4(dst + 32 * c + 4 * k, __uint_as_float(a[4 * k]), __uint_as_float(a[4 * k + 1]),
-                       __uint_as_float(a[4 * k + 2]), __uint_as_float(a[4 * k + 3]));
+            st_shared_v4(row + ((k ^ (r & 7)) << 4), a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
         }
       }
       tc_fence_before();
+      if constexpr (L::TMA_REDUCE) fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::B_DQEMPTY));
+      if (lane == 0) {
+        mbar_arrive(bar(L::B_DQEMPTY));  // the dQ columns of TMEM are free again
+        if constexpr (L::TMA_REDUCE) mbar_arrive(bar(L::B_STAGED));
+      }
+      if (L::TMA_REDUCE && warp == 12) {
+        // one thread reduces the staged tile into the accumulators, then hands
+        // the stage back to the producer once the boxes have been read
+        bool staged = true;
+        if (lane == 0) {
+          staged = mbar_wait(bar(L::B_STAGED), it & 1u, g);
+          if (staged) {
+            const int32_t y = static_cast<int32_t>(static_cast<int64_t>(w.bh) * p.Npad + qb * 128);
+#pragma unroll
+            for (int b = 0; b < D / 32; ++b) tma_reduce_add_2d(&tm_dq, box(b), 32 * b, y);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+            issued = true;
+            mbar_arrive(bar(L::B_QEMPTY + s));
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, staged ? 1 : 0, 0)) break;  // the whole warp leaves
+      }
     }
+    if (issued) bulk_wait_group0();  // the reductions have landed before the CTA exits
   }
 
   tc_fence_before();
@@ -739,7 +784,8 @@ cudaError_t launch_pre_t(const BwdParams& p, cudaStream_t stream) {
 
 template <int D, bool DROPOUT>
 cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+                          const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdParams& p,
+                          cudaStream_t stream) {
   using L = BwdLayout<D>;
   auto kern = bwd_main_kernel<D, DROPOUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -747,7 +793,7 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   if (e != cudaSuccess) return e;
   const unsigned tiles = static_cast<unsigned>((p.N + 127) / 128), bh = static_cast<unsigned>(p.B * p.H);
   const dim3 grid = p.tiles_major ? dim3(bh, tiles) : dim3(tiles, bh);
-  kern<<<grid, kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, p);
+  kern<<<grid, kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError();
 }
 
@@ -767,12 +813,12 @@ cudaError_t launch_bwd_pre(int d, const BwdParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
-                            const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p,
-                            cudaStream_t stream) {
-  if (d == 64) return dropout ? launch_main_t<64, true>(tq, tk, tv, tdo, p, stream)
-                              : launch_main_t<64, false>(tq, tk, tv, tdo, p, stream);
-  if (d == 128) return dropout ? launch_main_t<128, true>(tq, tk, tv, tdo, p, stream)
-                               : launch_main_t<128, false>(tq, tk, tv, tdo, p, stream);
+                            const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdq,
+                            const BwdParams& p, cudaStream_t stream) {
+  if (d == 64) return dropout ? launch_main_t<64, true>(tq, tk, tv, tdo, tdq, p, stream)
+                              : launch_main_t<64, false>(tq, tk, tv, tdo, tdq, p, stream);
+  if (d == 128) return dropout ? launch_main_t<128, true>(tq, tk, tv, tdo, tdq, p, stream)
+                               : launch_main_t<128, false>(tq, tk, tv, tdo, tdq, p, stream);
   return cudaErrorInvalidValue;
 }
 

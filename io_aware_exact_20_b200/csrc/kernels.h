@@ -72,8 +72,8 @@ cudaError_t launch_fwd(int d, bool dropout, const CUtensorMap& tq, const CUtenso
 // kernel (dK, dV, dQ accumulators), and the dQ conversion.
 cudaError_t launch_bwd_pre(int d, const BwdParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
-                            const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p,
-                            cudaStream_t stream);
+                            const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdq,
+                            const BwdParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_post(int d, const BwdParams& p, cudaStream_t stream);
 
 cudaError_t launch_dropout_mask(uint8_t* keep, int B, int H, int N, uint32_t threshold,

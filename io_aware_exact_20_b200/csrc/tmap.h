@@ -44,4 +44,21 @@ inline bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t d, uint6
   return r == CUDA_SUCCESS;
 }
 
+// fp32 matrix [rows][cols] at `base`; box = 32 columns (128 bytes) x
+// box_rows, 128-byte swizzle.  Used to reduce-add dQ tiles into the backward's
+// fp32 accumulators.
+inline bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                             uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fa
