@@ -9,8 +9,9 @@
 //   dV = P_drop^T dO,   dK = scale dS^T Q,   dQ = scale dS K.
 //
 // Three kernels:
-//   bwd_pre   D_i, LSE_i * log2(e) (+inf for rows without keys and padding
-//             rows, so that their P is exactly 0), zeroed dQ accumulators;
+//   bwd_pre   -D_i, -LSE_i * log2(e) (-inf for rows without keys and
+//             padding rows, so that their P is exactly 0), zeroed dQ
+//             accumulators;
 //   bwd_main  one CTA per (b, h, 128-key tile), looping over the query tiles
 //             that tile meets; dK, dV stay in TMEM for the whole loop, dQ
 //             partial products are added into fp32 accumulators;
@@ -41,6 +42,8 @@
 // feature, column = query) in the dP^T columns once dP^T has been consumed.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "kernels.h"
 #include "philox.cuh"
 #include "ptx.cuh"
@@ -62,7 +65,7 @@ struct BwdLayout {
   static constexpr uint32_t OFF_Q = 2 * TILE;
   static constexpr uint32_t OFF_DO = OFF_Q + STAGES * TILE;
   static constexpr uint32_t OFF_DS = OFF_DO + STAGES * TILE;  // [128 keys][128 queries] bf16
-  static constexpr uint32_t OFF_LD = OFF_DS + 2 * PANEL;      // per stage: lse2[128], delta[128]
+  static constexpr uint32_t OFF_LD = OFF_DS + 2 * PANEL;      // per stage: -lse2[128], -delta[128]
   static constexpr uint32_t OFF_BAR = OFF_LD + STAGES * 1024;
   static constexpr int B_KV = 0;
   static constexpr int B_QFULL = 1;
@@ -147,13 +150,13 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
 #pragma unroll
   for (int m = G / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
   if (part == 0) {
-    p.ws_delta[row] = (i < p.N) ? acc : 0.f;
-    float l2 = INFINITY;
+    p.ws_delta[row] = (i < p.N) ? -acc : 0.f;
+    float nl2 = -INFINITY;
     if (i < p.N) {
       const float l = p.lse[static_cast<size_t>(bh) * p.N + i];
-      if (l != -INFINITY) l2 = l * kLog2e;
+      if (l != -INFINITY) nl2 = -l * kLog2e;
     }
-    p.ws_lse2[row] = l2;
+    p.ws_lse2[row] = nl2;
   }
   float4* dq = reinterpret_cast<float4*>(p.ws_dq + row * D + part * 8);
   dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -451,6 +454,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int jg = w.kb * 128 + j;
     const bool key_live = jg < w.kv_len;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+    const float2 rs2 = make_float2(p.drop_rscale, p.drop_rscale);
     bool ok = true;
     int it = 0;
     for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
@@ -459,8 +464,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // before the waits (they do not depend on S or dP).  A block covers
       // eight keys, which are the eight lanes of an aligned group: lane r of
       // the group computes the block of query q0 + 8 g + r, then the eight
-      // 32-bit masks are exchanged so every lane holds its own key's bits:
-      // keep(query qoff + 8 g + r) = bit (8 g + lane % 8) of kw[c][r].
+      // 32-bit masks are exchanged and shifted so that every lane holds its
+      // own key's bits: keep(query qoff + 8 g + r) = bit 8 g of kw[c][r].
       uint32_t kw[2][8];
 #pragma unroll
       for (int c = 0; c < 2; ++c)
@@ -481,60 +486,87 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             own |= keep_byte(rnd, thr) << (8 * gq);
           }
 #pragma unroll
-          for (int r = 0; r < 8; ++r) kw[c][r] = __shfl_sync(0xffffffffu, own, (lane & ~7) | r);
+          for (int r = 0; r < 8; ++r)
+            kw[c][r] = __shfl_sync(0xffffffffu, own, (lane & ~7) | r) >> (lane & 7);
         }
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + s), (it / L::STAGES) & 1u, g));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL), it & 1u, g));
+      // -LSE log2e and -D of the tile's 128 queries
+      const float* nlse = reinterpret_cast<const float*>(smem + L::OFF_LD + s * 1024);
+      const float* ndlt = nlse + 128;
+      const bool diag = w.causal && qb == w.kb;
+      // only the diagonal tile of a causal mask and padding keys need masking;
+      // the choice must be warp-uniform (the TMEM loads and stores in both
+      // versions are warp-collective)
+      const bool masked = __any_sync(0xffffffffu, diag || !key_live);
+
+      // P for queries qoff + 4 k4 + [0, 4) of this key: exp2(S^T scale log2e - LSE log2e)
+      auto p_quad = [&](auto mask_tag, const uint32_t* sv, int qoff, int k4, float pv[4]) {
+        constexpr bool MASKED = decltype(mask_tag)::value;
+        const float4 lv = reinterpret_cast<const float4*>(nlse + qoff)[k4];
+        const float2 x01 = fma2(make_float2(__uint_as_float(sv[4 * k4]), __uint_as_float(sv[4 * k4 + 1])),
+                                sl2, make_float2(lv.x, lv.y));
+        const float2 x23 = fma2(make_float2(__uint_as_float(sv[4 * k4 + 2]), __uint_as_float(sv[4 * k4 + 3])),
+                                sl2, make_float2(lv.z, lv.w));
+        pv[0] = fast_exp2(x01.x);
+        pv[1] = fast_exp2(x01.y);
+        pv[2] = fast_exp2(x23.x);
+        pv[3] = fast_exp2(x23.y);
+        if constexpr (MASKED) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (!key_live || (diag && qoff + 4 * k4 + e < j)) pv[e] = 0.f;
+        }
+      };
+      // keep bit of query qoff + 4 k4 + e (= 8 g + r, g = k4 / 2, r = 4 (k4 % 2) + e)
+      auto keep_of = [&](int c, int k4, int e) -> bool {
+        return (kw[c][4 * (k4 & 1) + e] & (1u << (8 * (k4 >> 1)))) != 0u;
+      };
+
       if constexpr (kTwoPhase) {
         if (!ok) break;
         tc_fence_after();
-        const float* lse2 = reinterpret_cast<const float*>(smem + L::OFF_LD + s * 1024);
-        const float* dlt = lse2 + 128;
-        const bool diag = w.causal && qb == w.kb;
 
-        // ---- P phase: P = exp2(S^T scale log2e - LSE log2e), masked; the
-        // dropped P goes to TMEM for dV, the undropped P is kept as fp16 pairs
-        // (P <= 1 here) for the dS phase, negated where dropout drops the pair
-        // (P >= 0, and a P of 0 contributes nothing either way).
+        // ---- P phase: the dropped P goes to TMEM for dV, the undropped P is
+        // kept as fp16 pairs (P <= 1 here) for the dS phase, negated where
+        // dropout drops the pair (P >= 0, and a P of 0 contributes nothing
+        // either way).
         uint32_t pu[32];
+        auto p_phase = [&](auto mask_tag) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int qoff = 64 * wg + 32 * c;  // query offset within the tile
-          uint32_t sv[32];
-          tmem_ld32<0>(lane_addr + L::COL_S + qoff, sv);
-          tmem_wait_ld32<0>(sv);
-          const float4* l4 = reinterpret_cast<const float4*>(lse2 + qoff);
-          uint32_t ppk[16];
+          for (int c = 0; c < 2; ++c) {
+            const int qoff = 64 * wg + 32 * c;  // query offset within the tile
+            uint32_t sv[32];
+            tmem_ld32<0>(lane_addr + L::COL_S + qoff, sv);
+            tmem_wait_ld32<0>(sv);
+            uint32_t ppk[16];
 #pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 lv = l4[k4];
-            const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
-            float pe[4], pv4[4];
+            for (int k4 = 0; k4 < 8; ++k4) {
+              float pv[4], pe[4], pk4[4];
+              p_quad(mask_tag, sv, qoff, k4, pv);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k = 4 * k4 + e;
-              float pv = fast_exp2(fmaf(__uint_as_float(sv[k]), p.scale_log2, -lq[e]));
-              if (!key_live || (diag && qoff + k < j)) pv = 0.f;
-              float pd = pv, pkeep = pv;
-              if constexpr (DROPOUT) {
-                // query qoff + k, k = 4 k4 + e = 8 g + r with g = k4 / 2, r = 4 (k4 % 2) + e
-                const bool keep = (kw[c][4 * (k4 & 1) + e] >> (8 * (k4 >> 1) + (lane & 7))) & 1u;
-                pd = keep ? pv : 0.f;
-                pkeep = keep ? pv : -pv;
+              for (int e = 0; e < 4; ++e) {
+                pe[e] = pv[e];
+                pk4[e] = pv[e];
+                if constexpr (DROPOUT) {
+                  const bool keep = keep_of(c, k4, e);
+                  pe[e] = keep ? pv[e] : 0.f;
+                  pk4[e] = keep ? pv[e] : -pv[e];
+                }
               }
-              pe[e] = pd;
-              pv4[e] = pkeep;
+              ppk[2 * k4] = pack_bf16(pe[0], pe[1]);
+              ppk[2 * k4 + 1] = pack_bf16(pe[2], pe[3]);
+              pu[16 * c + 2 * k4] = pack_f16(pk4[0], pk4[1]);
+              pu[16 * c + 2 * k4 + 1] = pack_f16(pk4[2], pk4[3]);
             }
-            ppk[2 * k4] = pack_bf16(pe[0], pe[1]);
-            ppk[2 * k4 + 1] = pack_bf16(pe[2], pe[3]);
-            pu[16 * c + 2 * k4] = pack_f16(pv4[0], pv4[1]);
-            pu[16 * c + 2 * k4 + 1] = pack_f16(pv4[2], pv4[3]);
+            // P^T (bf16 pairs) into TMEM: queries [64 wg, 64 wg + 64) -> columns
+            // [64 wg, 64 wg + 32), inside this warpgroup's S^T columns already read
+            tmem_st16<0>(lane_addr + L::COL_S + 64 * wg + 16 * c, ppk);
           }
-          // P^T (bf16 pairs) into TMEM: queries [64 wg, 64 wg + 64) -> columns
-          // [64 wg, 64 wg + 32), inside this warpgroup's S^T columns already read
-          tmem_st16<0>(lane_addr + L::COL_S + 64 * wg + 16 * c, ppk);
-        }
+        };
+        if (masked) p_phase(std::true_type{});
+        else p_phase(std::false_type{});
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -552,29 +584,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t dv[32];
           tmem_ld32<0>(lane_addr + L::COL_DP + qoff, dv);
           tmem_wait_ld32<0>(dv);
-          const float4* d4 = reinterpret_cast<const float4*>(dlt + qoff);
+          const float2* d2 = reinterpret_cast<const float2*>(ndlt + qoff);
           uint32_t dpk[16];
 #pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 dl = d4[k4];
-            const float dq[4] = {dl.x, dl.y, dl.z, dl.w};
-            const float2 p01 = unpack_f16(pu[16 * c + 2 * k4]);
-            const float2 p23 = unpack_f16(pu[16 * c + 2 * k4 + 1]);
-            const float pv4[4] = {p01.x, p01.y, p23.x, p23.y};
-            float ds[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k = 4 * k4 + e;
-              float dpv = __uint_as_float(dv[k]);
-              float pv = pv4[e];
-              if constexpr (DROPOUT) {
-                dpv = (pv >= 0.f) ? dpv * p.drop_rscale : 0.f;  // negative: dropped
-                pv = fabsf(pv);
-              }
-              ds[e] = pv * (dpv - dq[e]);
+          for (int k2 = 0; k2 < 16; ++k2) {
+            float2 pv = unpack_f16(pu[16 * c + k2]);
+            float2 dp = make_float2(__uint_as_float(dv[2 * k2]), __uint_as_float(dv[2 * k2 + 1]));
+            float2 t;
+            if constexpr (DROPOUT) {
+              // negative P: dropped
+              dp.x = (pv.x >= 0.f) ? dp.x : 0.f;
+              dp.y = (pv.y >= 0.f) ? dp.y : 0.f;
+              pv = make_float2(fabsf(pv.x), fabsf(pv.y));
+              t = fma2(dp, rs2, d2[k2]);
+            } else {
+              t = add2(dp, d2[k2]);
             }
-            dpk[2 * k4] = pack_bf16(ds[0], ds[1]);
-            dpk[2 * k4 + 1] = pack_bf16(ds[2], ds[3]);
+            const float2 ds = mul2(pv, t);
+            dpk[k2] = pack_bf16(ds.x, ds.y);
           }
           // dS^T row j into the 128-byte-swizzled [keys][queries] buffer, panel wg
           const uint32_t row_addr = sbase + L::OFF_DS + wg * L::PANEL + j * 128;
@@ -595,59 +622,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DSEMPTY), (it - 1) & 1u, g));
         if (!ok) break;
         tc_fence_after();
-        const float* lse2 = reinterpret_cast<const float*>(smem + L::OFF_LD + s * 1024);
-        const float* dlt = lse2 + 128;
-        const bool diag = w.causal && qb == w.kb;
+        auto both = [&](auto mask_tag) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int qoff = 64 * wg + 32 * c;  // query offset within the tile
-          uint32_t sv[32], dv[32];
-          tmem_ld32<0>(lane_addr + L::COL_S + qoff, sv);
-          tmem_ld32<0>(lane_addr + L::COL_DP + qoff, dv);
-          tmem_wait_ld32<0>(sv);
-          tmem_wait_ld32<0>(dv);
-          const float4* l4 = reinterpret_cast<const float4*>(lse2 + qoff);
-          const float4* d4 = reinterpret_cast<const float4*>(dlt + qoff);
-          uint32_t ppk[16], dpk[16];
+          for (int c = 0; c < 2; ++c) {
+            const int qoff = 64 * wg + 32 * c;  // query offset within the tile
+            uint32_t sv[32], dv[32];
+            tmem_ld32<0>(lane_addr + L::COL_S + qoff, sv);
+            tmem_ld32<0>(lane_addr + L::COL_DP + qoff, dv);
+            tmem_wait_ld32<0>(sv);
+            tmem_wait_ld32<0>(dv);
+            const float4* d4 = reinterpret_cast<const float4*>(ndlt + qoff);
+            uint32_t ppk[16], dpk[16];
 #pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 lv = l4[k4];
-            const float4 dl = d4[k4];
-            const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
-            const float dq[4] = {dl.x, dl.y, dl.z, dl.w};
-            float pe[4], ds[4];
+            for (int k4 = 0; k4 < 8; ++k4) {
+              float pv[4], pe[4], dp[4];
+              p_quad(mask_tag, sv, qoff, k4, pv);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k = 4 * k4 + e;
-              float pv = fast_exp2(fmaf(__uint_as_float(sv[k]), p.scale_log2, -lq[e]));
-              if (!key_live || (diag && qoff + k < j)) pv = 0.f;
-              float dpv = __uint_as_float(dv[k]);
-              float pd = pv;
-              if constexpr (DROPOUT) {
-                // query qoff + k, k = 4 k4 + e = 8 g + r with g = k4 / 2, r = 4 (k4 % 2) + e
-                const bool keep = (kw[c][4 * (k4 & 1) + e] >> (8 * (k4 >> 1) + (lane & 7))) & 1u;
-                pd = keep ? pv : 0.f;
-                dpv = keep ? dpv * p.drop_rscale : 0.f;
+              for (int e = 0; e < 4; ++e) {
+                pe[e] = pv[e];
+                dp[e] = __uint_as_float(dv[4 * k4 + e]);
+                if constexpr (DROPOUT) {
+                  const bool keep = keep_of(c, k4, e);
+                  pe[e] = keep ? pv[e] : 0.f;
+                  dp[e] = keep ? dp[e] : 0.f;
+                }
               }
-              pe[e] = pd;
-              ds[e] = pv * (dpv - dq[e]);
+              const float4 dl = d4[k4];
+              float2 t01, t23;
+              if constexpr (DROPOUT) {
+                t01 = fma2(make_float2(dp[0], dp[1]), rs2, make_float2(dl.x, dl.y));
+                t23 = fma2(make_float2(dp[2], dp[3]), rs2, make_float2(dl.z, dl.w));
+              } else {
+                t01 = add2(make_float2(dp[0], dp[1]), make_float2(dl.x, dl.y));
+                t23 = add2(make_float2(dp[2], dp[3]), make_float2(dl.z, dl.w));
+              }
+              const float2 ds01 = mul2(make_float2(pv[0], pv[1]), t01);
+              const float2 ds23 = mul2(make_float2(pv[2], pv[3]), t23);
+              ppk[2 * k4] = pack_bf16(pe[0], pe[1]);
+              ppk[2 * k4 + 1] = pack_bf16(pe[2], pe[3]);
+              dpk[2 * k4] = pack_bf16(ds01.x, ds01.y);
+              dpk[2 * k4 + 1] = pack_bf16(ds23.x, ds23.y);
             }
-            ppk[2 * k4] = pack_bf16(pe[0], pe[1]);
-            ppk[2 * k4 + 1] = pack_bf16(pe[2], pe[3]);
-            dpk[2 * k4] = pack_bf16(ds[0], ds[1]);
-            dpk[2 * k4 + 1] = pack_bf16(ds[2], ds[3]);
-          }
-          // P^T (bf16 pairs) into TMEM: queries [64 wg, 64 wg + 64) -> columns [64 wg, 64 wg + 32)
-          tmem_st16<0>(lane_addr + L::COL_S + 64 * wg + 16 * c, ppk);
-          // dS^T row j into the 128-byte-swizzled [keys][queries] buffer, panel wg
-          const uint32_t row_addr = sbase + L::OFF_DS + wg * L::PANEL + j * 128;
+            // P^T (bf16 pairs) into TMEM: queries [64 wg, 64 wg + 64) -> columns [64 wg, 64 wg + 32)
+            tmem_st16<0>(lane_addr + L::COL_S + 64 * wg + 16 * c, ppk);
+            // dS^T row j into the 128-byte-swizzled [keys][queries] buffer, panel wg
+            const uint32_t row_addr = sbase + L::OFF_DS + wg * L::PANEL + j * 128;
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const uint32_t chunk = static_cast<uint32_t>(4 * c + ch) ^ static_cast<uint32_t>(j & 7);
-            st_shared_v4(row_addr + chunk * 16, dpk[4 * ch], dpk[4 * ch + 1], dpk[4 * ch + 2],
-                         dpk[4 * ch + 3]);
+            for (int ch = 0; ch < 4; ++ch) {
+              const uint32_t chunk = static_cast<uint32_t>(4 * c + ch) ^ static_cast<uint32_t>(j & 7);
+              st_shared_v4(row_addr + chunk * 16, dpk[4 * ch], dpk[4 * ch + 1], dpk[4 * ch + 2],
+                           dpk[4 * ch + 3]);
+            }
           }
-        }
+        };
+        if (masked) both(std::true_type{});
+        else both(std::false_type{});
         fence_proxy_async_smem();
         tmem_wait_st();
         tc_fence_before();

@@ -45,15 +45,19 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // and one CTA's set-up and epilogue hide under the other's main loop.
 template <int NQ>
 struct FwdRoles {
-  static constexpr int THREADS = NQ == 2 ? 384 : 192;
+  // warpgroup 0: producer (warp 0), MMA issuer (warp 1), two idle warps;
+  // then one softmax warpgroup per Q tile
+  static constexpr int THREADS = 128 * (1 + NQ);
   static constexpr int MIN_BLOCKS = NQ == 2 ? 1 : 2;
-  static constexpr int SOFTMAX_WARP0 = NQ == 2 ? 4 : 2;  // warps before it: producer, MMA, idle
-  static constexpr int LAUNCH_REGS = 168;                // registers per thread at launch (checked)
-  // NQ = 2: setmaxnreg moves registers from the first warpgroup (72 each) to
-  // the two softmax warpgroups (216 each), within the 384 x 168 of the launch.
-  static constexpr bool SPLIT_REGS = NQ == 2;
-  static constexpr uint32_t REGS_CTL = 72, REGS_SOFTMAX = 216;
-  static_assert(!SPLIT_REGS || 4 * 32 * (REGS_CTL + 2 * REGS_SOFTMAX) <= THREADS * LAUNCH_REGS,
+  static constexpr int SOFTMAX_WARP0 = 4;
+  static constexpr int LAUNCH_REGS = NQ == 2 ? 168 : 128;  // registers per thread at launch (checked)
+  // setmaxnreg moves registers from the first warpgroup to the softmax
+  // warpgroups, within the THREADS x LAUNCH_REGS of the launch.
+  static constexpr bool SPLIT_REGS = true;
+  static constexpr uint32_t REGS_CTL = NQ == 2 ? 72 : 56;
+  static constexpr uint32_t REGS_SOFTMAX = NQ == 2 ? 216 : 200;
+  static constexpr int MAX_PARTS = NQ == 2 ? 8 : 4;  // independent max / sum chains per row
+  static_assert(128 * (REGS_CTL + NQ * REGS_SOFTMAX) <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
 };
 
@@ -322,19 +326,6 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
       bool ok = true;
       for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1)) {
         if (!w.act(t, kb)) continue;
-        // Dropout keep bits of this row for keys [128 kb, 128 kb + 128): they do
-        // not depend on S, so they are drawn while the Q K^T MMA runs.
-        uint32_t keepw[4] = {0u, 0u, 0u, 0u};
-        if constexpr (DROPOUT) {
-          const uint32_t thr = p.drop_threshold;
-#pragma unroll
-          for (int gq = 0; gq < 16; ++gq) {  // keys 8 gq .. 8 gq + 7 of the tile
-            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(kb * 16 + gq),
-                                              static_cast<uint32_t>(i), static_cast<uint32_t>(w.h),
-                                              static_cast<uint32_t>(w.b), p.rk);
-            keepw[gq >> 2] |= keep_byte(rnd, thr) << (8 * (gq & 3));
-          }
-        }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + t), cnt & 1u, g));
         if (!ok) break;
         tc_fence_after();
@@ -351,23 +342,21 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
         const int j0 = kb * 128;
         const bool need_mask = (w.causal && kb == w.qb0 + t) || (j0 + 128 > w.kv_len);
         // row maximum with independent partial maxima (short dependency chains;
-        // as many as the register budget allows)
-        constexpr int kParts = R::SPLIT_REGS ? 8 : 2;
+        // as many as the register budget allows), two scores per max instruction
+        constexpr int kParts = R::MAX_PARTS;
         float mxp[kParts];
 #pragma unroll
         for (int u = 0; u < kParts; ++u) mxp[u] = -INFINITY;
         if (need_mask) {
           const int lim = w.causal ? min(w.kv_len - j0, i - j0 + 1) : (w.kv_len - j0);
 #pragma unroll
-          for (int j = 0; j < 128; ++j) {
-            const float v = (j < lim) ? __uint_as_float(sr[j]) : -INFINITY;
-            sr[j] = __float_as_uint(v);
-            mxp[j % kParts] = fmaxf(mxp[j % kParts], v);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 128; ++j) mxp[j % kParts] = fmaxf(mxp[j % kParts], __uint_as_float(sr[j]));
+          for (int j = 0; j < 128; ++j)
+            if (j >= lim) sr[j] = __float_as_uint(-INFINITY);
         }
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          mxp[c % kParts] =
+              fmax3(mxp[c % kParts], __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]));
         float mx = mxp[0];
 #pragma unroll
         for (int u = 1; u < kParts; ++u) mx = fmaxf(mx, mxp[u]);
@@ -375,31 +364,51 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
         const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         const float alpha = fast_exp2(m - m_use);  // 0 on the first tile, 1 if unchanged
-        float rsp[kParts];
+        // scaling and row sum on score pairs (one paired instruction each)
+        constexpr int kSums = kParts / 2;
+        float2 rsp[kSums];
 #pragma unroll
-        for (int u = 0; u < kParts; ++u) rsp[u] = 0.f;
+        for (int u = 0; u < kSums; ++u) rsp[u] = make_float2(0.f, 0.f);
+        const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-m_use, -m_use);
 #pragma unroll
-        for (int j = 0; j < 128; ++j) {
-          const float e = fast_exp2(fmaf(__uint_as_float(sr[j]), p.scale_log2, -m_use));
-          rsp[j % kParts] += e;
-          sr[j] = __float_as_uint(e);
+        for (int c = 0; c < 64; ++c) {
+          const float2 x =
+              fma2(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2, nm2);
+          const float2 e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          rsp[c % kSums] = add2(rsp[c % kSums], e);
+          sr[2 * c] = __float_as_uint(e.x);
+          sr[2 * c + 1] = __float_as_uint(e.y);
         }
-        float rs = rsp[0];
+        float rs = 0.f;
 #pragma unroll
-        for (int u = 1; u < kParts; ++u) rs += rsp[u];
+        for (int u = 0; u < kSums; ++u) rs += rsp[u].x + rsp[u].y;
         l = l * alpha + rs;
         m = m_new;
 
-        if constexpr (DROPOUT) {
-#pragma unroll
-          for (int j = 0; j < 128; ++j)
-            if (((keepw[j >> 5] >> (j & 31)) & 1u) == 0u) sr[j] = 0u;
-        }
-
         uint32_t pk[64];
+        if constexpr (DROPOUT) {
+          const uint32_t thr = p.drop_threshold;
+          const uint32_t thr_hi = thr << 16;
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          pk[c] = pack_bf16(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]));
+          for (int gq = 0; gq < 16; ++gq) {
+            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(kb * 16 + gq),
+                                              static_cast<uint32_t>(i), static_cast<uint32_t>(w.h),
+                                              static_cast<uint32_t>(w.b), p.rk);
+            const uint32_t wv[4] = {rnd.w0, rnd.w1, rnd.w2, rnd.w3};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int c = 4 * gq + u;
+              const float lo = ((wv[u] & 0xFFFFu) >= thr) ? __uint_as_float(sr[2 * c]) : 0.f;
+              const float hi = (wv[u] >= thr_hi) ? __uint_as_float(sr[2 * c + 1]) : 0.f;
+              pk[c] = pack_bf16(lo, hi);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            pk[c] = pack_bf16(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]));
+        }
         tmem_st32<0>(s_addr + 0, pk);
         tmem_st32<32>(s_addr + 32, pk);
 
@@ -415,7 +424,12 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
               tmem_ld32<0>(o_addr + 32 * c, orr);
               tmem_wait_ld32<0>(orr);
 #pragma unroll
-              for (int k = 0; k < 32; ++k) orr[k] = __float_as_uint(__uint_as_float(orr[k]) * alpha);
+              for (int k = 0; k < 16; ++k) {
+                const float2 o2 = mul2(make_float2(__uint_as_float(orr[2 * k]), __uint_as_float(orr[2 * k + 1])),
+                                       make_float2(alpha, alpha));
+                orr[2 * k] = __float_as_uint(o2.x);
+                orr[2 * k + 1] = __float_as_uint(o2.y);
+              }
               tmem_st32<0>(o_addr + 32 * c, orr);
             }
           }
@@ -449,7 +463,11 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
           uint32_t ob[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k)
-            ob[k] = pack_bf16(__uint_as_float(orr[2 * k]) * inv, __uint_as_float(orr[2 * k + 1]) * inv);
+          {
+            const float2 o2 = mul2(make_float2(__uint_as_float(orr[2 * k]), __uint_as_float(orr[2 * k + 1])),
+                                   make_float2(inv, inv));
+            ob[k] = pack_bf16(o2.x, o2.y);
+          }
           if (row_ok) {
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll

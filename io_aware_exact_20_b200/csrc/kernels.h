@@ -47,8 +47,8 @@ struct BwdParams {
   void* dq;                   // bf16 [B,H,N,d]
   void* dk;                   // bf16 [B,H,N,d]
   void* dv;                   // bf16 [B,H,N,d]
-  float* ws_lse2;             // fp32 [B*H][Npad]  LSE * log2(e), +inf where no key
-  float* ws_delta;            // fp32 [B*H][Npad]  sum_c dO_ic O_ic
+  float* ws_lse2;             // fp32 [B*H][Npad]  -LSE * log2(e), -inf where no key
+  float* ws_delta;            // fp32 [B*H][Npad]  -sum_c dO_ic O_ic
   float* ws_dq;               // fp32 [B*H][Npad][d] dQ accumulators (unscaled)
   const int32_t* seqlens;
   const uint8_t* block_mask;
