@@ -356,8 +356,9 @@ def run_ours(args):
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
-    if fa.last_device_status() != 0:
-        raise RuntimeError("device status after warm-up is not ok")
+    st = fa.last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up is {st}, not ok")
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     if world > 1:
