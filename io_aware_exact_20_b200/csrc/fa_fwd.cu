@@ -1,23 +1,33 @@
 // Forward pass of exact attention on sm_100a.
 //
-// Work unit: one (b, h) and 256 query rows, held as two 128-row Q tiles that
-// share every K/V tile the CTA loads.  The CTA walks the K/V tiles of its head
-// that at least one of its Q tiles needs (tiles that are fully masked by the
-// causal mask, the key lengths or the block mask are neither loaded nor
-// computed).  Per K/V tile and per active Q tile t:
+// Work unit: one (b, h) and NQ 128-row Q tiles (NQ = 2 at d = 128, 1 at
+// d = 64) that share every K/V tile the CTA loads.  The CTA walks the K/V tiles
+// of its head that at least one of its Q tiles needs (tiles that are fully
+// masked by the causal mask, the key lengths or the block mask are neither
+// loaded nor computed).
 //
-//   S_t = Q_t K^T           tcgen05.mma, bf16 x bf16 -> fp32 in TMEM
-//   P_t = exp2(S_t * scale * log2e - m_t)   online softmax, one thread per row
-//   O_t += P_t V            tcgen05.mma with P_t read from TMEM
+// Each Q tile is processed by KS softmax streams (KS = 2 at d = 64, else 1);
+// with KS = 2, stream h of a Q tile owns keys [128 kb + 64 h, 128 kb + 64 h + 64)
+// of every K/V tile kb, with KS = 1 the whole tile, and each stream keeps its
+// own running maximum, row sum and O accumulator.  Per K/V tile and active
+// stream:
 //
-// Roles, two Q tiles per CTA (384 threads):
-//   warp 0       TMA producer: Q tiles once, then K/V tiles into a ring
-//   warp 1       TMEM allocator and single-thread MMA issuer
-//   warps 2-3    idle
-//   warps 4-7    softmax for Q tile 0   (thread = row, TMEM lanes 0..127)
-//   warps 8-11   softmax for Q tile 1
-// One Q tile per CTA (192 threads, two CTAs per SM): warps 0 and 1 as above,
-// warps 2-5 softmax.
+//   S = Q_t K_h^T           tcgen05.mma, bf16 x bf16 -> fp32 in TMEM
+//   P = exp2(S * scale * log2e - m)   online softmax, one thread per row
+//   O_h += P V_h            tcgen05.mma with P read from TMEM
+//
+// and at the end the streams of a Q tile merge: with M = max_h m_h,
+// O = sum_h 2^(m_h - M) O_h / sum_h 2^(m_h - M) l_h (the softmax of a key range
+// split in two, recombined from per-part statistics as in the pages' tiling
+// section).  The d = 64 forward is limited by how well the softmax warps hide
+// their latencies, and the split gives each SM sub-partition more of them; at
+// d = 128 the O accumulators leave no TMEM for it.
+//
+// Roles:
+//   warp 0            TMA producer: Q tiles once, then K/V tiles into a ring
+//   warp 1            TMEM allocator and single-thread MMA issuer
+//   warps 2-3         idle
+//   warpgroup 1 + s   softmax stream s (thread = row, TMEM lanes 0..127)
 //
 // The running maximum m is only moved when a new block raises it by more than
 // 8 (in log2 units); until then exp2 values may reach 2^8, and O and the row
@@ -25,8 +35,9 @@
 // LSE = ln2 * (m + log2 l) are unchanged (the online-softmax rescaling of the
 // tiling section of the pages, applied lazily).
 //
-// TMEM columns: S/P of tile t at [128 t, 128 t + 128) (P packed as bf16 pairs in
-// the first 64 columns), O of tile t at [256 + D t, 256 + D t + D).
+// TMEM columns: S/P of stream s at [KW s, KW s + KW) (KW = 128 / KS keys; P
+// packed as bf16 pairs in the first KW / 2 columns), O of stream s at
+// [KW NS + D s, KW NS + D s + D), NS = NQ KS streams.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -39,52 +50,63 @@ namespace {
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-// Q tiles per CTA.  Two (the default) share every K/V tile between two 128-row
-// Q tiles, with the two softmax warpgroups ping-ponging on the tensor core.
-// One (d = 64, short sequences) halves the CTA so that two CTAs share an SM
-// and one CTA's set-up and epilogue hide under the other's main loop.
-template <int NQ>
-struct FwdRoles {
-  // warpgroup 0: producer (warp 0), MMA issuer (warp 1), two idle warps;
-  // then one softmax warpgroup per Q tile
-  static constexpr int THREADS = 128 * (1 + NQ);
+// Per head dimension:
+//   d = 128: two Q tiles per CTA (NQ = 2) share every K/V tile, one softmax
+//            stream each (KS = 1); the four accumulators fill TMEM.
+//   d = 64:  one Q tile per CTA (NQ = 1) and two CTAs per SM, the tile's keys
+//            split between two softmax streams (KS = 2): four softmax
+//            warpgroups per SM either way, but each CTA walks only the K/V
+//            tiles its own Q tile needs (which matters under block masks) and
+//            one CTA's set-up and epilogue hide under the other's main loop.
+template <int D>
+struct FwdCfg {
+  static constexpr int NQ = D == 64 ? 1 : 2;  // Q tiles per CTA
+  static constexpr int KS = D == 64 ? 2 : 1;  // softmax streams per Q tile
+  static constexpr int NS = NQ * KS;          // softmax streams = softmax warpgroups
+  static constexpr int KW = 128 / KS;         // keys per stream per K/V tile
+  static constexpr int THREADS = 128 * (1 + NS);
   static constexpr int MIN_BLOCKS = NQ == 2 ? 1 : 2;
-  static constexpr int SOFTMAX_WARP0 = 4;
-  static constexpr int LAUNCH_REGS = NQ == 2 ? 168 : 128;  // registers per thread at launch (checked)
-  // setmaxnreg moves registers from the first warpgroup to the softmax
-  // warpgroups, within the THREADS x LAUNCH_REGS of the launch.
-  static constexpr bool SPLIT_REGS = true;
-  static constexpr uint32_t REGS_CTL = NQ == 2 ? 72 : 56;
-  static constexpr uint32_t REGS_SOFTMAX = NQ == 2 ? 216 : 200;
-  static constexpr int MAX_PARTS = NQ == 2 ? 8 : 4;  // independent max / sum chains per row
-  static_assert(128 * (REGS_CTL + NQ * REGS_SOFTMAX) <= THREADS * LAUNCH_REGS,
+  // registers per thread at launch (checked before the first launch): the
+  // largest multiple of 8 that MIN_BLOCKS CTAs of THREADS threads can hold
+  static constexpr int LAUNCH_REGS = (65536 / (THREADS * MIN_BLOCKS)) & ~7;
+  // setmaxnreg moves registers from warpgroup 0 (producer, MMA issuer) to the
+  // softmax warpgroups, within the THREADS x LAUNCH_REGS of the launch
+  static constexpr uint32_t REGS_CTL = KS == 1 ? 72 : 32;
+  static constexpr uint32_t REGS_SOFTMAX =
+      ((THREADS * LAUNCH_REGS - 128 * REGS_CTL) / (128 * NS)) & ~7u;
+  static constexpr int MAX_PARTS = KW == 128 ? 8 : 4;  // max / sum chains per row
+  static_assert(128 * (REGS_CTL + NS * REGS_SOFTMAX) <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
+  static_assert(REGS_SOFTMAX <= 256 && REGS_SOFTMAX >= 96, "softmax register budget");
 };
 
-template <int D, int NQ>
+template <int D>
 struct FwdLayout {
+  using C = FwdCfg<D>;
+  static constexpr int NQ = C::NQ;
   static constexpr int PANELS = D / 64;                 // 64-column, 128-byte-swizzled panels
   static constexpr uint32_t PANEL = 128u * 128u;        // bytes of one [128 rows][64 cols] panel
   static constexpr uint32_t TILE = PANEL * PANELS;      // bytes of one 128-row tile
-  static constexpr int STAGES = NQ == 1 ? 2 : (D == 64 ? 4 : 2);  // K/V ring depth
+  static constexpr int STAGES = 2;                      // K/V ring depth
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_KV = NQ * TILE;
-  static constexpr uint32_t OFF_BAR = OFF_KV + STAGES * 2 * TILE;
+  static constexpr uint32_t OFF_XCH = OFF_KV + STAGES * 2 * TILE;  // [NS][128] (m, l) for the merge
+  static constexpr uint32_t OFF_BAR = OFF_XCH + (C::KS > 1 ? C::NS * 128 * 8 : 0);
   static constexpr int B_QFULL = 0;
   static constexpr int B_KFULL = 2;
   static constexpr int B_VFULL = B_KFULL + STAGES;
   static constexpr int B_KVEMPTY = B_VFULL + STAGES;
-  static constexpr int B_SFULL = B_KVEMPTY + STAGES;
-  static constexpr int B_PFULL = B_SFULL + 2;
-  static constexpr int B_ODONE = B_PFULL + 2;
-  static constexpr int B_DRAIN = B_ODONE + 2;
+  static constexpr int B_SFULL = B_KVEMPTY + STAGES;  // per stream
+  static constexpr int B_PFULL = B_SFULL + C::NS;     // per stream
+  static constexpr int B_ODONE = B_PFULL + C::NS;     // per stream
+  static constexpr int B_DRAIN = B_ODONE + C::NS;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16;
-  static constexpr uint32_t O_COL = 128 * NQ;
   static constexpr uint32_t TMEM_COLS = NQ == 2 ? 512 : 256;
+  static constexpr uint32_t O_COL = C::KW * C::NS;
   static_assert(SMEM <= (NQ == 2 ? 232448u : 113u * 1024u), "shared memory budget");
-  static_assert(O_COL + NQ * D <= TMEM_COLS, "TMEM budget");
+  static_assert(O_COL + C::NS * D <= TMEM_COLS, "TMEM budget");
 };
 
 // Which (Q tile, K/V tile) pairs of this CTA take part.
@@ -101,6 +123,11 @@ struct FwdWork {
     if (bm != nullptr && bm[static_cast<size_t>(qb) * nblk + kb] == 0) return false;
     return true;
   }
+  // stream (Q tile t, key part hp of kw keys): also skipped when all its keys
+  // are past the key length
+  __device__ __forceinline__ bool act_s(int t, int hp, int kw, int kb) const {
+    return act(t, kb) && kb * 128 + hp * kw < kv_len;
+  }
   __device__ __forceinline__ bool any(int kb) const { return act(0, kb) || act(1, kb); }
   __device__ __forceinline__ int next(int kb) const {
     while (kb < kb_end && !any(kb)) ++kb;
@@ -108,12 +135,19 @@ struct FwdWork {
   }
 };
 
-template <int D, bool DROPOUT, int NQ>
-__global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCKS)
+// Barrier `kId` among the 256 threads of the two softmax warpgroups of a Q tile.
+template <int kId>
+__device__ __forceinline__ void named_bar_sync() {
+  asm volatile("bar.sync %0, 256;" ::"n"(kId) : "memory");
+}
+
+template <int D, bool DROPOUT>
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdLayout<D, NQ>;
-  using R = FwdRoles<NQ>;
+  using L = FwdLayout<D>;
+  using C = FwdCfg<D>;
+  constexpr int NQ = C::NQ, NS = C::NS, KS = C::KS, KW = C::KW;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {  // the swizzled layouts need 1024-byte alignment
@@ -151,11 +185,11 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
 
   if (threadIdx.x == 0) {
     *abort_flag = 0u;
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(bar(L::B_QFULL + t), 1);
-      mbar_init(bar(L::B_SFULL + t), 1);
-      mbar_init(bar(L::B_PFULL + t), 4);  // one arrival per softmax warp
-      mbar_init(bar(L::B_ODONE + t), 1);
+    for (int t = 0; t < 2; ++t) mbar_init(bar(L::B_QFULL + t), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(L::B_SFULL + s), 1);
+      mbar_init(bar(L::B_PFULL + s), 4);  // one arrival per softmax warp
+      mbar_init(bar(L::B_ODONE + s), 1);
     }
     for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(bar(L::B_KFULL + s), 1);
@@ -176,8 +210,8 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
 
   // Each role runs inside the branch that sets its register budget, so that
   // the compiler allocates every role's code under its own limit.
-  if (warp < R::SOFTMAX_WARP0) {
-  if constexpr (R::SPLIT_REGS) setmaxnreg_dec<R::REGS_CTL>();
+  if (warp < 4) {
+  setmaxnreg_dec<C::REGS_CTL>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
@@ -219,27 +253,32 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
+      // the stream loops unroll while they are short (keeps the issuer's
+      // registers in check with four streams)
+      constexpr int kUnrollS = KS == 1 ? NS : 1;
+      constexpr uint32_t kIdS = idesc_bf16(128, KW, false, false);
       constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);
-      bool q_ready[2] = {false, false};
-      bool o_init[2] = {false, false};
-      uint32_t p_cnt[2] = {0u, 0u};
+      uint32_t q_ready = 0u;  // bit t: Q tile t has landed
+      uint32_t o_init = 0u;  // bit s: stream s has accumulated into its O
+      uint32_t p_par = 0u;   // bit s: parity of stream s's next P-full phase
       bool ok = true;
 
-      auto issue_s = [&](int t, uint32_t kaddr) {
-        const uint32_t qaddr = sbase + L::OFF_Q + t * L::TILE;
+      // S of stream s = (Q tile s / KS, key part s % KS) for the K tile at kaddr
+      auto issue_s = [&](int s, uint32_t kaddr) {
+        const uint32_t qaddr = sbase + L::OFF_Q + (s / KS) * L::TILE;
+        const uint32_t kpart = kaddr + static_cast<uint32_t>((s % KS) * KW) * 128u;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::PANEL + (kk & 3) * 32;
-          mma_ss(tmem + 128 * t, sdesc_sw128(qaddr + off, 16, 1024),
-                 sdesc_sw128(kaddr + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + KW * s, sdesc_sw128(qaddr + off, 16, 1024),
+                 sdesc_sw128(kpart + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(L::B_SFULL + t));
+        mma_commit(bar(L::B_SFULL + s));
       };
       auto ensure_q = [&](int t) -> bool {
-        if (q_ready[t]) return true;
+        if ((q_ready >> t) & 1u) return true;
         if (!mbar_wait(bar(L::B_QFULL + t), 0, g)) return false;
-        q_ready[t] = true;
+        q_ready |= 1u << t;
         return true;
       };
 
@@ -247,41 +286,46 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
       int it = 0;
       if (kb < w.kb_end) {
         ok = mbar_wait(bar(L::B_KFULL + 0), 0, g);
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!w.act(t, kb)) continue;
-          ok = ensure_q(t);
+#pragma unroll(kUnrollS)
+        for (int s = 0; s < NS; ++s) {
+          if (!ok || !w.act_s(s / KS, s % KS, KW, kb)) continue;
+          ok = ensure_q(s / KS);
           if (ok) {
             tc_fence_after();
-            issue_s(t, sbase + L::OFF_KV);
+            issue_s(s, sbase + L::OFF_KV);
           }
         }
       }
       while (ok && kb < w.kb_end) {
-        const int s = it % L::STAGES;
+        const int st = it % L::STAGES;
         const uint32_t ph = (it / L::STAGES) & 1u;
         const int kbn = w.next(kb + 1);
         const int sn = (it + 1) % L::STAGES;
         const uint32_t phn = ((it + 1) / L::STAGES) & 1u;
         bool kn_ready = false;
-        if (!mbar_wait(bar(L::B_VFULL + s), ph, g)) break;
-        const uint32_t vaddr = sbase + L::OFF_KV + s * 2 * L::TILE + L::TILE;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (w.act(t, kb)) {
-            if (!mbar_wait(bar(L::B_PFULL + t), p_cnt[t] & 1u, g)) {
+        if (!mbar_wait(bar(L::B_VFULL + st), ph, g)) break;
+        const uint32_t vaddr = sbase + L::OFF_KV + st * 2 * L::TILE + L::TILE;
+#pragma unroll(kUnrollS)
+        for (int s = 0; s < NS; ++s) {
+          if (!ok) break;
+          if (w.act_s(s / KS, s % KS, KW, kb)) {
+            if (!mbar_wait(bar(L::B_PFULL + s), (p_par >> s) & 1u, g)) {
               ok = false;
               break;
             }
-            ++p_cnt[t];
+            p_par ^= 1u << s;
             tc_fence_after();
+            // this stream's keys are rows [KW (s % KS), KW (s % KS) + KW) of the V tile
+            const uint32_t vpart = vaddr + static_cast<uint32_t>((s % KS) * KW) * 128u;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tmem + L::O_COL + D * t, tmem + 128 * t + 8 * kk,
-                     sdesc_sw128(vaddr + kk * 2048, L::PANEL, 1024), kIdPV,
-                     (o_init[t] || kk > 0) ? 1u : 0u);
-            o_init[t] = true;
-            mma_commit(bar(L::B_ODONE + t));
+            for (int kk = 0; kk < KW / 16; ++kk)
+              mma_ts(tmem + L::O_COL + D * s, tmem + KW * s + 8 * kk,
+                     sdesc_sw128(vpart + kk * 2048, L::PANEL, 1024), kIdPV,
+                     (((o_init >> s) & 1u) != 0u || kk > 0) ? 1u : 0u);
+            o_init |= 1u << s;
+            mma_commit(bar(L::B_ODONE + s));
           }
-          if (kbn < w.kb_end && w.act(t, kbn)) {
+          if (kbn < w.kb_end && w.act_s(s / KS, s % KS, KW, kbn)) {
             if (!kn_ready) {
               if (!mbar_wait(bar(L::B_KFULL + sn), phn, g)) {
                 ok = false;
@@ -289,16 +333,16 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
               }
               kn_ready = true;
             }
-            if (!ensure_q(t)) {
+            if (!ensure_q(s / KS)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_s(t, sbase + L::OFF_KV + sn * 2 * L::TILE);
+            issue_s(s, sbase + L::OFF_KV + sn * 2 * L::TILE);
           }
         }
         if (!ok) break;
-        mma_commit(bar(L::B_KVEMPTY + s));
+        mma_commit(bar(L::B_KVEMPTY + st));
         kb = kbn;
         ++it;
       }
@@ -306,55 +350,62 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
       mma_commit(bar(L::B_DRAIN));
       mbar_wait_drain(bar(L::B_DRAIN), 0, 1000000000ull);
       for (int t = 0; t < 2; ++t)
-        if ((t == 0 || w.exists1) && !q_ready[t]) mbar_wait_drain(bar(L::B_QFULL + t), 0, 100000000ull);
+        if ((t == 0 || w.exists1) && !((q_ready >> t) & 1u))
+          mbar_wait_drain(bar(L::B_QFULL + t), 0, 100000000ull);
     }
   }
   } else {
-    if constexpr (R::SPLIT_REGS) setmaxnreg_inc<R::REGS_SOFTMAX>();
+    setmaxnreg_inc<C::REGS_SOFTMAX>();
     // -------------------------------------------------------------- softmax
-    const int t = (warp - R::SOFTMAX_WARP0) >> 2;
+    const int s = (warp - 4) >> 2;  // stream
+    const int t = s / KS;           // Q tile
+    const int hp = s % KS;          // key part
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const int i = w.q0 + 128 * t + r;
     if (t == 0 || w.exists1) {
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-      const uint32_t s_addr = lane_addr + 128 * t;
-      const uint32_t o_addr = lane_addr + L::O_COL + D * t;
+      const uint32_t s_addr = lane_addr + KW * s;
+      const uint32_t o_addr = lane_addr + L::O_COL + D * s;
       float m = -INFINITY;  // reference maximum, log2 units of scaled scores
       float l = 0.f;        // row sum of exp2(x - m)
       uint32_t cnt = 0;     // active K/V tiles processed so far
       bool ok = true;
       for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1)) {
-        if (!w.act(t, kb)) continue;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + t), cnt & 1u, g));
+        if (!w.act_s(t, hp, KW, kb)) continue;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + s), cnt & 1u, g));
         if (!ok) break;
         tc_fence_after();
-        uint32_t sr[128];
+        uint32_t sr[KW];
         tmem_ld32<0>(s_addr + 0, sr);
         tmem_ld32<32>(s_addr + 32, sr);
-        tmem_ld32<64>(s_addr + 64, sr);
-        tmem_ld32<96>(s_addr + 96, sr);
+        if constexpr (KW == 128) {
+          tmem_ld32<64>(s_addr + 64, sr);
+          tmem_ld32<96>(s_addr + 96, sr);
+        }
         tmem_wait_ld32<0>(sr);
         tmem_wait_ld32<32>(sr);
-        tmem_wait_ld32<64>(sr);
-        tmem_wait_ld32<96>(sr);
+        if constexpr (KW == 128) {
+          tmem_wait_ld32<64>(sr);
+          tmem_wait_ld32<96>(sr);
+        }
 
-        const int j0 = kb * 128;
-        const bool need_mask = (w.causal && kb == w.qb0 + t) || (j0 + 128 > w.kv_len);
+        const int j0 = kb * 128 + KW * hp;  // first key of this block
+        const bool need_mask = (w.causal && kb == w.qb0 + t) || (j0 + KW > w.kv_len);
         // row maximum with independent partial maxima (short dependency chains;
         // as many as the register budget allows), two scores per max instruction
-        constexpr int kParts = R::MAX_PARTS;
+        constexpr int kParts = C::MAX_PARTS;
         float mxp[kParts];
 #pragma unroll
         for (int u = 0; u < kParts; ++u) mxp[u] = -INFINITY;
         if (need_mask) {
           const int lim = w.causal ? min(w.kv_len - j0, i - j0 + 1) : (w.kv_len - j0);
 #pragma unroll
-          for (int j = 0; j < 128; ++j)
+          for (int j = 0; j < KW; ++j)
             if (j >= lim) sr[j] = __float_as_uint(-INFINITY);
         }
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < KW / 2; ++c)
           mxp[c % kParts] =
               fmax3(mxp[c % kParts], __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]));
         float mx = mxp[0];
@@ -372,7 +423,7 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
         const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 nm2 = make_float2(-m_use, -m_use);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < KW / 2; ++c) {
           const float2 x =
               fma2(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2, nm2);
           const float2 e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
@@ -386,13 +437,17 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
         l = l * alpha + rs;
         m = m_new;
 
-        uint32_t pk[64];
+        uint32_t pk[KW / 2];
         if constexpr (DROPOUT) {
+          // Philox call gq of this row covers keys j0 + 8 gq .. j0 + 8 gq + 7;
+          // its word u holds the uniforms of keys j0 + 8 gq + 2u (low half) and
+          // j0 + 8 gq + 2u + 1 (high half), i.e. exactly bf16 pair 4 gq + u.
+          // high half >= t  <=>  word >= t << 16.
           const uint32_t thr = p.drop_threshold;
           const uint32_t thr_hi = thr << 16;
 #pragma unroll
-          for (int gq = 0; gq < 16; ++gq) {
-            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(kb * 16 + gq),
+          for (int gq = 0; gq < KW / 8; ++gq) {
+            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>((j0 >> 3) + gq),
                                               static_cast<uint32_t>(i), static_cast<uint32_t>(w.h),
                                               static_cast<uint32_t>(w.b), p.rk);
             const uint32_t wv[4] = {rnd.w0, rnd.w1, rnd.w2, rnd.w3};
@@ -406,15 +461,15 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < KW / 2; ++c)
             pk[c] = pack_bf16(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]));
         }
         tmem_st32<0>(s_addr + 0, pk);
-        tmem_st32<32>(s_addr + 32, pk);
+        if constexpr (KW == 128) tmem_st32<32>(s_addr + 32, pk);
 
         if (cnt > 0) {
           // previous O += P V is complete (it precedes the S MMA just consumed)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ODONE + t), (cnt - 1) & 1u, g));
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ODONE + s), (cnt - 1) & 1u, g));
           if (!ok) break;
           tc_fence_after();
           if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -437,46 +492,102 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_PFULL + t));
+        if (lane == 0) mbar_arrive(bar(L::B_PFULL + s));
         ++cnt;
       }
 
       // ------------------------------------------------------------ epilogue
       if (ok && cnt > 0)
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ODONE + t), (cnt - 1) & 1u, g));
-      if (ok) {
-        tc_fence_after();
-        const bool row_ok = i < p.N;
-        const float inv = (l > 0.f) ? p.drop_rscale / l : 0.f;
-        __nv_bfloat16* orow =
-            reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(w.bh) * p.N + i) * D;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ODONE + s), (cnt - 1) & 1u, g));
+      const bool row_ok = i < p.N;
+      __nv_bfloat16* orow =
+          reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(w.bh) * p.N + i) * D;
+      if constexpr (KS == 1) {
+        if (ok) {
+          tc_fence_after();
+          const float inv = (l > 0.f) ? p.drop_rscale / l : 0.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t orr[32];
-          if (cnt > 0) {
-            tmem_ld32<0>(o_addr + 32 * c, orr);
-            tmem_wait_ld32<0>(orr);
-          } else {
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            if (cnt > 0) {
+              tmem_ld32<0>(o_addr + 32 * c, orr);
+              tmem_wait_ld32<0>(orr);
+            } else {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) orr[k] = 0u;
+              for (int k = 0; k < 32; ++k) orr[k] = 0u;
+            }
+            uint32_t ob[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float2 o2 = mul2(make_float2(__uint_as_float(orr[2 * k]), __uint_as_float(orr[2 * k + 1])),
+                                     make_float2(inv, inv));
+              ob[k] = pack_bf16(o2.x, o2.y);
+            }
+            if (row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                dst[k] = make_uint4(ob[4 * k], ob[4 * k + 1], ob[4 * k + 2], ob[4 * k + 3]);
+            }
           }
-          uint32_t ob[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-          {
-            const float2 o2 = mul2(make_float2(__uint_as_float(orr[2 * k]), __uint_as_float(orr[2 * k + 1])),
-                                   make_float2(inv, inv));
-            ob[k] = pack_bf16(o2.x, o2.y);
-          }
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              dst[k] = make_uint4(ob[4 * k], ob[4 * k + 1], ob[4 * k + 2], ob[4 * k + 3]);
-          }
+          if (row_ok)
+            p.lse[static_cast<size_t>(w.bh) * p.N + i] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
         }
-        if (row_ok)
-          p.lse[static_cast<size_t>(w.bh) * p.N + i] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+      } else {
+        // Merge the two streams of this Q tile.  A stream that processed no
+        // block never wrote its O accumulator: it zeroes it first.  Both
+        // warpgroups publish their row statistics and meet at a named barrier
+        // (reached on every path: every wait above is bounded); then each
+        // writes D / 2 output columns from both streams' accumulators.
+        if (cnt == 0) {
+          uint32_t z[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) z[k] = 0u;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tmem_st32<0>(o_addr + 32 * c, z);
+          tmem_wait_st();
+        }
+        float2* xch = reinterpret_cast<float2*>(smem + L::OFF_XCH);
+        xch[s * 128 + r] = make_float2(m, l);
+        tc_fence_before();
+        if (t == 0) named_bar_sync<1>();
+        else named_bar_sync<2>();
+        tc_fence_after();
+        const float2 st0 = xch[(KS * t) * 128 + r];
+        const float2 st1 = xch[(KS * t + 1) * 128 + r];
+        if (ok) {
+          const float mm = fmaxf(st0.x, st1.x);
+          const float mref = (mm == -INFINITY) ? 0.f : mm;
+          const float f0 = fast_exp2(st0.x - mref), f1 = fast_exp2(st1.x - mref);
+          const float lt = st0.y * f0 + st1.y * f1;
+          const float inv = (lt > 0.f) ? p.drop_rscale / lt : 0.f;
+          const float2 g0 = make_float2(f0 * inv, f0 * inv), g1 = make_float2(f1 * inv, f1 * inv);
+          const uint32_t oc0 = lane_addr + L::O_COL + D * (KS * t) + (D / 2) * hp;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t a[32], bb[32];
+            tmem_ld32<0>(oc0 + 32 * c, a);
+            tmem_ld32<0>(oc0 + D + 32 * c, bb);
+            tmem_wait_ld32<0>(a);
+            tmem_wait_ld32<0>(bb);
+            uint32_t ob[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float2 x0 = make_float2(__uint_as_float(a[2 * k]), __uint_as_float(a[2 * k + 1]));
+              const float2 x1 = make_float2(__uint_as_float(bb[2 * k]), __uint_as_float(bb[2 * k + 1]));
+              const float2 o2 = fma2(x1, g1, mul2(x0, g0));
+              ob[k] = pack_bf16(o2.x, o2.y);
+            }
+            if (row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + (D / 2) * hp + 32 * c);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                dst[k] = make_uint4(ob[4 * k], ob[4 * k + 1], ob[4 * k + 2], ob[4 * k + 3]);
+            }
+          }
+          if (row_ok && hp == 0)
+            p.lse[static_cast<size_t>(w.bh) * p.N + i] = (lt > 0.f) ? (mref + log2f(lt)) * kLn2 : -INFINITY;
+        }
       }
     }
   }
@@ -490,12 +601,12 @@ __global__ void __launch_bounds__(FwdRoles<NQ>::THREADS, FwdRoles<NQ>::MIN_BLOCK
   }
 }
 
-template <int D, bool DROPOUT, int NQ>
+template <int D, bool DROPOUT>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, cudaStream_t stream) {
-  using L = FwdLayout<D, NQ>;
-  using R = FwdRoles<NQ>;
-  auto kern = fwd_kernel<D, DROPOUT, NQ>;
+  using L = FwdLayout<D>;
+  using C = FwdCfg<D>;
+  auto kern = fwd_kernel<D, DROPOUT>;
   // The setmaxnreg split is sized for exactly LAUNCH_REGS registers per thread
   // at launch; with any other count an increase could wait forever.
   static int regs_checked = 0;
@@ -503,34 +614,27 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     cudaFuncAttributes attr{};
     cudaError_t e = cudaFuncGetAttributes(&attr, kern);
     if (e != cudaSuccess) return e;
-    if (R::SPLIT_REGS && attr.numRegs != R::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+    if (attr.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
     regs_checked = 1;
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::SMEM));
   if (e != cudaSuccess) return e;
-  const unsigned tiles = static_cast<unsigned>((p.N + 128 * NQ - 1) / (128 * NQ));
+  const unsigned tiles = static_cast<unsigned>((p.N + 128 * C::NQ - 1) / (128 * C::NQ));
   const unsigned bh = static_cast<unsigned>(p.B * p.H);
   const dim3 grid = p.tiles_major ? dim3(bh, tiles) : dim3(tiles, bh);
-  kern<<<grid, R::THREADS, L::SMEM, stream>>>(tq, tk, tv, p);
+  kern<<<grid, C::THREADS, L::SMEM, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
-
-// One Q tile per CTA (two CTAs per SM) pays off when the sequences are short,
-// where each CTA has few K/V tiles to amortise its set-up and epilogue.
-inline bool one_tile_per_cta(int d, int N) { return d == 64 && N <= 4096; }
 
 }  // namespace
 
 cudaError_t launch_fwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, cudaStream_t stream) {
-  if (d == 64 && one_tile_per_cta(d, p.N))
-    return dropout ? launch_fwd_t<64, true, 1>(tq, tk, tv, p, stream)
-                   : launch_fwd_t<64, false, 1>(tq, tk, tv, p, stream);
-  if (d == 64) return dropout ? launch_fwd_t<64, true, 2>(tq, tk, tv, p, stream)
-                              : launch_fwd_t<64, false, 2>(tq, tk, tv, p, stream);
-  if (d == 128) return dropout ? launch_fwd_t<128, true, 2>(tq, tk, tv, p, stream)
-                               : launch_fwd_t<128, false, 2>(tq, tk, tv, p, stream);
+  if (d == 64) return dropout ? launch_fwd_t<64, true>(tq, tk, tv, p, stream)
+                              : launch_fwd_t<64, false>(tq, tk, tv, p, stream);
+  if (d == 128) return dropout ? launch_fwd_t<128, true>(tq, tk, tv, p, stream)
+                               : launch_fwd_t<128, false>(tq, tk, tv, p, stream);
   return cudaErrorInvalidValue;
 }
 
