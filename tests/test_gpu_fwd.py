@@ -69,7 +69,7 @@ CASES = [
     (2, 2, 256, 64, True, None, None, 0.1),        # dropout
     (2, 2, 384, 128, False, (100, 384), None, 0.2),
     (1, 3, 700, 64, True, (500, 700), 0.4, 0.3),
-    # d = 64 beyond N = 4096 runs two Q tiles per CTA through three S buffers
+    # d = 64 rows longer than 4096 (many K/V tiles per key-split stream)
     (1, 1, 4200, 64, False, None, 0.3, 0.0),
     (1, 2, 4224, 64, True, None, None, 0.1),
     (1, 1, 4400, 64, True, (2000, 4400), 0.4, 0.0),
