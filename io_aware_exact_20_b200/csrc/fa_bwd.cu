@@ -390,11 +390,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           qb = qbn;
         }
       } else {
-        // serialized order: dV, dK, dQ once P and dS are both ready, then the
-        // next tile's S^T and dP^T
+        // serialized order, once P and dS are both ready: dV, then the next
+        // tile's S^T (it overwrites S^T / P only after the dV MMAs, which
+        // execute first) and, at d = 64, its dP^T (the dP^T columns were read
+        // by this tile's P / dS warps already), then dK and dQ.  The next
+        // tile's S^T / dP^T are ready while dK and dQ still run.  At d = 128
+        // the dQ^T tile lives in the dP^T columns, so dP^T comes last.
         for (int qb = q_first; ok && qb < w.nqb; ++it) {
           const int s = it % L::STAGES;
           const int qbn = w.next(qb + 1);
+          const int sn = (it + 1) % L::STAGES;
           if (!mbar_wait(bar(L::B_PFULL), it & 1u, g)) break;
           tc_fence_after();
           const uint32_t q_addr = sbase + L::OFF_Q + s * L::TILE;
@@ -405,6 +410,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_ts(tmem + L::COL_DV, tmem + L::COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
                    sdesc_sw128(do_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
                    (it > 0 || kk > 0) ? 1u : 0u);
+          if (qbn < w.nqb) {
+            if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
+            tc_fence_after();
+            issue_sdp(sn, false);
+            if (L::SEPARATE_DQ) issue_sdp(sn, true);
+          }
           // dK += dS^T Q   (A = dS^T K-major in shared memory, B = Q MN-major)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -429,15 +440,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_commit(bar(L::B_DQFULL));
           mma_commit(bar(L::B_DSEMPTY));
           if constexpr (!L::TMA_REDUCE) mma_commit(bar(L::B_QEMPTY + s));
-          if (qbn < w.nqb) {
-            const int sn = (it + 1) % L::STAGES;
-            if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
+          if (!L::SEPARATE_DQ && qbn < w.nqb) {
+            if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
             tc_fence_after();
-            issue_sdp(sn, false);
-            if (!L::SEPARATE_DQ) {
-              if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
-              tc_fence_after();
-            }
             issue_sdp(sn, true);
           }
           qb = qbn;
