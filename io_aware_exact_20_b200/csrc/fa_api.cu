@@ -126,7 +126,7 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
   p.nblk = (N + 127) / 128;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * kLog2e);
   p.causal = causal != 0;
-  p.tiles_major = fa::tiles_major_order(B, H, N, d) ? 1 : 0;
+  p.group_heads = fa::order_group_heads(B, H, N, d, causal != 0);
   p.drop_threshold = dr.threshold;
   p.drop_rscale = dr.rscale;
   p.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
@@ -223,7 +223,7 @@ fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void*
   p.seqlens = seqlens;
   p.block_mask = block_mask;
   p.causal = causal != 0;
-  p.tiles_major = fa::tiles_major_order(B, H, N, d) ? 1 : 0;
+  p.group_heads = fa::order_group_heads(B, H, N, d, causal != 0);
   p.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
   p.seed_hi = static_cast<uint32_t>(seed >> 32);
   p.rk = fa::philox_round_keys(seed);

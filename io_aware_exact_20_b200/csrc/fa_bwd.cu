@@ -212,8 +212,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
 
   BwdWork w;
-  w.kb = static_cast<int>(p.tiles_major ? blockIdx.y : blockIdx.x);  // key tile 0 is heaviest
-  w.bh = static_cast<int>(p.tiles_major ? blockIdx.x : blockIdx.y);
+  grid_unit(blockIdx.x, p.B * p.H, (p.N + 127) / 128, p.group_heads, &w.bh, &w.kb);  // key tile 0 is heaviest
   w.b = w.bh / p.H;
   w.h = w.bh % p.H;
   {
@@ -825,9 +824,9 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::SMEM));
   if (e != cudaSuccess) return e;
-  const unsigned tiles = static_cast<unsigned>((p.N + 127) / 128), bh = static_cast<unsigned>(p.B * p.H);
-  const dim3 grid = p.tiles_major ? dim3(bh, tiles) : dim3(tiles, bh);
-  kern<<<grid, kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, tdq, p);
+  const long long ctas = static_cast<long long>((p.N + 127) / 128) * p.B * p.H;
+  if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(ctas), kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError();
 }
 

@@ -165,11 +165,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   FwdWork w;
   {
     const int nqp = (p.N + 128 * NQ - 1) / (128 * NQ);
-    const int tile = static_cast<int>(p.tiles_major ? blockIdx.y : blockIdx.x);
+    int tile = 0;
+    grid_unit(blockIdx.x, p.B * p.H, nqp, p.group_heads, &w.bh, &tile);
     const int qp = nqp - 1 - tile;  // heaviest causal rows first
     w.q0 = qp * 128 * NQ;
     w.qb0 = qp * NQ;
-    w.bh = static_cast<int>(p.tiles_major ? blockIdx.x : blockIdx.y);
     w.b = w.bh / p.H;
     w.h = w.bh % p.H;
     w.exists1 = NQ == 2 && (w.q0 + 128) < p.N;
@@ -620,10 +620,9 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::SMEM));
   if (e != cudaSuccess) return e;
-  const unsigned tiles = static_cast<unsigned>((p.N + 128 * C::NQ - 1) / (128 * C::NQ));
-  const unsigned bh = static_cast<unsigned>(p.B * p.H);
-  const dim3 grid = p.tiles_major ? dim3(bh, tiles) : dim3(tiles, bh);
-  kern<<<grid, C::THREADS, L::SMEM, stream>>>(tq, tk, tv, p);
+  const long long ctas = static_cast<long long>((p.N + 128 * C::NQ - 1) / (128 * C::NQ)) * p.B * p.H;
+  if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(ctas), C::THREADS, L::SMEM, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
