@@ -28,7 +28,9 @@
  *    (row-major, d fastest), in device memory, 16-byte aligned.
  *  - LSE is fp32 [B, H, N], natural logarithm; a row with no valid key has
  *    LSE = -inf and O = 0.
- *  - d is 64 or 128.  1 <= N; B * H <= 65535.
+ *  - d is 64 or 128.  1 <= N <= 2^23; B * H <= 65535 and
+ *    B * H * ceil(N / 128) <= 2^31 - 1 (one thread block per head and
+ *    128-row tile); larger requests return FA_ERR_UNSUPPORTED.
  *  - softmax_scale multiplies Q K^T before masking (typically 1/sqrt(d)).
  *  - causal != 0: query i attends key j only if j <= i.
  *  - seqlens: NULL, or device int32[B]; keys j >= seqlens[b] are masked for
@@ -68,7 +70,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, p out of range */
-  FA_ERR_UNSUPPORTED = 2, /* valid request the kernels do not cover (d not 64/128, B*H too large) */
+  FA_ERR_UNSUPPORTED = 2, /* valid request the kernels do not cover (d not 64/128, sizes too large) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed */
   FA_ERR_TIMEOUT = 4,     /* a kernel gave up on a pipeline wait (reported by fa_last_device_status) */
   FA_ERR_WORKSPACE = 5    /* workspace missing or smaller than fa_bwd_workspace_size() */

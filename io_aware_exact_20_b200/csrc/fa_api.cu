@@ -41,6 +41,8 @@ fa_status_t check_shape(int B, int H, int N, int d, float scale, float dropout_p
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * H > 65535) return FA_ERR_UNSUPPORTED;
   if (N > (1 << 23)) return FA_ERR_UNSUPPORTED;
+  // one CTA per (b, h, 128-row tile) in a 1-D grid
+  if (static_cast<int64_t>(B) * H * ((N + 127) / 128) > 0x7FFFFFFF) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 

@@ -55,6 +55,8 @@ A16 = 1 << 20  # a fake, 16-byte aligned address: validation fails before use
     (dict(d=96), 2), (dict(scale=0.0), 1), (dict(scale=float("inf")), 1),
     (dict(p=1.0), 1), (dict(p=-0.1), 1), (dict(p=float("nan")), 1),
     (dict(B=300, H=300), 2), (dict(lse=A16 + 2), 1),
+    (dict(N=(1 << 23) + 1), 2),                       # N beyond 2^23
+    (dict(B=65535, H=1, N=1 << 23), 2),               # 65535 x 65536 tiles > 2^31 - 1
 ])
 def test_fwd_rejects_bad_arguments_without_launching(lib, args, code):
     so = lib.library()
