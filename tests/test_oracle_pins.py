@@ -101,6 +101,63 @@ def test_philox4x32_vectorised_equals_scalar_definition():
         assert tuple(int(v[n]) for v in vec) == want
 
 
+def _curand_host_library():
+    """cuRAND's shared library (host generators run on the CPU, no GPU needed)."""
+    import ctypes
+    import glob
+    import sys
+    pats = ["/usr/local/cuda/lib64/libcurand.so.10*", "/usr/local/cuda/lib64/libcurand.so*"]
+    for p in sys.path:
+        pats.append(os.path.join(p, "nvidia", "curand", "lib", "libcurand.so*"))
+    for pat in pats:
+        for path in sorted(glob.glob(pat)):
+            try:
+                return ctypes.CDLL(path)
+            except OSError:
+                continue
+    return None
+
+
+def curand_philox_words(seed, n):
+    """The first n 32-bit outputs of cuRAND's host Philox4x32-10 generator
+    (CURAND_RNG_PSEUDO_PHILOX4_32_10 = 161) seeded with `seed`, obtained by
+    running the library; nothing of its internals is read."""
+    import ctypes
+    lib = _curand_host_library()
+    if lib is None:
+        pytest.skip("libcurand not found")
+    gen = ctypes.c_void_p()
+    assert lib.curandCreateGeneratorHost(ctypes.byref(gen), 161) == 0
+    try:
+        assert lib.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
+        buf = (ctypes.c_uint32 * n)()
+        assert lib.curandGenerate(gen, buf, ctypes.c_size_t(n)) == 0
+        return [int(x) for x in buf]
+    finally:
+        lib.curandDestroyGenerator(gen)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 0xFFFFFFFF, 1 << 32, 0x0123456789ABCDEF,
+                                  0x5EED000000000002, 0xDEADBEEFCAFEF00D,
+                                  0xFFFFFFFFFFFFFFFF, 0x5EED0002])
+def test_philox4x32_known_answers_from_curand(seed):
+    """Known-answer pin of the 32-bit instance, multipliers included: cuRAND's
+    host Philox4x32-10 generator is an independent implementation of the same
+    published definition (Salmon et al., SC'11).  Seeded with s it uses key
+    (s mod 2^32, s >> 32) and emits block k of its stream from counter
+    (0, 0, k, 0) (layout found by experiment: block 0 at counter 0, later blocks
+    step counter word 2).  A wrong digit in either multiplier, a swapped key
+    word or a wrong Weyl step changes every word."""
+    blocks = 16
+    words = curand_philox_words(seed, 4 * blocks)
+    key = [seed & 0xFFFFFFFF, seed >> 32]
+    for k in range(blocks):
+        assert tuple(words[4 * k:4 * k + 4]) == philox_block([0, 0, k, 0], key, 32, 10), k
+    # the vectorised instance the dropout bits use gives the same words
+    vec = philox4x32_10(0, 0, np.arange(blocks, dtype=np.uint64), 0, key[0], key[1])
+    assert np.array_equal(np.stack(vec, axis=1).ravel(), np.array(words, dtype=np.uint32))
+
+
 def test_philox4x32_words_are_uniform():
     """Chi-square of byte values and the mean of 2^20 words: a generator with a
     dropped round or a wrong multiplier on a structured counter sequence fails."""
