@@ -29,7 +29,11 @@ running max m and row sum l are the readings used here).
 
 Readings taken where the pages are silent (all are repeated in the design doc):
   * scale is a caller-given float applied to Q K^T before masking and the max;
-  * causal: query i may attend key j iff j <= i (0-based, N_q = N_k = N);
+  * causal: query i may attend key j iff j <= i + (N_k - N_q) (0-based; the
+    last query is aligned with the last key, "bottom-right"; with N_q = N_k
+    this is j <= i).  When N_q > N_k the first N_q - N_k queries see no key.
+    Key padding does not move the alignment: N_k is the key count of the
+    layout (or of the packed sequence), not the padded length;
   * key padding: per-batch length L_b, keys j >= L_b are invalid; query rows
     are not masked (they still attend the valid keys);
   * block mask: uint8 [ceil(N/128)]^2 shared by all (b, h); entry 0 removes the
@@ -64,11 +68,13 @@ BLOCK = 128  # block-mask granularity (128 x 128 blocks of (query, key) pairs)
 # masks and dropout bits
 # ----------------------------------------------------------------------------
 
-def valid_mask(n, rows, causal=False, kv_len=None, block_mask=None):
+def valid_mask(n, rows, causal=False, kv_len=None, block_mask=None, n_q=None):
     """Boolean [len(rows), n]: which (query i, key j) pairs take part.
 
-    rows: query indices (int array).  kv_len: valid key count for this batch
-    entry (None = n).  block_mask: uint8 [nb, nb] or None.
+    n: number of keys.  rows: query indices (int array).  kv_len: valid key
+    count for this batch entry (None = n).  block_mask: uint8 [nbq, nbk] or
+    None.  n_q: number of queries (None = n); under the causal mask query i
+    sees key j iff j <= i + (n - n_q).
     """
     rows = np.asarray(rows, dtype=np.int64)
     i = rows[:, None]
@@ -77,7 +83,8 @@ def valid_mask(n, rows, causal=False, kv_len=None, block_mask=None):
     if kv_len is not None:
         ok &= j < int(kv_len)
     if causal:
-        ok &= j <= i
+        off = 0 if n_q is None else int(n) - int(n_q)
+        ok &= j <= i + off
     if block_mask is not None:
         bm = np.asarray(block_mask).astype(bool)
         ok &= bm[i // BLOCK, j // BLOCK]
@@ -144,7 +151,7 @@ def safe_softmax(s, valid):
 
 def _head_forward(q, k, v, scale, rows, causal, kv_len, block_mask, keep, rscale):
     s = scale * (q[rows] @ k.T)
-    valid = valid_mask(k.shape[0], rows, causal, kv_len, block_mask)
+    valid = valid_mask(k.shape[0], rows, causal, kv_len, block_mask, n_q=q.shape[0])
     p, lse, _, _ = safe_softmax(s, valid)
     pd = p if keep is None else p * keep * rscale
     return pd @ v, lse
@@ -154,14 +161,16 @@ def attention_forward(q, k, v, scale, causal=False, seqlens=None, dropout_p=0.0,
                       seed=0, block_mask=None, heads=None, rows=None, slab=256):
     """O and LSE of standard attention.
 
-    q, k, v: float64 [B, H, N, d].  Returns (O [B,H,R,d], LSE [B,H,R]) where R
-    indexes ``rows`` (default all N rows).  ``heads`` optionally restricts the
+    q: float64 [B, H, N_q, d]; k, v: [B, H, N_k, d] (N_k may differ from N_q).
+    Returns (O [B,H,R,d], LSE [B,H,R]) where R indexes ``rows`` (default all
+    N_q rows).  ``heads`` optionally restricts the
     computation to a list of (b, h) pairs (other entries are left NaN).  Rows
     are processed in slabs of ``slab`` rows only to bound memory: every row is
     computed independently, so the slab size does not change any value.
     """
     q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
     B, H, N, d = q.shape
+    Nk = k.shape[2]
     rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
     out = np.full((B, H, rows.size, d), np.nan)
     lse = np.full((B, H, rows.size), np.nan)
@@ -174,7 +183,7 @@ def attention_forward(q, k, v, scale, causal=False, seqlens=None, dropout_p=0.0,
             rr = rows[r0:r0 + slab]
             keep = None
             if p32 > 0:
-                keep = dropout_keep(seed, p32, b, h, rr, N)
+                keep = dropout_keep(seed, p32, b, h, rr, Nk)
             o, l = _head_forward(q[b, h], k[b, h], v[b, h], scale, rr, causal,
                                  kv_len, block_mask, keep, rscale)
             out[b, h, r0:r0 + rr.size] = o
@@ -198,7 +207,7 @@ def head_backward(q, k, v, dout, scale, causal=False, kv_len=None, block_mask=No
     n = k.shape[0]
     rows = np.arange(q.shape[0])
     s = scale * (q @ k.T)
-    valid = valid_mask(n, rows, causal, kv_len, block_mask)
+    valid = valid_mask(n, rows, causal, kv_len, block_mask, n_q=q.shape[0])
     p, _, _, _ = safe_softmax(s, valid)
     p32 = float(np.float32(dropout_p))
     if keep is None or p32 == 0:
@@ -220,9 +229,11 @@ def head_backward(q, k, v, dout, scale, causal=False, kv_len=None, block_mask=No
 
 def attention_backward(q, k, v, dout, scale, causal=False, seqlens=None,
                        dropout_p=0.0, seed=0, block_mask=None, heads=None):
-    """dQ, dK, dV (float64 [B,H,N,d]) for every (b, h) in ``heads`` (default all)."""
+    """dQ [B,H,N_q,d], dK, dV [B,H,N_k,d] (float64) for every (b, h) in
+    ``heads`` (default all)."""
     q, k, v, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
     B, H, N, d = q.shape
+    Nk = k.shape[2]
     dq = np.full_like(q, np.nan)
     dk = np.full_like(k, np.nan)
     dv = np.full_like(v, np.nan)
@@ -230,7 +241,7 @@ def attention_backward(q, k, v, dout, scale, causal=False, seqlens=None,
     p32 = float(np.float32(dropout_p))
     for b, h in pairs:
         kv_len = None if seqlens is None else int(seqlens[b])
-        keep = dropout_keep(seed, p32, b, h, np.arange(N), N) if p32 > 0 else None
+        keep = dropout_keep(seed, p32, b, h, np.arange(N), Nk) if p32 > 0 else None
         g = head_backward(q[b, h], k[b, h], v[b, h], dout[b, h], scale, causal,
                           kv_len, block_mask, keep, p32)
         dq[b, h], dk[b, h], dv[b, h] = g[0], g[1], g[2]
@@ -247,7 +258,7 @@ def _row_terms(q, k, v, dout, scale, rows, causal, kv_len, block_mask, keep, dro
     own row of S, of dP = dO V^T and its own D_i)."""
     n = k.shape[0]
     s = scale * (q[rows] @ k.T)
-    valid = valid_mask(n, rows, causal, kv_len, block_mask)
+    valid = valid_mask(n, rows, causal, kv_len, block_mask, n_q=q.shape[0])
     p, _, _, _ = safe_softmax(s, valid)
     p32 = float(np.float32(dropout_p))
     if keep is None or p32 == 0:

@@ -573,3 +573,183 @@ def test_sampled_backward_with_dropout_matches_finite_differences():
                 args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
                 num[a, c] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
         assert np.linalg.norm(num - g) / np.linalg.norm(num) < 1e-6, name
+
+
+# ---------------------------------------------------------------------------
+# N_q != N_k (bottom-right causal alignment) and packed variable-length batches
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("nq,nk", [(3, 7), (7, 3), (5, 5), (1, 9), (9, 1), (130, 260)])
+def test_bottom_right_causal_mask_brute_force(nq, nk):
+    """Query i sees key j iff j <= i + nk - nq: written as plain loops; a
+    top-left alignment or an off-by-one in the offset fails."""
+    got = valid_mask(nk, np.arange(nq), True, None, None, n_q=nq)
+    for i in range(nq):
+        for j in range(nk):
+            assert got[i, j] == (j - i <= nk - nq)
+
+
+@pytest.mark.parametrize("nq,nk,kv", [(40, 100, None), (100, 40, None), (64, 200, 150),
+                                      (200, 64, 50), (1, 33, None)])
+def test_bottom_right_causal_matches_torch_lower_right(nq, nk, kv):
+    """torch's causal_lower_right bias is an independent definition of the
+    bottom-right alignment: SDPA with it (and autograd) must give the oracle's
+    O and gradients on every row that has a key (rows without one: O = 0,
+    LSE = -inf, no gradient)."""
+    import torch
+    from torch.nn.attention.bias import causal_lower_right
+
+    rng = np.random.default_rng(nq * 7 + nk)
+    H, d = 2, 8
+    q, do = _rand((1, H, nq, d), rng), _rand((1, H, nq, d), rng)
+    k, v = _rand((1, H, nk, d), rng), _rand((1, H, nk, d), rng)
+    seq = None if kv is None else np.array([kv], dtype=np.int32)
+    o, lse = attention_forward(q, k, v, 0.3, True, seq)
+    dq, dk, dv = attention_backward(q, k, v, do, 0.3, True, seq)
+    mask = causal_lower_right(nq, nk)._materialize(torch.device("cpu"))
+    if kv is not None:
+        mask = mask & (torch.arange(nk) < kv)[None, :]
+    has = mask.any(dim=-1).numpy()
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.3)
+    to = torch.where(torch.tensor(has)[:, None], to, torch.zeros_like(to))
+    (to * torch.tensor(do)).sum().backward()
+    assert np.abs(o - to.detach().numpy()).max() < 1e-12
+    assert (o[:, :, ~has] == 0).all() and np.isneginf(lse[:, :, ~has]).all()
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.abs(mine - ref.numpy()).max() < 1e-10
+
+
+@pytest.mark.parametrize("nq,nk", [(50, 130), (130, 50)])
+def test_zero_q_bottom_right_closed_form(nq, nk):
+    """Q = 0 under the bottom-right causal mask: row i has
+    n_i = clip(i + nk - nq + 1, 0, nk) valid keys, the first n_i of them, so
+    O_i = mean(V_0 .. V_{n_i - 1}) and LSE_i = ln n_i (n_i = 0: O = 0, -inf)."""
+    rng = np.random.default_rng(41)
+    d = 4
+    q = np.zeros((1, 1, nq, d))
+    k, v = _rand((1, 1, nk, d), rng), _rand((1, 1, nk, d), rng)
+    o, lse = attention_forward(q, k, v, 0.5, True)
+    for i in range(nq):
+        n = min(max(i + nk - nq + 1, 0), nk)
+        if n == 0:
+            assert (o[0, 0, i] == 0).all() and np.isneginf(lse[0, 0, i])
+        else:
+            assert np.abs(o[0, 0, i] - v[0, 0, :n].mean(axis=0)).max() < 1e-12
+            assert abs(lse[0, 0, i] - math.log(n)) < 1e-12
+
+
+def _pack(seqs):
+    """[B] list of [H, n_b, d] arrays -> packed [sum n_b, H, d] and offsets."""
+    cu = np.concatenate([[0], np.cumsum([s.shape[1] for s in seqs])]).astype(np.int32)
+    packed = np.concatenate([s.transpose(1, 0, 2) for s in seqs], axis=0)
+    return packed, cu
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equals_each_sequence_on_its_own(causal):
+    """Packed sequences (lengths 0, 1, 129, 300, 77 queries against other key
+    counts) give, row for row, the padded oracle run on each sequence alone
+    (no dropout: the padded call would number the sequence 0).  Catches wrong
+    offsets, a token / head transposition or attention leaking across
+    sequences."""
+    from oracle import attention_forward_varlen, attention_backward_varlen
+    rng = np.random.default_rng(51)
+    H, d, scale = 2, 8, 0.35
+    lq = [0, 1, 129, 300, 77]
+    lk = [5, 1, 200, 300, 31]
+    qs = [_rand((H, n, d), rng) for n in lq]
+    dos = [_rand((H, n, d), rng) for n in lq]
+    ks = [_rand((H, n, d), rng) for n in lk]
+    vs = [_rand((H, n, d), rng) for n in lk]
+    q, cu_q = _pack(qs)
+    do, _ = _pack(dos)
+    k, cu_k = _pack(ks)
+    v, _ = _pack(vs)
+    o, lse = attention_forward_varlen(q, k, v, cu_q, cu_k, scale, causal)
+    dq, dk, dv = attention_backward_varlen(q, k, v, do, cu_q, cu_k, scale, causal)
+    for b in range(len(lq)):
+        if lq[b] == 0:
+            continue
+        ro, rl = attention_forward(qs[b][None], ks[b][None], vs[b][None], scale, causal)
+        rg = attention_backward(qs[b][None], ks[b][None], vs[b][None], dos[b][None], scale,
+                                causal)
+        sq = slice(cu_q[b], cu_q[b + 1])
+        sk = slice(cu_k[b], cu_k[b + 1])
+        # equal up to BLAS summation order (strided vs contiguous operands)
+        assert np.abs(o[sq].transpose(1, 0, 2) - ro[0]).max() < 1e-12
+        empty = np.isneginf(rl[0])
+        assert np.array_equal(np.isneginf(lse[:, sq]), empty)
+        assert np.abs(np.where(empty, 0.0, lse[:, sq] - np.where(empty, 0.0, rl[0]))).max() < 1e-12
+        assert np.abs(dq[sq].transpose(1, 0, 2) - rg[0][0]).max() < 1e-10
+        assert np.abs(dk[sk].transpose(1, 0, 2) - rg[1][0]).max() < 1e-10
+        assert np.abs(dv[sk].transpose(1, 0, 2) - rg[2][0]).max() < 1e-10
+
+
+def test_varlen_dropout_and_key_lengths_use_the_sequence_index():
+    """With dropout the keep bits of sequence b are those of batch entry b:
+    packed sequences of equal query and key length equal a padded batch whose
+    entry b holds sequence b at its start, the rest masked by key lengths."""
+    from oracle import attention_forward_varlen, attention_backward_varlen
+    rng = np.random.default_rng(52)
+    H, d, N, p, seed = 2, 8, 140, 0.25, 99
+    lens = [140, 60, 131]
+    full = [_rand((4, H, N, d), rng) for _ in range(len(lens))]  # q, k, v, dO per sequence
+    seqs = [[f[x][:, :n] for f, n in zip(full, lens)] for x in range(4)]
+    q, cu = _pack(seqs[0])
+    k, _ = _pack(seqs[1])
+    v, _ = _pack(seqs[2])
+    do, _ = _pack(seqs[3])
+    pq, pk, pv, pdo = (np.stack([f[x] for f in full]) for x in range(4))
+    seqlens = np.array(lens, dtype=np.int32)
+    for causal in (False, True):
+        o, lse = attention_forward_varlen(q, k, v, cu, cu, 0.3, causal, None, p, seed)
+        dq, dk, dv = attention_backward_varlen(q, k, v, do, cu, cu, 0.3, causal, None, p, seed)
+        ro, rl = attention_forward(pq, pk, pv, 0.3, causal, seqlens, p, seed)
+        rdq, rdk, rdv = attention_backward(pq, pk, pv, pdo, 0.3, causal, seqlens, p, seed)
+        for b, n in enumerate(lens):
+            s = slice(cu[b], cu[b + 1])
+            # padded rows of the padded batch only add masked keys (and, for
+            # causal, N = N_k keeps the alignment), so rows i < n agree
+            assert np.abs(o[s].transpose(1, 0, 2) - ro[b][:, :n]).max() < 1e-12
+            assert np.abs(lse[:, s] - rl[b][:, :n]).max() < 1e-12
+            # dK, dV of keys j < n: the padded batch's extra query rows i >= n
+            # see those keys too (key padding masks keys, not queries), so
+            # only dQ rows are comparable
+            assert np.abs(dq[s].transpose(1, 0, 2) - rdq[b][:, :n]).max() < 1e-10
+    # key lengths inside packed sequences: keys past seqlens_k[b] are masked
+    o1, _ = attention_forward_varlen(q, k, v, cu, cu, 0.3, False, np.array([10, 60, 20]))
+    o2, _ = attention_forward_varlen(q, k, v, cu, cu, 0.3, False, None)
+    assert np.array_equal(o1[cu[1]:cu[2]], o2[cu[1]:cu[2]])       # 60 = the full length
+    assert not np.allclose(o1[cu[0]:cu[1]], o2[cu[0]:cu[1]])
+
+
+def test_varlen_backward_matches_finite_differences():
+    """Packed backward (bottom-right causal, dropout, a key length) against
+    central differences of L = sum(O * dO)."""
+    from oracle import attention_forward_varlen, attention_backward_varlen
+    rng = np.random.default_rng(53)
+    H, d, p, seed = 1, 3, 0.3, 5
+    cu_q = np.array([0, 4, 4, 9], dtype=np.int32)
+    cu_k = np.array([0, 6, 8, 11], dtype=np.int32)
+    skl = np.array([5, 2, 3], dtype=np.int32)
+    q, do = _rand((9, H, d), rng), _rand((9, H, d), rng)
+    k, v = _rand((11, H, d), rng), _rand((11, H, d), rng)
+
+    def loss(q_, k_, v_):
+        o, _ = attention_forward_varlen(q_, k_, v_, cu_q, cu_k, 0.6, True, skl, p, seed)
+        return float((o * do).sum())
+
+    grads = attention_backward_varlen(q, k, v, do, cu_q, cu_k, 0.6, True, skl, p, seed)
+    eps = 1e-6
+    for name, x, g in zip("qkv", (q, k, v), grads):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            a = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num[idx] = (loss(*a) - loss(*m)) / (2 * eps)
+        err = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+        assert err < 1e-6, (name, err)
