@@ -16,6 +16,7 @@ from .attention_ref import (  # noqa: F401
     head_backward_cols,
     head_backward_rows,
     head_forward_rows,
+    merge_partials,
     safe_softmax,
     valid_mask,
 )

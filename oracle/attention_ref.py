@@ -318,3 +318,28 @@ def head_backward_cols(q, k, v, dout, scale, cols, causal=False, kv_len=None,
         dv += pd[:, cols].T @ dout[rows]
         dk += scale * (ds[:, cols].T @ q[rows])
     return dk, dv
+
+
+# ----------------------------------------------------------------------------
+# combining partial results over disjoint key sets
+# ----------------------------------------------------------------------------
+
+def merge_partials(o_a, lse_a, o_b, lse_b):
+    """(O, LSE) over the union of two disjoint key sets from the results over
+    each set alone: LSE = ln(e^LSE_a + e^LSE_b), O = e^(LSE_a - LSE) O_a +
+    e^(LSE_b - LSE) O_b.  This is the definition of the softmax over a union
+    (the normaliser is the sum of the parts' normalisers), the rule the
+    pages' tiling applies between key blocks (suanlizi.com summary,
+    分块计算（Tiling）).  Empty parts have LSE = -inf and add nothing."""
+    o_a, o_b = np.asarray(o_a, dtype=np.float64), np.asarray(o_b, dtype=np.float64)
+    lse_a, lse_b = np.asarray(lse_a, dtype=np.float64), np.asarray(lse_b, dtype=np.float64)
+    m = np.maximum(lse_a, lse_b)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    ea = np.where(np.isneginf(lse_a), 0.0, np.exp(lse_a - m_safe))
+    eb = np.where(np.isneginf(lse_b), 0.0, np.exp(lse_b - m_safe))
+    s = ea + eb
+    with np.errstate(divide="ignore", invalid="ignore"):
+        lse = np.where(s > 0, m_safe + np.log(np.where(s > 0, s, 1.0)), -np.inf)
+        wa = np.where(s > 0, ea / np.where(s > 0, s, 1.0), 0.0)
+        wb = np.where(s > 0, eb / np.where(s > 0, s, 1.0), 0.0)
+    return wa[..., None] * o_a + wb[..., None] * o_b, lse

@@ -753,3 +753,48 @@ def test_varlen_backward_matches_finite_differences():
             num[idx] = (loss(*a) - loss(*m)) / (2 * eps)
         err = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
         assert err < 1e-6, (name, err)
+
+
+# ---------------------------------------------------------------------------
+# merging partial results over disjoint key sets (context parallelism)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_merge_of_key_blocks_equals_attention_over_all_keys(causal):
+    """Attention of Q against key blocks 0..3 taken apart (each block's own
+    (O, LSE), causal only on the diagonal block, blocks past it skipped) and
+    merged left to right equals attention over all keys: the decomposition a
+    context-parallel ring computes.  A wrong weight (no renormalisation, a
+    missing exp) or a mishandled empty block fails."""
+    from oracle import merge_partials
+    rng = np.random.default_rng(61)
+    W, n, d = 4, 50, 8
+    q, k, v = (_rand((1, 2, W * n, d), rng) for _ in range(3))
+    o_full, l_full = attention_forward(q, k, v, 0.4, causal)
+    for r in range(W):  # query block r
+        qr = q[:, :, r * n:(r + 1) * n]
+        o = np.zeros_like(qr)
+        lse = np.full(qr.shape[:-1], -np.inf)
+        for c in range(W):  # key block c
+            if causal and c > r:
+                continue
+            kc, vc = k[:, :, c * n:(c + 1) * n], v[:, :, c * n:(c + 1) * n]
+            op, lp = attention_forward(qr, kc, vc, 0.4, causal and c == r)
+            o, lse = merge_partials(o, lse, op, lp)
+        assert np.abs(o - o_full[:, :, r * n:(r + 1) * n]).max() < 1e-12
+        assert np.abs(lse - l_full[:, :, r * n:(r + 1) * n]).max() < 1e-12
+
+
+def test_merge_with_empty_parts():
+    """Empty parts (LSE = -inf) change nothing; two empty parts stay empty."""
+    from oracle import merge_partials
+    rng = np.random.default_rng(62)
+    o = rng.standard_normal((5, 4))
+    lse = rng.standard_normal(5)
+    inf = np.full(5, -np.inf)
+    o2, l2 = merge_partials(o, lse, np.zeros((5, 4)), inf)
+    assert np.array_equal(o2, o) and np.array_equal(l2, lse)
+    o3, l3 = merge_partials(np.ones((5, 4)), inf, o, lse)
+    assert np.array_equal(o3, o) and np.array_equal(l3, lse)
+    o4, l4 = merge_partials(np.ones((5, 4)), inf, np.ones((5, 4)), inf)
+    assert (o4 == 0).all() and np.isneginf(l4).all()
