@@ -13,6 +13,7 @@ from .attention_ref import (  # noqa: F401
     dropout_scale,
     dropout_threshold,
     head_backward,
+    head_backward_block,
     head_backward_cols,
     head_backward_rows,
     head_forward_rows,

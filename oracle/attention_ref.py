@@ -343,3 +343,33 @@ def merge_partials(o_a, lse_a, o_b, lse_b):
         wa = np.where(s > 0, ea / np.where(s > 0, s, 1.0), 0.0)
         wb = np.where(s > 0, eb / np.where(s > 0, s, 1.0), 0.0)
     return wa[..., None] * o_a + wb[..., None] * o_b, lse
+
+
+def head_backward_block(q, k, v, dout, lse, delta, scale, causal=False, n_q=None, n_k=None,
+                        q0=0, k0=0):
+    """The part of one head's backward that comes from one block of keys,
+    given the softmax statistics of the full row (its LSE and
+    D_i = sum_c dO_ic O_ic over all keys): with P = exp(scale Q K_blk^T - LSE),
+    dP = dO V_blk^T and dS = P (dP - D),
+
+        dQ_part = scale dS K_blk,  dK_blk = scale dS^T Q,  dV_blk = P^T dO.
+
+    Summed over disjoint key blocks this is the full backward (the recomputation
+    of the pages needs only LSE and D per row: suanlizi.com summary, 重计算).
+    q, dout: [R, d] rows q0 .. of a sequence of n_q queries; k, v: [C, d] keys
+    k0 .. of n_k keys; causal (bottom-right): key j valid iff j <= i + n_k - n_q.
+    No dropout."""
+    q, k, v, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    rows = q0 + np.arange(q.shape[0])[:, None]
+    cols = k0 + np.arange(k.shape[0])[None, :]
+    s = scale * (q @ k.T)
+    valid = np.ones(s.shape, dtype=bool)
+    if causal:
+        valid = cols <= rows + ((n_k or 0) - (n_q or 0))
+    lse = np.asarray(lse, dtype=np.float64)[:, None]
+    with np.errstate(invalid="ignore"):
+        p = np.where(valid & np.isfinite(lse), np.exp(s - np.where(np.isfinite(lse), lse, 0.0)),
+                     0.0)
+    dp = dout @ v.T
+    ds = p * (dp - np.asarray(delta, dtype=np.float64)[:, None])
+    return scale * (ds @ k), scale * (ds.T @ q), p.T @ dout

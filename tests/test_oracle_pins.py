@@ -798,3 +798,32 @@ def test_merge_with_empty_parts():
     assert np.array_equal(o3, o) and np.array_equal(l3, lse)
     o4, l4 = merge_partials(np.ones((5, 4)), inf, np.ones((5, 4)), inf)
     assert (o4 == 0).all() and np.isneginf(l4).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_backward_sums_to_the_full_backward(causal):
+    """The per-key-block backward given the full rows' LSE and D, summed over
+    blocks (query blocks x key blocks), equals the full backward: the
+    decomposition a context-parallel ring uses.  Dropping the D term, using
+    the block's own LSE or a wrong causal offset fails."""
+    from oracle import head_backward_block
+    rng = np.random.default_rng(63)
+    W, n, d, scale = 3, 40, 8, 0.45
+    N = W * n
+    q, k, v, do = (_rand((N, d), rng) for _ in range(4))
+    dq, dk, dv, _ = head_backward(q, k, v, do, scale, causal)
+    o, lse = attention_forward(q[None, None], k[None, None], v[None, None], scale, causal)
+    delta = (do * o[0, 0]).sum(axis=1)
+    gq, gk, gv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for r in range(W):
+        rs = slice(r * n, (r + 1) * n)
+        for c in range(W):
+            cs = slice(c * n, (c + 1) * n)
+            a, b, e = head_backward_block(q[rs], k[cs], v[cs], do[rs], lse[0, 0, rs], delta[rs],
+                                          scale, causal, N, N, r * n, c * n)
+            gq[rs] += a
+            gk[cs] += b
+            gv[cs] += e
+    assert np.abs(gq - dq).max() < 1e-10
+    assert np.abs(gk - dk).max() < 1e-10
+    assert np.abs(gv - dv).max() < 1e-10
