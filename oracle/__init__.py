@@ -22,4 +22,5 @@ from .attention_ref import (  # noqa: F401
     valid_mask,
 )
 from .philox_ref import philox4x32_10, philox_block, weyl_constants  # noqa: F401
+from .projection_ref import qkv_projection  # noqa: F401
 from .varlen_ref import attention_backward_varlen, attention_forward_varlen  # noqa: F401

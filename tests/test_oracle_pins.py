@@ -827,3 +827,46 @@ def test_block_backward_sums_to_the_full_backward(causal):
     assert np.abs(gq - dq).max() < 1e-10
     assert np.abs(gk - dk).max() < 1e-10
     assert np.abs(gv - dv).max() < 1e-10
+
+
+# ---------------------------------------------------------------------------
+# QKV projection (the layer in front of attention)
+# ---------------------------------------------------------------------------
+
+def test_qkv_projection_brute_force():
+    """Every output element as an explicit sum over the model dimension, with
+    the stated column / token mapping written out as loops."""
+    from oracle import qkv_projection
+    rng = np.random.default_rng(91)
+    B, N, H, d, Dm = 2, 3, 2, 4, 5
+    x = rng.standard_normal((B * N, Dm))
+    w = rng.standard_normal((3 * H * d, Dm))
+    bias = rng.standard_normal(3 * H * d)
+    q, k, v = qkv_projection(x, w, bias, B, H, d)
+    for which, out in enumerate((q, k, v)):
+        for b in range(B):
+            for h in range(H):
+                for n in range(N):
+                    for e in range(d):
+                        c = which * H * d + h * d + e
+                        want = sum(x[b * N + n, f] * w[c, f] for f in range(Dm)) + bias[c]
+                        assert abs(out[b, h, n, e] - want) < 1e-12
+
+
+def test_qkv_projection_matches_torch_linear():
+    """torch.nn.functional.linear, split into q, k, v and heads with
+    view / permute: an independent route to the same tensors."""
+    import torch
+    from oracle import qkv_projection
+    rng = np.random.default_rng(92)
+    B, N, H, d, Dm = 3, 17, 4, 8, 24
+    x = rng.standard_normal((B * N, Dm))
+    w = rng.standard_normal((3 * H * d, Dm))
+    bias = rng.standard_normal(3 * H * d)
+    q, k, v = qkv_projection(x, w, bias, B, H, d)
+    y = torch.nn.functional.linear(torch.tensor(x), torch.tensor(w), torch.tensor(bias))
+    ref = y.view(B, N, 3, H, d).permute(2, 0, 3, 1, 4)
+    for i, got in enumerate((q, k, v)):
+        assert np.abs(got - ref[i].numpy()).max() < 1e-12
+    q0, _, _ = qkv_projection(x, w, None, B, H, d)
+    assert np.abs(q0 - (q - bias[:H * d].reshape(1, H, 1, d))).max() < 1e-12
