@@ -28,7 +28,8 @@
  *    (row-major, d fastest), in device memory, 16-byte aligned.
  *  - LSE is fp32 [B, H, N], natural logarithm; a row with no valid key has
  *    LSE = -inf and O = 0.
- *  - d is 64 or 128.  1 <= N <= 2^23; B * H <= 65535 and
+ *  - d is 32, 64, 96 or 128 (32 and 96 run the 64- and 128-wide kernels on
+ *    zero-filled columns).  1 <= N <= 2^23; B * H <= 65535 and
  *    B * H * ceil(N / 128) <= 2^31 - 1 (one thread block per head and
  *    128-row tile); larger requests return FA_ERR_UNSUPPORTED.
  *  - softmax_scale multiplies Q K^T before masking (typically 1/sqrt(d)).
@@ -70,7 +71,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, p out of range */
-  FA_ERR_UNSUPPORTED = 2, /* valid request the kernels do not cover (d not 64/128, sizes too large) */
+  FA_ERR_UNSUPPORTED = 2, /* valid request the kernels do not cover (d not 32/64/96/128, sizes too large) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed */
   FA_ERR_TIMEOUT = 4,     /* a kernel gave up on a pipeline wait (reported by fa_last_device_status) */
   FA_ERR_WORKSPACE = 5    /* workspace missing or smaller than fa_bwd_workspace_size() */
@@ -83,8 +84,9 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
                    float dropout_p, uint64_t seed, const uint8_t* block_mask, void* stream);
 
 /* Bytes of device workspace fa_bwd needs for these sizes: per (b, h) and per
- * query row rounded up to a multiple of 128, one fp32 log2-domain LSE, one
- * fp32 D_i = sum_c dO_ic O_ic and d fp32 dQ accumulators.  0 on bad sizes. */
+ * query row rounded up to a multiple of 128, one fp32 -LSE_i * log2(e), one
+ * fp32 -D_i = -sum_c dO_ic O_ic and D fp32 dQ accumulators (D = 64 for
+ * d <= 64, else 128).  0 on bad sizes. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /* Backward pass.  Given the forward inputs, its outputs o and lse, and dout
@@ -103,9 +105,11 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
 /* The three launches fa_bwd makes, exposed so that each can be timed or
  * scheduled on its own.  Called in this order on one stream with the same
  * workspace they are exactly fa_bwd.
- *  fa_bwd_prepare: from o, lse, dout fills the workspace with D_i, the
- *    log2-domain LSE (+inf where a row has no key, so its P is 0) and zeroed
- *    dQ accumulators.  Reads the softmax statistics the forward saved.
+ *  fa_bwd_prepare: from o, lse, dout fills the workspace with -D_i, the
+ *    negated log2-domain LSE -LSE_i * log2(e) (-inf for rows without keys and
+ *    for the padding rows up to the next multiple of 128, so that their P is
+ *    exactly 0) and zeroed dQ accumulators.  Reads the softmax statistics the
+ *    forward saved.
  *  fa_bwd_main: recomputes P block by block from those statistics (the
  *    recomputation of the pages) and writes dk, dv (bf16) and the fp32 dQ
  *    accumulators in the workspace.
@@ -130,7 +134,13 @@ fa_status_t fa_bwd_finish(void* dq, int B, int H, int N, int d, float softmax_sc
  *  - Returns FA_ERR_WORKSPACE, launching nothing, when
  *    fa_bwd_workspace_size(B,H,N,d) exceeds 64 MiB (67108864 bytes).
  *  - The first call on a device looks the array's address up with
- *    cudaGetSymbolAddress; make that first call before any stream capture.
+ *    cudaGetSymbolAddress.  Under CUDA's lazy module loading (the default)
+ *    that lookup is also when the module holding the array is loaded on the
+ *    device, i.e. when its 64 MiB is reserved: make the first call at
+ *    start-up, outside any allocator callback and before any stream capture
+ *    (or set CUDA_MODULE_LOADING=EAGER to reserve it when the library is
+ *    loaded).  The address is cached per device and context and looked up
+ *    again after a context teardown such as cudaDeviceReset.
  *  - All calls on a device share the array and it keeps the last call's
  *    contents; each call rewrites everything that must start at zero before
  *    using it.  Calls whose kernels overlap on the GPU (unordered streams)
@@ -141,6 +151,122 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
                            int H, int N, int d, float softmax_scale, int causal,
                            const int32_t* seqlens, float dropout_p, uint64_t seed,
                            const uint8_t* block_mask, void* stream);
+
+/* ------------------------------------------------------------------------
+ * General layouts: strided tensors, packed variable-length batches, N_q != N_k
+ * ------------------------------------------------------------------------
+ * The pages' BERT-large workload is a batch of sequences of different
+ * lengths (researchpapers.dev "FlashAttention 详解", section 关键结果); the
+ * entry points below take them packed, with no padding rows, as well as
+ * token-major ([B, N, H, d]) or any other strided layout whose d is
+ * contiguous, different query and key counts, and head dims 32, 64, 96, 128.
+ * The computation is the one above, per batch entry (or packed sequence) b:
+ *  - positions i, j are counted inside sequence b (masks, dropout counter);
+ *  - causal: query i attends key j iff j <= i + Nk_b - Nq_b, Nq_b / Nk_b the
+ *    sequence's query / key counts (bottom-right alignment: the last query
+ *    sees every key; rows with no key get O = 0, LSE = -inf); seqlens_k
+ *    masks keys j >= seqlens_k[b] without moving this alignment;
+ *  - block_mask: device uint8 [ceil(seqlen_q / 128)][ceil(seqlen_k / 128)],
+ *    indexed by (i / 128, j / 128), shared by all sequences and heads.
+ *
+ * Element strides of one tensor viewed as [batch, head, row, d], d contiguous.
+ * Every stride must be a non-negative multiple of 8 elements (16 bytes); the
+ * batch stride is ignored for the packed layout. */
+typedef struct {
+  int64_t batch, head, row;
+} fa_strides_t;
+
+typedef struct {
+  int batch;     /* B: batch entries (padded layout) or packed sequences */
+  int heads;     /* H */
+  int head_dim;  /* d: 32, 64, 96 or 128 */
+  /* Padded layout: rows of every batch entry (queries, keys).  Packed layout:
+   * an upper bound of every sequence's query / key count (longer sequences
+   * are cut to it). */
+  int seqlen_q, seqlen_k;
+  /* Packed layout: device int32[B + 1] offsets (0 = cu[0] <= ... <= cu[B]);
+   * sequence b's queries are rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 of
+   * Q, O, dO, dQ, its keys rows cu_seqlens_k[b] .. of K, V, dK, dV.  Both
+   * NULL for the padded layout, both set for the packed one.  Offsets are
+   * clamped to [0, total] on the device, so bad offsets give wrong results
+   * but never touch memory outside the tensors. */
+  const int32_t* cu_seqlens_q;
+  const int32_t* cu_seqlens_k;
+  int total_q, total_k; /* packed layout: rows of the packed tensors (>= 1) */
+  const int32_t* seqlens_k; /* key padding: device int32[B] or NULL */
+  float softmax_scale;
+  int causal;
+  float dropout_p;
+  uint64_t seed;
+  const uint8_t* block_mask;
+  fa_strides_t q, k, v, o, dout, dq, dk, dv;
+} fa_attention_desc_t;
+
+/* Forward pass for a general layout.  LSE is fp32 [B, H, seqlen_q]
+ * contiguous (padded layout) or [H, total_q] (packed layout).  Rows of O and
+ * LSE past a sequence's end (padded layout) or that belong to no sequence
+ * (packed layout) are not written. */
+fa_status_t fa_fwd_ex(const fa_attention_desc_t* desc, const void* q, const void* k,
+                      const void* v, void* o, float* lse, void* stream);
+
+/* Workspace bytes of fa_bwd_ex: padded layout B * H * ceil(seqlen_q / 128) * 128
+ * rows, packed layout H * (ceil(total_q / 128) * 128 + 256 B) rows, each of
+ * 8 + 4 D bytes (D = 64 for d <= 64, else 128).  0 if the description is
+ * invalid. */
+size_t fa_bwd_ex_workspace_size(const fa_attention_desc_t* desc);
+
+/* Backward pass for a general layout (dQ like Q, dK / dV like K / V; the
+ * strides of each come from the description).  Same workspace rules as
+ * fa_bwd.  dK, dV rows of keys beyond a sequence's key length are 0. */
+fa_status_t fa_bwd_ex(const fa_attention_desc_t* desc, const void* q, const void* k,
+                      const void* v, const void* o, const float* lse, const void* dout, void* dq,
+                      void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Combining partial results (context-parallel attention)
+ * ------------------------------------------------------------------------
+ * When the keys are split into disjoint blocks that are processed apart (one
+ * block per GPU, the blocks passed around a ring), each block b gives a
+ * partial (O_b, LSE_b) normalised over its own keys, and the full result is
+ * LSE = ln sum_b exp(LSE_b), O = sum_b exp(LSE_b - LSE) O_b: the rescaling
+ * of the online softmax across key blocks (suanlizi.com summary, section
+ * 分块计算（Tiling）; researchpapers.dev, section 分块与重计算), applied between
+ * kernel calls instead of inside one.  The pages name multi-GPU IO-aware
+ * attention as the next step (suanlizi.com summary, future-work section on
+ * multi-GPU IO optimisation).
+ *
+ * fa_merge_partial: o_acc (fp32 [rows, d], 16-byte aligned) and lse_acc
+ *   (fp32 [rows]) hold the result so far (start: any finite o_acc, lse_acc =
+ *   -inf); merges in o_part (bf16 [rows, d], contiguous) with lse_part.
+ *   d in {32, 64, 96, 128}.  A part or accumulator with LSE = -inf adds
+ *   nothing; both empty gives O = 0, LSE = -inf.
+ * fa_accumulate_bf16: acc[i] += part[i] for i < n (fp32 += bf16), n a multiple
+ *   of 8, both 16-byte aligned: sums of gradient parts over key / query blocks.
+ * fa_convert_f32_bf16: out[i] = bf16(in[i]) (round to nearest even), n a
+ *   multiple of 8.
+ * All three are asynchronous on `stream` and allocate nothing. */
+fa_status_t fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part,
+                             const float* lse_part, int64_t rows, int d, void* stream);
+fa_status_t fa_accumulate_bf16(float* acc, const void* part, int64_t n, void* stream);
+fa_status_t fa_convert_f32_bf16(void* out, const float* in, int64_t n, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Fused QKV projection in front of attention
+ * ------------------------------------------------------------------------
+ * The pages extend IO-awareness to the model's other layers, which all read
+ * and write HBM (suanlizi.com summary, section IO-感知优化的普遍性).  This is
+ * the layer that feeds attention: with x bf16 [B N, d_model] (token t = b N + n,
+ * row-major), w bf16 [3 H d, d_model] (the three projection matrices stacked,
+ * as one linear layer stores them) and bias bf16 [3 H d] or NULL,
+ *   Y = x w^T + bias (fp32 accumulation, rounded once to bf16),
+ *   Q[b, h, n, e] = Y[b N + n, h d + e], K and V from columns H d + ... and
+ *   2 H d + ..., each written as bf16 [B, H, N, d] (fa_fwd's layout),
+ * with no intermediate [B N, 3 H d] tensor.  d is 64 or 128, H d a multiple of
+ * 128, d_model a multiple of 8, B N <= 65535 * 128; all pointers 16-byte
+ * aligned device memory owned by the caller.  Asynchronous on `stream`;
+ * bounded waits as in the attention kernels. */
+fa_status_t fa_qkv_projection(const void* x, const void* w, const void* bias, void* q, void* k,
+                              void* v, int B, int N, int H, int d, int d_model, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* fa_status_string(fa_status_t status);

@@ -21,6 +21,8 @@ from .build import LIB_PATH
 
 __all__ = [
     "FaError", "library", "forward", "backward", "backward_phases", "bwd_workspace_size",
+    "forward_general", "backward_general", "general_workspace_size",
+    "merge_partial", "accumulate_bf16", "convert_f32_bf16", "qkv_projection",
     "dropout_mask", "last_device_status", "set_wait_timeout_ns",
     "wait_timeout_probe", "STATUS",
 ]
@@ -45,8 +47,34 @@ _LIB = None
 _vp, _i, _f, _u64, _sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
                           ctypes.c_uint64, ctypes.c_size_t)
 
+class Strides(ctypes.Structure):
+    """fa_strides_t: element strides of a [batch, head, row, d] view."""
+    _fields_ = [("batch", ctypes.c_int64), ("head", ctypes.c_int64), ("row", ctypes.c_int64)]
+
+
+class AttentionDesc(ctypes.Structure):
+    """fa_attention_desc_t (include/fa.h), field for field."""
+    _fields_ = [
+        ("batch", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+        ("seqlen_q", ctypes.c_int), ("seqlen_k", ctypes.c_int),
+        ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+        ("total_q", ctypes.c_int), ("total_k", ctypes.c_int),
+        ("seqlens_k", ctypes.c_void_p),
+        ("softmax_scale", ctypes.c_float), ("causal", ctypes.c_int),
+        ("dropout_p", ctypes.c_float), ("seed", ctypes.c_uint64),
+        ("block_mask", ctypes.c_void_p),
+        ("q", Strides), ("k", Strides), ("v", Strides), ("o", Strides), ("dout", Strides),
+        ("dq", Strides), ("dk", Strides), ("dv", Strides),
+    ]
+
+
+_DP = ctypes.POINTER(AttentionDesc)
+
 # name -> (restype, argtypes); must match include/fa.h
 SIGNATURES = {
+    "fa_fwd_ex": (_i, [_DP, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fa_bwd_ex_workspace_size": (_sz, [_DP]),
+    "fa_bwd_ex": (_i, [_DP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fa_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _f, _u64, _vp, _vp]),
     "fa_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
     "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
@@ -57,6 +85,10 @@ SIGNATURES = {
     "fa_bwd_finish": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "fa_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                             _vp, _f, _u64, _vp, _vp]),
+    "fa_qkv_projection": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "fa_merge_partial": (_i, [_vp, _vp, _vp, _vp, ctypes.c_int64, _i, _vp]),
+    "fa_accumulate_bf16": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
+    "fa_convert_f32_bf16": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_last_device_status": (_i, [_vp]),
     "fa_set_wait_timeout_ns": (None, [_u64]),
@@ -233,3 +265,207 @@ def wait_timeout_probe(device=None):
     import torch
     _check(library().fa_debug_wait_timeout(_stream_ptr(device or torch.cuda.current_device())),
            "fa_debug_wait_timeout")
+
+
+# ---------------------------------------------------------------------------
+# general layouts: [B, H, N, d] / [B, N, H, d] with any strides, packed
+# variable-length batches [T, H, d], N_q != N_k, d in {32, 64, 96, 128}
+# ---------------------------------------------------------------------------
+
+def _strides(t, layout):
+    if t is None:
+        return Strides(0, 0, 0)
+    if t.stride(-1) != 1:
+        raise ValueError("the head dimension must be contiguous")
+    if layout == "bhsd":
+        return Strides(t.stride(0), t.stride(1), t.stride(2))
+    if layout == "bshd":
+        return Strides(t.stride(0), t.stride(2), t.stride(1))
+    if layout == "thd":
+        return Strides(0, t.stride(1), t.stride(0))
+    raise ValueError(f"unknown layout {layout!r}")
+
+
+def _dims(t, layout):
+    """(batch, rows, heads, d) of a tensor in the given layout."""
+    if layout == "bhsd":
+        return t.shape[0], t.shape[2], t.shape[1], t.shape[3]
+    if layout == "bshd":
+        return t.shape[0], t.shape[1], t.shape[2], t.shape[3]
+    return None, t.shape[0], t.shape[1], t.shape[2]
+
+
+def _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, scale, causal,
+          seqlens_k, dropout_p, seed, block_mask, tensors):
+    import torch
+    for t in (q, k):
+        if not t.is_cuda or t.dtype != torch.bfloat16:
+            raise ValueError("tensors must be bfloat16 on a CUDA device")
+    Bq, Nq, H, d = _dims(q, layout)
+    Bk, Nk, Hk, dk = _dims(k, layout)
+    if H != Hk or d != dk:
+        raise ValueError("q and k must have the same heads and head dim")
+    keep = []
+    a = AttentionDesc()
+    a.heads, a.head_dim = H, d
+    if layout == "thd":
+        if cu_seqlens_q is None or cu_seqlens_k is None:
+            raise ValueError("the packed layout needs cu_seqlens_q and cu_seqlens_k")
+        cq = torch.as_tensor(cu_seqlens_q, dtype=torch.int32, device=q.device).contiguous()
+        ck = torch.as_tensor(cu_seqlens_k, dtype=torch.int32, device=q.device).contiguous()
+        keep += [cq, ck]
+        a.batch = cq.numel() - 1
+        a.cu_seqlens_q, a.cu_seqlens_k = cq.data_ptr(), ck.data_ptr()
+        a.total_q, a.total_k = Nq, Nk
+        if max_seqlen_q is None or max_seqlen_k is None:
+            raise ValueError("the packed layout needs max_seqlen_q and max_seqlen_k")
+        a.seqlen_q, a.seqlen_k = int(max_seqlen_q), int(max_seqlen_k)
+    else:
+        if Bq != Bk:
+            raise ValueError("q and k must have the same batch size")
+        a.batch, a.seqlen_q, a.seqlen_k = Bq, Nq, Nk
+    sl, bm = _masks(seqlens_k, block_mask, q.device)
+    keep += [sl, bm]
+    a.seqlens_k = _ptr(sl)
+    a.block_mask = _ptr(bm)
+    a.softmax_scale = float(d ** -0.5 if scale is None else scale)
+    a.causal = int(bool(causal))
+    a.dropout_p = float(dropout_p)
+    a.seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+    for name, t in tensors.items():
+        setattr(a, name, _strides(t, layout))
+    return a, keep
+
+
+def forward_general(q, k, v, *, layout="bhsd", cu_seqlens_q=None, cu_seqlens_k=None,
+                    max_seqlen_q=None, max_seqlen_k=None, scale=None, causal=False,
+                    seqlens_k=None, dropout_p=0.0, seed=0, block_mask=None, out=None, lse=None):
+    """O, LSE for a general layout (fa_fwd_ex).
+
+    layout "bhsd": q [B, H, N_q, d], k / v [B, H, N_k, d]; "bshd": q [B, N_q, H, d],
+    k / v [B, N_k, H, d]; "thd": packed q [T_q, H, d], k / v [T_k, H, d] with int32
+    offsets cu_seqlens_q / cu_seqlens_k ([B + 1]) and the longest lengths.  Any
+    strides with d contiguous (multiples of 8 elements).  The causal mask is
+    bottom-right aligned per sequence.  LSE: [B, H, N_q] or [H, T_q] (packed).
+    """
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    a, keep = _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, scale,
+                    causal, seqlens_k, dropout_p, seed, block_mask,
+                    dict(q=q, k=k, v=v, o=out))
+    if lse is None:
+        if layout == "thd":
+            lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+        else:
+            B, Nq, H, _ = _dims(q, layout)
+            lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    code = library().fa_fwd_ex(ctypes.byref(a), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                               _stream_ptr(q.device))
+    _check(code, "fa_fwd_ex")
+    del keep
+    return out, lse
+
+
+def general_workspace_size(q, k, **kw):
+    """Workspace bytes of backward_general for these tensors and options."""
+    a, keep = _desc(q, k, kw.get("layout", "bhsd"), kw.get("cu_seqlens_q"),
+                    kw.get("cu_seqlens_k"), kw.get("max_seqlen_q"), kw.get("max_seqlen_k"),
+                    kw.get("scale"), kw.get("causal", False), kw.get("seqlens_k"),
+                    kw.get("dropout_p", 0.0), kw.get("seed", 0), kw.get("block_mask"),
+                    dict(q=q, k=k, v=k, o=q, dout=q, dq=q, dk=k, dv=k))
+    return int(library().fa_bwd_ex_workspace_size(ctypes.byref(a)))
+
+
+def backward_general(q, k, v, o, lse, dout, *, layout="bhsd", cu_seqlens_q=None,
+                     cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None, scale=None,
+                     causal=False, seqlens_k=None, dropout_p=0.0, seed=0, block_mask=None,
+                     workspace=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV for a general layout (fa_bwd_ex); arguments as forward_general."""
+    import torch
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    a, keep = _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, scale,
+                    causal, seqlens_k, dropout_p, seed, block_mask,
+                    dict(q=q, k=k, v=v, o=o, dout=dout, dq=dq, dk=dk, dv=dv))
+    lib = library()
+    need = int(lib.fa_bwd_ex_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    code = lib.fa_bwd_ex(ctypes.byref(a), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                         _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _stream_ptr(q.device))
+    _check(code, "fa_bwd_ex")
+    del keep
+    return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# combining partial results (context-parallel attention)
+# ---------------------------------------------------------------------------
+
+def merge_partial(o_acc, lse_acc, o_part, lse_part):
+    """o_acc (fp32 [..., d]), lse_acc (fp32 [...]) <- merge with the partial
+    result o_part (bf16 [..., d]), lse_part (fp32 [...]); in place."""
+    import torch
+    for t, dt in ((o_acc, torch.float32), (lse_acc, torch.float32), (o_part, torch.bfloat16),
+                  (lse_part, torch.float32)):
+        if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
+            raise ValueError("merge_partial: contiguous CUDA tensors of the documented dtypes")
+    d = o_acc.shape[-1]
+    rows = o_acc.numel() // d
+    if o_part.numel() != o_acc.numel() or lse_acc.numel() != rows or lse_part.numel() != rows:
+        raise ValueError("merge_partial: shapes differ")
+    _check(library().fa_merge_partial(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part),
+                                      rows, d, _stream_ptr(o_acc.device)), "fa_merge_partial")
+
+
+def accumulate_bf16(acc, part):
+    """acc (fp32) += part (bf16), elementwise, in place."""
+    import torch
+    if acc.dtype != torch.float32 or part.dtype != torch.bfloat16 or acc.numel() != part.numel():
+        raise ValueError("accumulate_bf16: fp32 accumulator and bf16 part of one size")
+    if not (acc.is_cuda and part.is_cuda and acc.is_contiguous() and part.is_contiguous()):
+        raise ValueError("accumulate_bf16: contiguous CUDA tensors")
+    _check(library().fa_accumulate_bf16(_ptr(acc), _ptr(part), acc.numel(),
+                                        _stream_ptr(acc.device)), "fa_accumulate_bf16")
+
+
+def convert_f32_bf16(src, out=None):
+    """bf16 copy of an fp32 tensor (round to nearest even)."""
+    import torch
+    if src.dtype != torch.float32 or not src.is_cuda or not src.is_contiguous():
+        raise ValueError("convert_f32_bf16: a contiguous fp32 CUDA tensor")
+    out = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device) if out is None else out
+    _check(library().fa_convert_f32_bf16(_ptr(out), _ptr(src), src.numel(),
+                                         _stream_ptr(src.device)), "fa_convert_f32_bf16")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# fused QKV projection
+# ---------------------------------------------------------------------------
+
+def qkv_projection(x, weight, bias, batch, heads, head_dim, q=None, k=None, v=None):
+    """Q, K, V [B, H, N, d] = split_heads(x @ weight.T + bias) in one kernel.
+
+    x: bf16 [B * N, d_model] (or [B, N, d_model]); weight: bf16 [3 H d, d_model];
+    bias: bf16 [3 H d] or None."""
+    import torch
+    x2 = x.reshape(-1, x.shape[-1])
+    for t in (x2, weight) + (() if bias is None else (bias,)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("qkv_projection: contiguous bf16 CUDA tensors")
+    T, dm = x2.shape
+    if T % batch:
+        raise ValueError("qkv_projection: tokens not divisible by the batch size")
+    N = T // batch
+    shape = (batch, heads, N, head_dim)
+    q, k, v = (torch.empty(shape, dtype=torch.bfloat16, device=x.device) if t is None else t
+               for t in (q, k, v))
+    code = library().fa_qkv_projection(_ptr(x2), _ptr(weight), _ptr(bias), _ptr(q), _ptr(k),
+                                       _ptr(v), batch, N, heads, head_dim, dm,
+                                       _stream_ptr(x.device))
+    _check(code, "fa_qkv_projection")
+    return q, k, v

@@ -1,9 +1,15 @@
 // C ABI of the attention library: argument validation, TMA descriptor set-up
 // and kernel launch.  See include/fa.h for the contract of every entry point.
+//
+// Every entry point first turns its arguments into one validated Problem (the
+// classic [B, H, N, d] calls are the padded layout with contiguous strides and
+// N_q = N_k = N); the launches below only ever see a Problem.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
 
+#include "devctx.h"
 #include "fa.h"
 #include "kernels.h"
 #include "tmap.h"
@@ -14,38 +20,19 @@ namespace {
 // file-scope __device__ variable, so no allocation happens at run time).
 __device__ int g_status_word;
 
-constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices] = {nullptr};
-std::mutex g_status_mutex;
-uint64_t g_timeout_ns = 4000000000ull;
+fa::SymbolAddressCache g_status_cache;
+std::atomic<uint64_t> g_timeout_ns{4000000000ull};
 
+// Device address of the status word in the current device's context.
 int* status_word() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_status_mutex);
-  if (g_status_ptr[dev] == nullptr) {
+  return static_cast<int*>(g_status_cache.get([]() -> void* {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int*>(ptr);
-  }
-  return g_status_ptr[dev];
+    return ptr;
+  }));
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-
-// Checks shared by the forward and backward entry points.
-fa_status_t check_shape(int B, int H, int N, int d, float scale, float dropout_p) {
-  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(B) * H > 65535) return FA_ERR_UNSUPPORTED;
-  if (N > (1 << 23)) return FA_ERR_UNSUPPORTED;
-  // one CTA per (b, h, 128-row tile) in a 1-D grid
-  if (static_cast<int64_t>(B) * H * ((N + 127) / 128) > 0x7FFFFFFF) return FA_ERR_UNSUPPORTED;
-  return FA_OK;
-}
-
 bool tensor_ok(const void* p) { return p != nullptr && aligned(p, 16); }
 
 struct Dropout {
@@ -64,8 +51,326 @@ Dropout dropout_params(float p) {
 }
 
 constexpr double kLog2e = 1.4426950408889634074;
+constexpr int kMaxRows = 1 << 23;
 
-int64_t padded_rows(int N) { return (static_cast<int64_t>(N) + 127) / 128 * 128; }
+// Kernel width for a head dimension (0 if unsupported): 32 and 96 run the 64-
+// and 128-wide kernels, whose extra columns TMA fills with zeros.
+int kernel_dim(int d) {
+  if (d == 32 || d == 64) return 64;
+  if (d == 96 || d == 128) return 128;
+  return 0;
+}
+
+// A validated request.
+struct Problem {
+  int B, H, d, D;
+  int nq, nk;                  // padded: rows per entry; packed: longest sequence
+  bool packed;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int total_q, total_k;        // packed: rows of the tensors
+  const int32_t* seqlens;
+  float scale;
+  int causal;
+  float dropout_p;
+  uint64_t seed;
+  const uint8_t* block_mask;
+  fa_strides_t q, k, v, o, dout, dq, dk, dv;
+
+  int rows_q() const { return packed ? total_q : nq; }
+  int rows_k() const { return packed ? total_k : nk; }
+  int tb() const { return packed ? 1 : B; }
+};
+
+bool strides_ok(const fa_strides_t& s, bool packed) {
+  if (s.head < 0 || s.row < 0 || (!packed && s.batch < 0)) return false;
+  if (s.head % 8 || s.row % 8 || (!packed && s.batch % 8)) return false;
+  return s.head < (int64_t{1} << 36) && s.row < (int64_t{1} << 36) &&
+         (packed || s.batch < (int64_t{1} << 36));
+}
+
+// The tensors a call uses: the forward reads Q, K, V and writes O; the
+// backward (and its workspace size) uses all eight.  Strides of unused tensors
+// are not looked at.
+enum Uses { kForward, kBackward };
+
+fa_status_t resolve(const fa_attention_desc_t* a, Problem* p, Uses uses) {
+  if (a == nullptr) return FA_ERR_INVALID_ARG;
+  if (a->batch < 1 || a->heads < 1 || a->seqlen_q < 1 || a->seqlen_k < 1)
+    return FA_ERR_INVALID_ARG;
+  if (!(a->softmax_scale > 0.f) || !std::isfinite(a->softmax_scale)) return FA_ERR_INVALID_ARG;
+  if (!(a->dropout_p >= 0.f && a->dropout_p < 1.f)) return FA_ERR_INVALID_ARG;
+  if ((a->cu_seqlens_q == nullptr) != (a->cu_seqlens_k == nullptr)) return FA_ERR_INVALID_ARG;
+  const bool packed = a->cu_seqlens_q != nullptr;
+  if (packed && (!aligned(a->cu_seqlens_q, 4) || !aligned(a->cu_seqlens_k, 4) ||
+                 a->total_q < 1 || a->total_k < 1))
+    return FA_ERR_INVALID_ARG;
+  if (a->seqlens_k != nullptr && !aligned(a->seqlens_k, 4)) return FA_ERR_INVALID_ARG;
+  const int D = kernel_dim(a->head_dim);
+  if (D == 0) return FA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(a->batch) * a->heads > 65535) return FA_ERR_UNSUPPORTED;
+  if (a->seqlen_q > kMaxRows || a->seqlen_k > kMaxRows) return FA_ERR_UNSUPPORTED;
+  // one CTA per (b, h, 128-row tile) in a 1-D grid
+  const int64_t tiles = (static_cast<int64_t>(a->seqlen_q > a->seqlen_k ? a->seqlen_q : a->seqlen_k) +
+                         127) / 128;
+  if (static_cast<int64_t>(a->batch) * a->heads * tiles > 0x7FFFFFFF) return FA_ERR_UNSUPPORTED;
+  const fa_strides_t* all[8] = {&a->q, &a->k, &a->v, &a->o, &a->dout, &a->dq, &a->dk, &a->dv};
+  for (int t = 0; t < (uses == kForward ? 4 : 8); ++t) {
+    const fa_strides_t* s = all[t];
+    if (!strides_ok(*s, packed)) return FA_ERR_INVALID_ARG;
+    // a zero stride would make heads / entries / rows share memory
+    if ((a->heads > 1 && s->head == 0) || (!packed && a->batch > 1 && s->batch == 0) ||
+        s->row == 0)
+      return FA_ERR_INVALID_ARG;
+  }
+  p->B = a->batch;
+  p->H = a->heads;
+  p->d = a->head_dim;
+  p->D = D;
+  p->nq = a->seqlen_q;
+  p->nk = a->seqlen_k;
+  p->packed = packed;
+  p->cu_q = a->cu_seqlens_q;
+  p->cu_k = a->cu_seqlens_k;
+  p->total_q = packed ? a->total_q : 0;
+  p->total_k = packed ? a->total_k : 0;
+  p->seqlens = a->seqlens_k;
+  p->scale = a->softmax_scale;
+  p->causal = a->causal != 0;
+  p->dropout_p = a->dropout_p;
+  p->seed = a->seed;
+  p->block_mask = a->block_mask;
+  p->q = a->q;
+  p->k = a->k;
+  p->v = a->v;
+  p->o = a->o;
+  p->dout = a->dout;
+  p->dq = a->dq;
+  p->dk = a->dk;
+  p->dv = a->dv;
+  if (packed) {  // the batch coordinate is always 0
+    for (fa_strides_t* s : {&p->q, &p->k, &p->v, &p->o, &p->dout, &p->dq, &p->dk, &p->dv})
+      s->batch = 0;
+  }
+  return FA_OK;
+}
+
+// The classic contiguous [B, H, N, d] request.
+fa_attention_desc_t classic_desc(int B, int H, int N, int d, float scale, int causal,
+                                 const int32_t* seqlens, float dropout_p, uint64_t seed,
+                                 const uint8_t* block_mask) {
+  fa_attention_desc_t a{};
+  a.batch = B;
+  a.heads = H;
+  a.head_dim = d;
+  a.seqlen_q = N;
+  a.seqlen_k = N;
+  a.seqlens_k = seqlens;
+  a.softmax_scale = scale;
+  a.causal = causal;
+  a.dropout_p = dropout_p;
+  a.seed = seed;
+  a.block_mask = block_mask;
+  const fa_strides_t s{static_cast<int64_t>(H) * N * d, static_cast<int64_t>(N) * d, d};
+  a.q = a.k = a.v = a.o = a.dout = a.dq = a.dk = a.dv = s;
+  return a;
+}
+
+fa::Strides kstrides(const fa_strides_t& s) { return fa::Strides{s.batch, s.head, s.row}; }
+
+fa::Rows kernel_rows(const Problem& p) {
+  fa::Rows r;
+  r.cu_q = p.cu_q;
+  r.cu_k = p.cu_k;
+  r.nq = p.nq;
+  r.nk = p.nk;
+  r.total_q = p.total_q;
+  r.total_k = p.total_k;
+  return r;
+}
+
+// TMA view {d, rows, H, batch} of a bf16 tensor; box 64 x 128 x 1 x 1.
+bool tmap(CUtensorMap* m, const void* base, const Problem& p, const fa_strides_t& s, int rows) {
+  fa::TmapDesc t = fa::tmap_desc_zero();
+  t.base = base;
+  t.dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  t.rank = 4;
+  t.dims[0] = static_cast<uint64_t>(p.d);
+  t.dims[1] = static_cast<uint64_t>(rows);
+  t.dims[2] = static_cast<uint64_t>(p.H);
+  t.dims[3] = static_cast<uint64_t>(p.tb());
+  // a zero stride (a single head or batch entry) is described as the
+  // smallest legal one; that coordinate is always 0
+  t.strides[0] = static_cast<uint64_t>(s.row ? s.row : 8) * 2;
+  t.strides[1] = static_cast<uint64_t>(s.head ? s.head : 8) * 2;
+  t.strides[2] = static_cast<uint64_t>(s.batch ? s.batch : 8) * 2;
+  t.box[0] = 64;
+  t.box[1] = 128;
+  t.box[2] = 1;
+  t.box[3] = 1;
+  return fa::tmap_cache().encode(t, m);
+}
+
+// LSE element strides of a batch entry and a head.
+void lse_strides(const Problem& p, long long* sb, long long* sh) {
+  if (p.packed) {
+    *sb = 0;
+    *sh = p.total_q;
+  } else {
+    *sb = static_cast<long long>(p.H) * p.nq;
+    *sh = p.nq;
+  }
+}
+
+// Rows of each workspace array (a multiple of 128), with the padded layout's
+// rows per (b, h) or the packed layout's rows per head.
+int64_t ws_rows(const Problem& p, int* npad, int64_t* rtot) {
+  if (!p.packed) {
+    *npad = (p.nq + 127) / 128 * 128;
+    *rtot = 0;
+    return static_cast<int64_t>(p.B) * p.H * *npad;
+  }
+  *npad = 0;
+  *rtot = (static_cast<int64_t>(p.total_q) + 127) / 128 * 128 + 256ll * p.B;
+  return static_cast<int64_t>(p.H) * *rtot;
+}
+
+size_t workspace_bytes_of(const Problem& p) {
+  int npad = 0;
+  int64_t rtot = 0;
+  const uint64_t rows = static_cast<uint64_t>(ws_rows(p, &npad, &rtot));
+  const uint64_t bytes = rows * (4ull + 4ull + 4ull * p.D);
+  return static_cast<size_t>((bytes + 255) / 256 * 256);
+}
+
+fa_status_t run_fwd(const Problem& pr, const void* q, const void* k, const void* v, void* o,
+                    float* lse, void* stream) {
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(o)) return FA_ERR_INVALID_ARG;
+  if (lse == nullptr || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  int* status = status_word();
+  if (status == nullptr) return FA_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (!tmap(&tq, q, pr, pr.q, pr.rows_q()) || !tmap(&tk, k, pr, pr.k, pr.rows_k()) ||
+      !tmap(&tv, v, pr, pr.v, pr.rows_k()))
+    return FA_ERR_UNSUPPORTED;
+  const Dropout dr = dropout_params(pr.dropout_p);
+  fa::FwdParams p{};
+  p.o = o;
+  p.so = kstrides(pr.o);
+  p.lse = lse;
+  lse_strides(pr, &p.lse_sb, &p.lse_sh);
+  p.seqlens = pr.seqlens;
+  p.block_mask = pr.block_mask;
+  p.nbq = (pr.nq + 127) / 128;
+  p.nbk = (pr.nk + 127) / 128;
+  p.status = status;
+  p.rows = kernel_rows(pr);
+  p.B = pr.B;
+  p.H = pr.H;
+  p.d_real = pr.d;
+  p.scale_log2 = static_cast<float>(static_cast<double>(pr.scale) * kLog2e);
+  p.causal = pr.causal;
+  p.group_heads = fa::order_group_heads(pr.B, pr.H, fa::fwd_head_bytes(pr.nk, pr.D), pr.causal);
+  p.drop_threshold = dr.threshold;
+  p.drop_rscale = dr.rscale;
+  p.seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
+  p.seed_hi = static_cast<uint32_t>(pr.seed >> 32);
+  p.rk = fa::philox_round_keys(pr.seed);
+  p.timeout_ns = g_timeout_ns.load();
+  const cudaError_t e =
+      fa::launch_fwd(pr.D, dr.threshold != 0, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Scalar and workspace fields shared by the three backward launches.
+fa_status_t bwd_params(fa::BwdParams* p, const Problem& pr, const void* workspace,
+                       size_t workspace_bytes) {
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < workspace_bytes_of(pr))
+    return FA_ERR_WORKSPACE;
+  int* status = status_word();
+  if (status == nullptr) return FA_ERR_CUDA;
+  const Dropout dr = dropout_params(pr.dropout_p);
+  *p = fa::BwdParams{};
+  int npad = 0;
+  int64_t rtot = 0;
+  const int64_t rows = ws_rows(pr, &npad, &rtot);
+  if (rows > 0x7FFFFFFFll) return FA_ERR_UNSUPPORTED;  // TMA row coordinate of the dQ reduce
+  p->ws_lse2 = static_cast<float*>(const_cast<void*>(workspace));
+  p->ws_delta = p->ws_lse2 + rows;
+  p->ws_dq = p->ws_delta + rows;
+  p->ws_rows = rows;
+  p->Npad = npad;
+  p->Rtot = rtot;
+  lse_strides(pr, &p->lse_sb, &p->lse_sh);
+  p->so = kstrides(pr.o);
+  p->sdo = kstrides(pr.dout);
+  p->sdq = kstrides(pr.dq);
+  p->sdk = kstrides(pr.dk);
+  p->sdv = kstrides(pr.dv);
+  p->seqlens = pr.seqlens;
+  p->block_mask = pr.block_mask;
+  p->nbq = (pr.nq + 127) / 128;
+  p->nbk = (pr.nk + 127) / 128;
+  p->status = status;
+  p->rows = kernel_rows(pr);
+  p->B = pr.B;
+  p->H = pr.H;
+  p->d_real = pr.d;
+  p->scale = pr.scale;
+  p->scale_log2 = static_cast<float>(static_cast<double>(pr.scale) * kLog2e);
+  p->causal = pr.causal;
+  p->group_heads = fa::order_group_heads(pr.B, pr.H, fa::bwd_head_bytes(pr.nq, pr.D), pr.causal);
+  p->drop_threshold = dr.threshold;
+  p->drop_rscale = dr.rscale;
+  p->seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
+  p->seed_hi = static_cast<uint32_t>(pr.seed >> 32);
+  p->rk = fa::philox_round_keys(pr.seed);
+  p->timeout_ns = g_timeout_ns.load();
+  return FA_OK;
+}
+
+// Tensor maps of the main backward kernel.
+struct BwdMaps {
+  CUtensorMap q, k, v, dout, dq;
+};
+
+fa_status_t bwd_maps(BwdMaps* m, const Problem& pr, const fa::BwdParams& p, const void* q,
+                     const void* k, const void* v, const void* dout) {
+  if (!tmap(&m->q, q, pr, pr.q, pr.rows_q()) || !tmap(&m->k, k, pr, pr.k, pr.rows_k()) ||
+      !tmap(&m->v, v, pr, pr.v, pr.rows_k()) || !tmap(&m->dout, dout, pr, pr.dout, pr.rows_q()))
+    return FA_ERR_UNSUPPORTED;
+  if (!fa::make_tmap_f32_2d(&m->dq, p.ws_dq, static_cast<uint64_t>(pr.D),
+                            static_cast<uint64_t>(p.ws_rows), 128))
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+fa_status_t run_bwd(const Problem& pr, const void* q, const void* k, const void* v, const void* o,
+                    const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(o) || !tensor_ok(dout) ||
+      !tensor_ok(dq) || !tensor_ok(dk) || !tensor_ok(dv))
+    return FA_ERR_INVALID_ARG;
+  if (lse == nullptr || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  fa::BwdParams p;
+  fa_status_t st = bwd_params(&p, pr, workspace, workspace_bytes);
+  if (st != FA_OK) return st;
+  BwdMaps m;
+  st = bwd_maps(&m, pr, p, q, k, v, dout);
+  if (st != FA_OK) return st;
+  p.o = o;
+  p.lse = lse;
+  p.dout = dout;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fa::launch_bwd_pre(pr.D, p, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (fa::launch_bwd_main(pr.D, p.drop_threshold != 0, m.q, m.k, m.v, m.dout, m.dq, p, s) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  return fa::launch_bwd_post(pr.D, p, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -83,7 +388,7 @@ const char* fa_status_string(fa_status_t s) {
   return "unknown status";
 }
 
-void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns < 1000000ull ? 1000000ull : ns; }
+void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns < 1000000ull ? 1000000ull : ns); }
 
 fa_status_t fa_last_device_status(void* stream) {
   int* w = status_word();
@@ -101,104 +406,61 @@ fa_status_t fa_last_device_status(void* stream) {
 fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                    int N, int d, float softmax_scale, int causal, const int32_t* seqlens,
                    float dropout_p, uint64_t seed, const uint8_t* block_mask, void* stream) {
-  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(o)) return FA_ERR_INVALID_ARG;
-  if (lse == nullptr || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
   if (seqlens != nullptr && !aligned(seqlens, 4)) return FA_ERR_INVALID_ARG;
-  fa_status_t st = check_shape(B, H, N, d, softmax_scale, dropout_p);
+  const fa_attention_desc_t a =
+      classic_desc(B, H, N, d, softmax_scale, causal, seqlens, dropout_p, seed, block_mask);
+  Problem pr;
+  const fa_status_t st = resolve(&a, &pr, kForward);
   if (st != FA_OK) return st;
+  return run_fwd(pr, q, k, v, o, lse, stream);
+}
 
-  int* status = status_word();
-  if (status == nullptr) return FA_ERR_CUDA;
-  CUtensorMap tq, tk, tv;
-  const uint64_t bh = static_cast<uint64_t>(B) * H;
-  if (!fa::make_tmap_bf16(&tq, q, d, N, bh, 128) || !fa::make_tmap_bf16(&tk, k, d, N, bh, 128) ||
-      !fa::make_tmap_bf16(&tv, v, d, N, bh, 128))
-    return FA_ERR_CUDA;
-
-  const Dropout dr = dropout_params(dropout_p);
-  fa::FwdParams p{};
-  p.o = o;
-  p.lse = lse;
-  p.seqlens = seqlens;
-  p.block_mask = block_mask;
-  p.status = status;
-  p.B = B;
-  p.H = H;
-  p.N = N;
-  p.nblk = (N + 127) / 128;
-  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * kLog2e);
-  p.causal = causal != 0;
-  p.group_heads = fa::order_group_heads(B, H, N, d, causal != 0);
-  p.drop_threshold = dr.threshold;
-  p.drop_rscale = dr.rscale;
-  p.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
-  p.seed_hi = static_cast<uint32_t>(seed >> 32);
-  p.rk = fa::philox_round_keys(seed);
-  p.timeout_ns = g_timeout_ns;
-  const cudaError_t e =
-      fa::launch_fwd(d, dr.threshold != 0, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+fa_status_t fa_fwd_ex(const fa_attention_desc_t* desc, const void* q, const void* k,
+                      const void* v, void* o, float* lse, void* stream) {
+  Problem pr;
+  const fa_status_t st = resolve(desc, &pr, kForward);
+  if (st != FA_OK) return st;
+  return run_fwd(pr, q, k, v, o, lse, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
-  const uint64_t rows = static_cast<uint64_t>(B) * H * padded_rows(N);
-  const uint64_t bytes = rows * (4ull + 4ull + 4ull * d);
-  return static_cast<size_t>((bytes + 255) / 256 * 256);
+  if (B < 1 || H < 1 || N < 1 || kernel_dim(d) == 0) return 0;
+  const fa_attention_desc_t a = classic_desc(B, H, N, d, 1.f, 0, nullptr, 0.f, 0, nullptr);
+  Problem pr;
+  if (resolve(&a, &pr, kBackward) != FA_OK) {  // sizes beyond the kernels' limits: still report the bytes
+    pr = Problem{};
+    pr.B = B;
+    pr.H = H;
+    pr.nq = N;
+    pr.D = kernel_dim(d);
+  }
+  return workspace_bytes_of(pr);
 }
 
-}  // extern "C"
-
-namespace {
-
-// Workspace views and scalar parameters shared by the three backward phases.
-fa_status_t bwd_params(fa::BwdParams* p, int B, int H, int N, int d, float softmax_scale,
-                       float dropout_p, const void* workspace, size_t workspace_bytes) {
-  fa_status_t st = check_shape(B, H, N, d, softmax_scale, dropout_p);
-  if (st != FA_OK) return st;
-  const size_t need = fa_bwd_workspace_size(B, H, N, d);
-  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need)
-    return FA_ERR_WORKSPACE;
-  int* status = status_word();
-  if (status == nullptr) return FA_ERR_CUDA;
-  const Dropout dr = dropout_params(dropout_p);
-  const int64_t npad = padded_rows(N);
-  const uint64_t bh = static_cast<uint64_t>(B) * H;
-  *p = fa::BwdParams{};
-  p->ws_lse2 = static_cast<float*>(const_cast<void*>(workspace));
-  p->ws_delta = p->ws_lse2 + bh * npad;
-  p->ws_dq = p->ws_delta + bh * npad;
-  p->status = status;
-  p->B = B;
-  p->H = H;
-  p->N = N;
-  p->Npad = static_cast<int>(npad);
-  p->nblk = (N + 127) / 128;
-  p->scale = softmax_scale;
-  p->scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * kLog2e);
-  p->drop_threshold = dr.threshold;
-  p->drop_rscale = dr.rscale;
-  p->timeout_ns = g_timeout_ns;
-  return FA_OK;
+size_t fa_bwd_ex_workspace_size(const fa_attention_desc_t* desc) {
+  Problem pr;
+  if (resolve(desc, &pr, kBackward) != FA_OK) return 0;
+  return workspace_bytes_of(pr);
 }
-
-}  // namespace
-
-extern "C" {
 
 fa_status_t fa_bwd_prepare(const void* o, const float* lse, const void* dout, int B, int H, int N,
                            int d, void* workspace, size_t workspace_bytes, void* stream) {
   if (!tensor_ok(o) || !tensor_ok(dout)) return FA_ERR_INVALID_ARG;
   if (lse == nullptr || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
-  fa::BwdParams p;
   // scale and dropout do not enter this phase: validate with neutral values
-  fa_status_t st = bwd_params(&p, B, H, N, d, 1.f, 0.f, workspace, workspace_bytes);
+  const fa_attention_desc_t a = classic_desc(B, H, N, d, 1.f, 0, nullptr, 0.f, 0, nullptr);
+  Problem pr;
+  fa_status_t st = resolve(&a, &pr, kBackward);
+  if (st != FA_OK) return st;
+  fa::BwdParams p;
+  st = bwd_params(&p, pr, workspace, workspace_bytes);
   if (st != FA_OK) return st;
   p.o = o;
   p.lse = lse;
   p.dout = dout;
-  return fa::launch_bwd_pre(d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK
-                                                                                     : FA_ERR_CUDA;
+  return fa::launch_bwd_pre(pr.D, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
 }
 
 fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dk,
@@ -210,39 +472,40 @@ fa_status_t fa_bwd_main(const void* q, const void* k, const void* v, const void*
       !tensor_ok(dv))
     return FA_ERR_INVALID_ARG;
   if (seqlens != nullptr && !aligned(seqlens, 4)) return FA_ERR_INVALID_ARG;
-  fa::BwdParams p;
-  fa_status_t st =
-      bwd_params(&p, B, H, N, d, softmax_scale, dropout_p, workspace, workspace_bytes);
+  const fa_attention_desc_t a =
+      classic_desc(B, H, N, d, softmax_scale, causal, seqlens, dropout_p, seed, block_mask);
+  Problem pr;
+  fa_status_t st = resolve(&a, &pr, kBackward);
   if (st != FA_OK) return st;
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  const uint64_t bh = static_cast<uint64_t>(B) * H;
-  if (!fa::make_tmap_bf16(&tq, q, d, N, bh, 128) || !fa::make_tmap_bf16(&tk, k, d, N, bh, 128) ||
-      !fa::make_tmap_bf16(&tv, v, d, N, bh, 128) || !fa::make_tmap_bf16(&tdo, dout, d, N, bh, 128) ||
-      !fa::make_tmap_f32_2d(&tdq, p.ws_dq, d, bh * static_cast<uint64_t>(p.Npad), 128))
-    return FA_ERR_CUDA;
+  fa::BwdParams p;
+  st = bwd_params(&p, pr, workspace, workspace_bytes);
+  if (st != FA_OK) return st;
+  BwdMaps m;
+  st = bwd_maps(&m, pr, p, q, k, v, dout);
+  if (st != FA_OK) return st;
+  p.dout = dout;
   p.dk = dk;
   p.dv = dv;
-  p.seqlens = seqlens;
-  p.block_mask = block_mask;
-  p.causal = causal != 0;
-  p.group_heads = fa::order_group_heads(B, H, N, d, causal != 0);
-  p.seed_lo = static_cast<uint32_t>(seed & 0xFFFFFFFFull);
-  p.seed_hi = static_cast<uint32_t>(seed >> 32);
-  p.rk = fa::philox_round_keys(seed);
-  const cudaError_t e = fa::launch_bwd_main(d, p.drop_threshold != 0, tq, tk, tv, tdo, tdq, p,
-                                            static_cast<cudaStream_t>(stream));
+  const cudaError_t e = fa::launch_bwd_main(pr.D, p.drop_threshold != 0, m.q, m.k, m.v, m.dout,
+                                            m.dq, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status_t fa_bwd_finish(void* dq, int B, int H, int N, int d, float softmax_scale,
                           const void* workspace, size_t workspace_bytes, void* stream) {
   if (!tensor_ok(dq)) return FA_ERR_INVALID_ARG;
+  const fa_attention_desc_t a =
+      classic_desc(B, H, N, d, softmax_scale, 0, nullptr, 0.f, 0, nullptr);
+  Problem pr;
+  fa_status_t st = resolve(&a, &pr, kBackward);
+  if (st != FA_OK) return st;
   fa::BwdParams p;
-  fa_status_t st = bwd_params(&p, B, H, N, d, softmax_scale, 0.f, workspace, workspace_bytes);
+  st = bwd_params(&p, pr, workspace, workspace_bytes);
   if (st != FA_OK) return st;
   p.dq = dq;
-  return fa::launch_bwd_post(d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK
-                                                                                     : FA_ERR_CUDA;
+  return fa::launch_bwd_post(pr.D, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
 }
 
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -250,22 +513,42 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
                    float softmax_scale, int causal, const int32_t* seqlens, float dropout_p,
                    uint64_t seed, const uint8_t* block_mask, void* workspace,
                    size_t workspace_bytes, void* stream) {
-  // validate everything before the first launch
-  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(o) || !tensor_ok(dout) ||
-      !tensor_ok(dq) || !tensor_ok(dk) || !tensor_ok(dv))
-    return FA_ERR_INVALID_ARG;
-  if (lse == nullptr || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
   if (seqlens != nullptr && !aligned(seqlens, 4)) return FA_ERR_INVALID_ARG;
-  fa::BwdParams chk;
-  fa_status_t st =
-      bwd_params(&chk, B, H, N, d, softmax_scale, dropout_p, workspace, workspace_bytes);
+  const fa_attention_desc_t a =
+      classic_desc(B, H, N, d, softmax_scale, causal, seqlens, dropout_p, seed, block_mask);
+  Problem pr;
+  const fa_status_t st = resolve(&a, &pr, kBackward);
   if (st != FA_OK) return st;
-  st = fa_bwd_prepare(o, lse, dout, B, H, N, d, workspace, workspace_bytes, stream);
+  return run_bwd(pr, q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, stream);
+}
+
+fa_status_t fa_bwd_ex(const fa_attention_desc_t* desc, const void* q, const void* k,
+                      const void* v, const void* o, const float* lse, const void* dout, void* dq,
+                      void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+  Problem pr;
+  const fa_status_t st = resolve(desc, &pr, kBackward);
   if (st != FA_OK) return st;
-  st = fa_bwd_main(q, k, v, dout, dk, dv, B, H, N, d, softmax_scale, causal, seqlens, dropout_p,
-                   seed, block_mask, workspace, workspace_bytes, stream);
-  if (st != FA_OK) return st;
-  return fa_bwd_finish(dq, B, H, N, d, softmax_scale, workspace, workspace_bytes, stream);
+  return run_bwd(pr, q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, stream);
+}
+
+fa_status_t fa_qkv_projection(const void* x, const void* w, const void* bias, void* q, void* k,
+                              void* v, int B, int N, int H, int d, int d_model, void* stream) {
+  if (!tensor_ok(x) || !tensor_ok(w) || !tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v))
+    return FA_ERR_INVALID_ARG;
+  if (bias != nullptr && !aligned(bias, 16)) return FA_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H < 1 || d_model < 8 || d_model % 8) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if ((static_cast<int64_t>(H) * d) % 128) return FA_ERR_UNSUPPORTED;
+  const int64_t T = static_cast<int64_t>(B) * N;
+  if (T > 65535ll * 128 || static_cast<int64_t>(H) * d * 3 / 128 > 0x7FFFFFFF ||
+      d_model > (1 << 24))
+    return FA_ERR_UNSUPPORTED;
+  int* status = status_word();
+  if (status == nullptr) return FA_ERR_CUDA;
+  const cudaError_t e = fa::launch_qkv_projection(x, w, bias, q, k, v, B, N, H, d, d_model, status,
+                                                  g_timeout_ns.load(),
+                                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status_t fa_debug_dropout_mask(uint8_t* keep, int B, int H, int N, float dropout_p,
@@ -283,7 +566,7 @@ fa_status_t fa_debug_wait_timeout(void* stream) {
   int* status = status_word();
   if (status == nullptr) return FA_ERR_CUDA;
   const cudaError_t e =
-      fa::launch_wait_timeout_probe(status, g_timeout_ns, static_cast<cudaStream_t>(stream));
+      fa::launch_wait_timeout_probe(status, g_timeout_ns.load(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -44,6 +44,7 @@
 
 #include <type_traits>
 
+#include "devctx.h"
 #include "kernels.h"
 #include "philox.cuh"
 #include "ptx.cuh"
@@ -101,14 +102,20 @@ struct BwdLayout {
   static_assert(COL_DK + D <= 512, "TMEM budget");
 };
 
+// The key tile of this CTA and the query tiles that meet it.  Rows and keys
+// are counted inside the CTA's sequence; qrow / krow are the tensor rows of the
+// sequence's first query / key, tb its batch coordinate and ws0 its first
+// workspace row.  Under the causal mask query i sees key j iff j <= i + off
+// (bottom-right alignment, off = keys - queries of the sequence).
 struct BwdWork {
-  int b, h, bh, kb, kv_len, nqb, qb_begin, nblk;
+  int b, h, bh, kb, kv_len, nqb, qb_begin, nbk, off, qrow, krow, tb, lk;
+  long long ws0;
   bool alive, causal;
   const uint8_t* bm;
 
   __device__ __forceinline__ bool act(int qb) const {
     if (!alive) return false;
-    if (bm != nullptr && bm[static_cast<size_t>(qb) * nblk + kb] == 0) return false;
+    if (bm != nullptr && bm[static_cast<size_t>(qb) * nbk + kb] == 0) return false;
     return true;
   }
   __device__ __forceinline__ int next(int qb) const {
@@ -121,22 +128,30 @@ struct BwdWork {
 // pre / post kernels
 // ---------------------------------------------------------------------------
 
+// Grid of the pre / post kernels: blockIdx.y = (b, h), blockIdx.x = a block
+// of kRowsPerBlock<D> query rows, D / 8 threads per row (8 columns each).
+template <int D>
+constexpr int kRowsPerBlock = 256 / (D / 8);
+
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   constexpr int G = D / 8;  // threads per row, 8 elements each
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t row = tid / G;
-  const int part = static_cast<int>(tid % G);
-  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Npad;
-  if (row >= rows) return;  // whole warps: rows is a multiple of 128
-  const int64_t bh = row / p.Npad;
-  const int i = static_cast<int>(row % p.Npad);
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh % p.H;
+  const Seq sq = seq_of(p.rows, b);
+  const int i = blockIdx.x * kRowsPerBlock<D> + static_cast<int>(threadIdx.x) / G;
+  const int part = static_cast<int>(threadIdx.x) % G;
+  // rows up to the next multiple of 128 are written (padding rows included);
+  // the bound is a multiple of the block's rows, so whole blocks leave
+  if (blockIdx.x * kRowsPerBlock<D> >= (sq.lq + 127) / 128 * 128) return;
   float acc = 0.f;
-  if (i < p.N) {
-    const size_t off = (static_cast<size_t>(bh) * p.N + i) * D + part * 8;
-    const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + off);
-    const uint4 gv =
-        *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + off);
+  if (i < sq.lq && part * 8 < p.d_real) {
+    const long long r = sq.q0 + i;
+    const uint4 ov = *reinterpret_cast<const uint4*>(
+        static_cast<const __nv_bfloat16*>(p.o) + sq.tb * p.so.b + h * p.so.h + r * p.so.r + part * 8);
+    const uint4 gv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) +
+                                                     sq.tb * p.sdo.b + h * p.sdo.h + r * p.sdo.r +
+                                                     part * 8);
     const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
     const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
 #pragma unroll
@@ -149,11 +164,12 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   }
 #pragma unroll
   for (int m = G / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  const long long row = ws_row0(p, b, h, sq.q0) + i;
   if (part == 0) {
-    p.ws_delta[row] = (i < p.N) ? -acc : 0.f;
+    p.ws_delta[row] = (i < sq.lq) ? -acc : 0.f;
     float nl2 = -INFINITY;
-    if (i < p.N) {
-      const float l = p.lse[static_cast<size_t>(bh) * p.N + i];
+    if (i < sq.lq) {
+      const float l = p.lse[sq.tb * p.lse_sb + h * p.lse_sh + sq.q0 + i];
       if (l != -INFINITY) nl2 = -l * kLog2e;
     }
     p.ws_lse2[row] = nl2;
@@ -165,14 +181,15 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
 
 template <int D>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(p.B) * p.H * p.N * (D / 8);
-  if (tid >= total) return;
-  const int64_t row = tid / (D / 8);  // bh * N + i
-  const int part = static_cast<int>(tid % (D / 8));
-  const int64_t bh = row / p.N;
-  const int64_t i = row % p.N;
-  const float4* src = reinterpret_cast<const float4*>(p.ws_dq + (bh * p.Npad + i) * D + part * 8);
+  constexpr int G = D / 8;
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh % p.H;
+  const Seq sq = seq_of(p.rows, b);
+  const int i = blockIdx.x * kRowsPerBlock<D> + static_cast<int>(threadIdx.x) / G;
+  const int part = static_cast<int>(threadIdx.x) % G;
+  if (i >= sq.lq || part * 8 >= p.d_real) return;
+  const float4* src = reinterpret_cast<const float4*>(
+      p.ws_dq + (ws_row0(p, b, h, sq.q0) + i) * D + part * 8);
   const float4 a = src[0], c = src[1];
   const float s = p.scale;
   uint4 out;
@@ -180,7 +197,8 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
   out.y = pack_bf16(a.z * s, a.w * s);
   out.z = pack_bf16(c.x * s, c.y * s);
   out.w = pack_bf16(c.z * s, c.w * s);
-  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dq) + row * D + part * 8) = out;
+  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dq) + sq.tb * p.sdq.b + h * p.sdq.h +
+                            static_cast<long long>(sq.q0 + i) * p.sdq.r + part * 8) = out;
 }
 
 // ---------------------------------------------------------------------------
@@ -212,19 +230,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
 
   BwdWork w;
-  grid_unit(blockIdx.x, p.B * p.H, (p.N + 127) / 128, p.group_heads, &w.bh, &w.kb);  // key tile 0 is heaviest
+  grid_unit(blockIdx.x, p.B * p.H, (p.rows.nk + 127) / 128, p.group_heads, &w.bh,
+            &w.kb);  // key tile 0 is heaviest
   w.b = w.bh / p.H;
   w.h = w.bh % p.H;
   {
-    int kv = p.N;
-    if (p.seqlens != nullptr) kv = max(0, min(p.seqlens[w.b], p.N));
+    const Seq sq = seq_of(p.rows, w.b);
+    // a sequence shorter than the longest has no key tile here: leave before
+    // any set-up (the whole CTA takes this branch)
+    if (w.kb * 128 >= sq.lk) return;
+    int kv = sq.lk;
+    if (p.seqlens != nullptr) kv = max(0, min(p.seqlens[w.b], sq.lk));
     w.kv_len = kv;
+    w.lk = sq.lk;
+    w.qrow = sq.q0;
+    w.krow = sq.k0;
+    w.tb = sq.tb;
+    w.off = sq.lk - sq.lq;
+    w.nqb = (sq.lq + 127) / 128;
+    w.ws0 = ws_row0(p, w.b, w.h, sq.q0);
   }
   w.alive = w.kb * 128 < w.kv_len;
-  w.nqb = (p.N + 127) / 128;
   w.causal = p.causal != 0;
-  w.qb_begin = w.causal ? w.kb : 0;
-  w.nblk = p.nblk;
+  if (w.causal) {
+    const int lo = w.kb * 128 - w.off;  // first query row that sees this tile's first key
+    w.qb_begin = lo <= 0 ? 0 : lo / 128;
+  } else {
+    w.qb_begin = 0;
+  }
+  w.nbk = p.nbk;
   w.bm = p.block_mask;
 
   if (threadIdx.x == 0) {
@@ -265,8 +299,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_map(&tm_do);
       mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::TILE);
       for (int pn = 0; pn < L::PANELS; ++pn) {
-        tma_load_3d(sbase + L::OFF_K + pn * L::PANEL, &tm_k, bar(L::B_KV), 64 * pn, w.kb * 128, w.bh);
-        tma_load_3d(sbase + L::OFF_V + pn * L::PANEL, &tm_v, bar(L::B_KV), 64 * pn, w.kb * 128, w.bh);
+        tma_load_4d(sbase + L::OFF_K + pn * L::PANEL, &tm_k, bar(L::B_KV), 64 * pn,
+                    w.krow + w.kb * 128, w.h, w.tb);
+        tma_load_4d(sbase + L::OFF_V + pn * L::PANEL, &tm_v, bar(L::B_KV), 64 * pn,
+                    w.krow + w.kb * 128, w.h, w.tb);
       }
       int it = 0;
       for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
@@ -275,12 +311,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (it >= L::STAGES && !mbar_wait(bar(L::B_QEMPTY + s), ph ^ 1u, g)) break;
         mbar_arrive_expect_tx(bar(L::B_QFULL + s), 2 * L::TILE + 1024);
         for (int pn = 0; pn < L::PANELS; ++pn) {
-          tma_load_3d(sbase + L::OFF_Q + s * L::TILE + pn * L::PANEL, &tm_q, bar(L::B_QFULL + s),
-                      64 * pn, qb * 128, w.bh);
-          tma_load_3d(sbase + L::OFF_DO + s * L::TILE + pn * L::PANEL, &tm_do, bar(L::B_QFULL + s),
-                      64 * pn, qb * 128, w.bh);
+          tma_load_4d(sbase + L::OFF_Q + s * L::TILE + pn * L::PANEL, &tm_q, bar(L::B_QFULL + s),
+                      64 * pn, w.qrow + qb * 128, w.h, w.tb);
+          tma_load_4d(sbase + L::OFF_DO + s * L::TILE + pn * L::PANEL, &tm_do, bar(L::B_QFULL + s),
+                      64 * pn, w.qrow + qb * 128, w.h, w.tb);
         }
-        const size_t roff = static_cast<size_t>(w.bh) * p.Npad + static_cast<size_t>(qb) * 128;
+        const long long roff = w.ws0 + static_cast<long long>(qb) * 128;
         bulk_load(sbase + L::OFF_LD + s * 1024, p.ws_lse2 + roff, 512, bar(L::B_QFULL + s));
         bulk_load(sbase + L::OFF_LD + s * 1024 + 512, p.ws_delta + roff, 512, bar(L::B_QFULL + s));
       }
@@ -499,7 +535,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // -LSE log2e and -D of the tile's 128 queries
       const float* nlse = reinterpret_cast<const float*>(smem + L::OFF_LD + s * 1024);
       const float* ndlt = nlse + 128;
-      const bool diag = w.causal && qb == w.kb;
+      // causal: query q of this tile sees this thread's key iff q >= qmin
+      const bool diag = w.causal && (w.kb * 128 + 127 > qb * 128 + w.off);
+      const int qmin = j + (w.kb - qb) * 128 - w.off;
       // only the diagonal tile of a causal mask and padding keys need masking;
       // the choice must be warp-uniform (the TMEM loads and stores in both
       // versions are warp-collective)
@@ -520,7 +558,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if constexpr (MASKED) {
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (!key_live || (diag && qoff + 4 * k4 + e < j)) pv[e] = 0.f;
+            if (!key_live || (diag && qoff + 4 * k4 + e < qmin)) pv[e] = 0.f;
         }
       };
       // keep bit of query qoff + 4 k4 + e (= 8 g + r, g = k4 / 2, r = 4 (k4 % 2) + e)
@@ -694,8 +732,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok && any_work) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_KVDONE), 0, g));
     if (ok) {
       tc_fence_after();
-      const bool row_ok = jg < p.N;
-      const size_t roff = (static_cast<size_t>(w.bh) * p.N + jg) * D;
+      const bool row_ok = jg < w.lk;
+      const long long kr = w.krow + jg;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         const int col = wg * (D / 2) + 32 * c;
@@ -709,9 +747,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) a[k] = bk[k] = 0u;
         }
-        if (row_ok) {
-          uint4* dvp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + roff + col);
-          uint4* dkp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + roff + col);
+        if (row_ok && col < p.d_real) {
+          uint4* dvp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + w.tb * p.sdv.b +
+                                                w.h * p.sdv.h + kr * p.sdv.r + col);
+          uint4* dkp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + w.tb * p.sdk.b +
+                                                w.h * p.sdk.h + kr * p.sdk.r + col);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             uint32_t vv[4], kk4[4];
@@ -748,7 +788,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if constexpr (L::DQ_T) {
         // lane r = feature r; column c = query qb * 128 + c: each warp's
         // reduction covers 32 consecutive floats of one accumulator row
-        float* dst = p.ws_dq + (static_cast<size_t>(w.bh) * p.Npad + qb * 128) * D + r;
+        float* dst = p.ws_dq + (w.ws0 + static_cast<long long>(qb) * 128) * D + r;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           uint32_t a[32];
@@ -784,7 +824,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0) {
           staged = mbar_wait(bar(L::B_STAGED), it & 1u, g);
           if (staged) {
-            const int32_t y = static_cast<int32_t>(static_cast<int64_t>(w.bh) * p.Npad + qb * 128);
+            const int32_t y = static_cast<int32_t>(w.ws0 + static_cast<long long>(qb) * 128);
 #pragma unroll
             for (int b = 0; b < D / 32; ++b) tma_reduce_add_2d(&tm_dq, box(b), 32 * b, y);
             bulk_commit_group();
@@ -808,10 +848,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+// (row blocks of the longest sequence rounded up to 128 rows) x (B * H)
+template <int D>
+dim3 prepost_grid(const BwdParams& p) {
+  const long long rows = (static_cast<long long>(p.rows.nq) + 127) / 128 * 128;
+  return dim3(static_cast<unsigned>(rows / kRowsPerBlock<D>), static_cast<unsigned>(p.B * p.H), 1);
+}
+
 template <int D>
 cudaError_t launch_pre_t(const BwdParams& p, cudaStream_t stream) {
-  const int64_t threads = static_cast<int64_t>(p.B) * p.H * p.Npad * (D / 8);
-  bwd_pre_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+  bwd_pre_kernel<D><<<prepost_grid<D>(p), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -821,10 +867,13 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           cudaStream_t stream) {
   using L = BwdLayout<D>;
   auto kern = bwd_main_kernel<D, DROPOUT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(L::SMEM));
+  static OncePerContext prepared;
+  cudaError_t e = prepared.run([&]() {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(L::SMEM));
+  });
   if (e != cudaSuccess) return e;
-  const long long ctas = static_cast<long long>((p.N + 127) / 128) * p.B * p.H;
+  const long long ctas = static_cast<long long>((p.rows.nk + 127) / 128) * p.B * p.H;
   if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   kern<<<static_cast<unsigned>(ctas), kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError();
@@ -832,8 +881,7 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 
 template <int D>
 cudaError_t launch_post_t(const BwdParams& p, cudaStream_t stream) {
-  const int64_t threads = static_cast<int64_t>(p.B) * p.H * p.N * (D / 8);
-  bwd_post_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+  bwd_post_kernel<D><<<prepost_grid<D>(p), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -40,6 +40,7 @@
 // [KW NS + D s, KW NS + D s + D), NS = NQ KS streams.
 #include <cuda_bf16.h>
 
+#include "devctx.h"
 #include "kernels.h"
 #include "philox.cuh"
 #include "ptx.cuh"
@@ -109,18 +110,23 @@ struct FwdLayout {
   static_assert(O_COL + C::NS * D <= TMEM_COLS, "TMEM budget");
 };
 
-// Which (Q tile, K/V tile) pairs of this CTA take part.
+// Which (Q tile, K/V tile) pairs of this CTA take part.  Rows and keys are
+// counted inside the CTA's sequence; qrow / krow are the tensor rows of the
+// sequence's first query / key and tb its batch coordinate.  Under the causal
+// mask query i sees key j iff j <= i + off, off = (keys) - (queries) of the
+// sequence (bottom-right alignment).
 struct FwdWork {
-  int b, h, bh, q0, qb0, kv_len, n_kb, kb_end, nblk;
+  int b, h, bh, q0, qb0, lq, kv_len, n_kb, kb_end, nbk, off, qrow, krow, tb;
   bool exists1, causal;
   const uint8_t* bm;
 
+  // last row of Q tile t that exists in the sequence
+  __device__ __forceinline__ int last_row(int t) const { return min(q0 + 128 * t + 127, lq - 1); }
   __device__ __forceinline__ bool act(int t, int kb) const {
     if (t == 1 && !exists1) return false;
     if (kb >= n_kb) return false;
-    const int qb = qb0 + t;
-    if (causal && kb > qb) return false;
-    if (bm != nullptr && bm[static_cast<size_t>(qb) * nblk + kb] == 0) return false;
+    if (causal && kb * 128 > last_row(t) + off) return false;
+    if (bm != nullptr && bm[static_cast<size_t>(qb0 + t) * nbk + kb] == 0) return false;
     return true;
   }
   // stream (Q tile t, key part hp of kw keys): also skipped when all its keys
@@ -164,7 +170,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
 
   FwdWork w;
   {
-    const int nqp = (p.N + 128 * NQ - 1) / (128 * NQ);
+    const int nqp = (p.rows.nq + 128 * NQ - 1) / (128 * NQ);
     int tile = 0;
     grid_unit(blockIdx.x, p.B * p.H, nqp, p.group_heads, &w.bh, &tile);
     const int qp = nqp - 1 - tile;  // heaviest causal rows first
@@ -172,14 +178,28 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     w.qb0 = qp * NQ;
     w.b = w.bh / p.H;
     w.h = w.bh % p.H;
-    w.exists1 = NQ == 2 && (w.q0 + 128) < p.N;
-    int kv = p.N;
-    if (p.seqlens != nullptr) kv = max(0, min(p.seqlens[w.b], p.N));
+    const Seq sq = seq_of(p.rows, w.b);
+    // a sequence shorter than the longest has no tile here: leave before any
+    // set-up (the whole CTA takes this branch)
+    if (w.q0 >= sq.lq) return;
+    w.lq = sq.lq;
+    w.qrow = sq.q0;
+    w.krow = sq.k0;
+    w.tb = sq.tb;
+    w.off = sq.lk - sq.lq;
+    w.exists1 = NQ == 2 && (w.q0 + 128) < sq.lq;
+    int kv = sq.lk;
+    if (p.seqlens != nullptr) kv = max(0, min(p.seqlens[w.b], sq.lk));
     w.kv_len = kv;
     w.n_kb = (kv + 127) / 128;
     w.causal = p.causal != 0;
-    w.kb_end = w.causal ? min(w.n_kb, w.qb0 + (w.exists1 ? 2 : 1)) : w.n_kb;
-    w.nblk = p.nblk;
+    if (w.causal) {
+      const int last = w.last_row(w.exists1 ? 1 : 0) + w.off;  // last key any row may see
+      w.kb_end = last < 0 ? 0 : min(w.n_kb, last / 128 + 1);
+    } else {
+      w.kb_end = w.n_kb;
+    }
+    w.nbk = p.nbk;
     w.bm = p.block_mask;
   }
 
@@ -222,8 +242,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         if (t == 1 && !w.exists1) break;
         mbar_arrive_expect_tx(bar(L::B_QFULL + t), L::TILE);
         for (int pn = 0; pn < L::PANELS; ++pn)
-          tma_load_3d(sbase + L::OFF_Q + t * L::TILE + pn * L::PANEL, &tm_q, bar(L::B_QFULL + t),
-                      64 * pn, w.q0 + 128 * t, w.bh);
+          tma_load_4d(sbase + L::OFF_Q + t * L::TILE + pn * L::PANEL, &tm_q, bar(L::B_QFULL + t),
+                      64 * pn, w.qrow + w.q0 + 128 * t, w.h, w.tb);
       }
       int it = 0;
       for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1), ++it) {
@@ -234,10 +254,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         const uint32_t vdst = kdst + L::TILE;
         mbar_arrive_expect_tx(bar(L::B_KFULL + s), L::TILE);
         for (int pn = 0; pn < L::PANELS; ++pn)
-          tma_load_3d(kdst + pn * L::PANEL, &tm_k, bar(L::B_KFULL + s), 64 * pn, kb * 128, w.bh);
+          tma_load_4d(kdst + pn * L::PANEL, &tm_k, bar(L::B_KFULL + s), 64 * pn, w.krow + kb * 128,
+                      w.h, w.tb);
         mbar_arrive_expect_tx(bar(L::B_VFULL + s), L::TILE);
         for (int pn = 0; pn < L::PANELS; ++pn)
-          tma_load_3d(vdst + pn * L::PANEL, &tm_v, bar(L::B_VFULL + s), 64 * pn, kb * 128, w.bh);
+          tma_load_4d(vdst + pn * L::PANEL, &tm_v, bar(L::B_VFULL + s), 64 * pn, w.krow + kb * 128,
+                      w.h, w.tb);
       }
       if (*abort_flag) {  // let the copies already issued land before the CTA exits
         for (int j = max(0, it - L::STAGES); j < it; ++j) {
@@ -391,7 +413,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         }
 
         const int j0 = kb * 128 + KW * hp;  // first key of this block
-        const bool need_mask = (w.causal && kb == w.qb0 + t) || (j0 + KW > w.kv_len);
+        // masking is needed where a key of this block lies past the first
+        // row's causal limit, or past the key length
+        const bool need_mask =
+            (w.causal && j0 + KW - 1 > w.q0 + 128 * t + w.off) || (j0 + KW > w.kv_len);
         // row maximum with independent partial maxima (short dependency chains;
         // as many as the register budget allows), two scores per max instruction
         constexpr int kParts = C::MAX_PARTS;
@@ -399,7 +424,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
 #pragma unroll
         for (int u = 0; u < kParts; ++u) mxp[u] = -INFINITY;
         if (need_mask) {
-          const int lim = w.causal ? min(w.kv_len - j0, i - j0 + 1) : (w.kv_len - j0);
+          const int lim = w.causal ? min(w.kv_len - j0, i + w.off - j0 + 1) : (w.kv_len - j0);
 #pragma unroll
           for (int j = 0; j < KW; ++j)
             if (j >= lim) sr[j] = __float_as_uint(-INFINITY);
@@ -499,9 +524,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       // ------------------------------------------------------------ epilogue
       if (ok && cnt > 0)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_ODONE + s), (cnt - 1) & 1u, g));
-      const bool row_ok = i < p.N;
-      __nv_bfloat16* orow =
-          reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(w.bh) * p.N + i) * D;
+      const bool row_ok = i < w.lq;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + w.tb * p.so.b +
+                            w.h * p.so.h + static_cast<long long>(w.qrow + i) * p.so.r;
+      float* lse_out = p.lse + w.tb * p.lse_sb + w.h * p.lse_sh + w.qrow + i;
       if constexpr (KS == 1) {
         if (ok) {
           tc_fence_after();
@@ -523,15 +549,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
                                      make_float2(inv, inv));
               ob[k] = pack_bf16(o2.x, o2.y);
             }
-            if (row_ok) {
+            if (row_ok && 32 * c < p.d_real) {
               uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 dst[k] = make_uint4(ob[4 * k], ob[4 * k + 1], ob[4 * k + 2], ob[4 * k + 3]);
             }
           }
-          if (row_ok)
-            p.lse[static_cast<size_t>(w.bh) * p.N + i] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+          if (row_ok) *lse_out = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
         }
       } else {
         // Merge the two streams of this Q tile.  A stream that processed no
@@ -578,15 +603,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
               const float2 o2 = fma2(x1, g1, mul2(x0, g0));
               ob[k] = pack_bf16(o2.x, o2.y);
             }
-            if (row_ok) {
+            if (row_ok && (D / 2) * hp + 32 * c < p.d_real) {
               uint4* dst = reinterpret_cast<uint4*>(orow + (D / 2) * hp + 32 * c);
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 dst[k] = make_uint4(ob[4 * k], ob[4 * k + 1], ob[4 * k + 2], ob[4 * k + 3]);
             }
           }
-          if (row_ok && hp == 0)
-            p.lse[static_cast<size_t>(w.bh) * p.N + i] = (lt > 0.f) ? (mref + log2f(lt)) * kLn2 : -INFINITY;
+          if (row_ok && hp == 0) *lse_out = (lt > 0.f) ? (mref + log2f(lt)) * kLn2 : -INFINITY;
         }
       }
     }
@@ -608,19 +632,20 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   using C = FwdCfg<D>;
   auto kern = fwd_kernel<D, DROPOUT>;
   // The setmaxnreg split is sized for exactly LAUNCH_REGS registers per thread
-  // at launch; with any other count an increase could wait forever.
-  static int regs_checked = 0;
-  if (!regs_checked) {
+  // at launch; with any other count an increase could wait forever.  Checked,
+  // with the shared-memory attribute set, once per device and context.
+  static OncePerContext prepared;
+  cudaError_t e = prepared.run([&]() -> cudaError_t {
     cudaFuncAttributes attr{};
-    cudaError_t e = cudaFuncGetAttributes(&attr, kern);
-    if (e != cudaSuccess) return e;
+    cudaError_t r = cudaFuncGetAttributes(&attr, kern);
+    if (r != cudaSuccess) return r;
     if (attr.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-    regs_checked = 1;
-  }
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(L::SMEM));
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(L::SMEM));
+  });
   if (e != cudaSuccess) return e;
-  const long long ctas = static_cast<long long>((p.N + 128 * C::NQ - 1) / (128 * C::NQ)) * p.B * p.H;
+  const long long ctas =
+      static_cast<long long>((p.rows.nq + 128 * C::NQ - 1) / (128 * C::NQ)) * p.B * p.H;
   if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   kern<<<static_cast<unsigned>(ctas), C::THREADS, L::SMEM, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();

@@ -6,18 +6,24 @@
 // allocator or a memory-pool callback that must not re-enter the allocator,
 // plugin hosts that forbid device allocations after start-up, or a framework
 // that has pre-reserved all device memory).  For them this file keeps the
-// workspace in a fixed, file-scope device array that the CUDA runtime creates
-// when it loads this library on a device, and forwards to the normal
+// workspace in a fixed, file-scope device array and forwards to the normal
 // backward with that array as the workspace.
 //
 // Limits and rules:
 //  - the array holds kNoAllocScratchBytes (64 MiB) on every device that loads
-//    the library, until the process exits; requests whose workspace
+//    this file's module, until the process exits; requests whose workspace
 //    (fa_bwd_workspace_size) exceeds it are rejected with FA_ERR_WORKSPACE
 //    before anything is launched;
-//  - the first call on a device looks up the array's device address with
-//    cudaGetSymbolAddress (with that device current) and caches it; make that
-//    first call before any stream capture;
+//  - the array comes into existence when the CUDA runtime loads this file's
+//    module on a device.  Under lazy module loading (the default since CUDA
+//    12.2) that happens inside the first fa_bwd_noalloc call on the device,
+//    when it looks up the array's device address with cudaGetSymbolAddress:
+//    that first call is where the 64 MiB is reserved (and where it fails with
+//    FA_ERR_CUDA if the device has no room).  Make it at start-up, outside any
+//    allocator callback and before any stream capture, or run the process
+//    with CUDA_MODULE_LOADING=EAGER so that loading the library reserves it;
+//  - the address is cached per device and per context; after a context
+//    teardown (cudaDeviceReset) the next call looks it up again;
 //  - every call on a device shares the one array, and it keeps whatever the
 //    last call left there; the backward's first launch rewrites every part
 //    that must start fresh (it zeroes the dQ accumulators and overwrites the
@@ -26,8 +32,8 @@
 //    ordering between them) race on the array and give wrong results:
 //    serialise them, for example by issuing them on one stream.
 #include <cstdint>
-#include <mutex>
 
+#include "devctx.h"
 #include "fa.h"
 #include "kernels.h"
 
@@ -37,24 +43,18 @@ constexpr size_t kNoAllocScratchBytes = size_t{64} << 20;
 
 static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
-std::mutex g_scratch_mutex;
+fa::SymbolAddressCache g_scratch_cache;
 
 // Device address of g_bwd_scratch on the current device (nullptr on error).
 // In host code the array's name is only a host-side handle, never a device
-// address, so the address must come from the runtime.
+// address, so the address must come from the runtime, with the device current.
 void* scratch_address() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  return g_scratch_cache.get([]() -> void* {
     void* ptr = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&ptr, g_bwd_scratch);
-    if (e != cudaSuccess || ptr == nullptr) return nullptr;
-    g_scratch_ptr[dev] = ptr;
-  }
-  return g_scratch_ptr[dev];
+    if (e != cudaSuccess) return nullptr;
+    return ptr;
+  });
 }
 
 }  // namespace

@@ -43,7 +43,10 @@ def test_workspace_size_formula(lib):
     # per (b,h): Npad rows x (lse2 + delta + d accumulators) fp32, rounded to 256 B
     assert so.fa_bwd_workspace_size(2, 3, 300, 64) == 2 * 3 * 384 * (8 + 256)
     assert so.fa_bwd_workspace_size(1, 1, 128, 128) == 128 * (8 + 512)
-    assert so.fa_bwd_workspace_size(1, 1, 128, 96) == 0
+    # d = 32 and 96 run the 64- and 128-wide kernels: accumulators of that width
+    assert so.fa_bwd_workspace_size(1, 1, 128, 96) == 128 * (8 + 512)
+    assert so.fa_bwd_workspace_size(1, 1, 128, 32) == 128 * (8 + 256)
+    assert so.fa_bwd_workspace_size(1, 1, 128, 80) == 0
     assert so.fa_bwd_workspace_size(0, 1, 128, 64) == 0
 
 
@@ -52,7 +55,7 @@ A16 = 1 << 20  # a fake, 16-byte aligned address: validation fails before use
 
 @pytest.mark.parametrize("args,code", [
     (dict(q=0), 1), (dict(k=A16 + 8), 1), (dict(B=0), 1), (dict(N=0), 1),
-    (dict(d=96), 2), (dict(scale=0.0), 1), (dict(scale=float("inf")), 1),
+    (dict(d=80), 2), (dict(d=256), 2), (dict(scale=0.0), 1), (dict(scale=float("inf")), 1),
     (dict(p=1.0), 1), (dict(p=-0.1), 1), (dict(p=float("nan")), 1),
     (dict(B=300, H=300), 2), (dict(lse=A16 + 2), 1),
     (dict(N=(1 << 23) + 1), 2),                       # N beyond 2^23
@@ -86,3 +89,67 @@ def test_product_path_has_no_cpu_fallback(lib):
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         lib.forward(q, q, q)
+
+
+def _desc(lib, **kw):
+    a = lib.AttentionDesc()
+    a.batch, a.heads, a.head_dim, a.seqlen_q, a.seqlen_k = 2, 3, 64, 256, 384
+    a.softmax_scale = 0.125
+    st = lib.Strides(3 * 256 * 64, 256 * 64, 64)
+    sk = lib.Strides(3 * 384 * 64, 384 * 64, 64)
+    for name in ("q", "o", "dout", "dq"):
+        setattr(a, name, st)
+    for name in ("k", "v", "dk", "dv"):
+        setattr(a, name, sk)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("change,code", [
+    (dict(), None),                                        # valid: workspace size > 0
+    (dict(head_dim=80), 2), (dict(head_dim=256), 2),
+    (dict(batch=0), 1), (dict(seqlen_k=0), 1), (dict(dropout_p=1.0), 1),
+    (dict(cu_seqlens_q=A16), 1),                           # packed needs both offsets
+    (dict(cu_seqlens_q=A16, cu_seqlens_k=A16), 1),          # ... and total_q, total_k >= 1
+    (dict(cu_seqlens_q=A16 + 2, cu_seqlens_k=A16, total_q=5, total_k=5), 1),
+    (dict(q=(3 * 256 * 64, 256 * 64, 60)), 1),              # row stride not a multiple of 8
+    (dict(k=(3 * 384 * 64, 0, 64)), 1),                     # heads sharing memory
+    (dict(o=(0, 256 * 64, 64)), 1),                         # batch entries sharing memory
+    (dict(seqlen_q=(1 << 23) + 1), 2),
+])
+def test_general_entry_points_validate_before_launching(lib, change, code):
+    so = lib.library()
+    kw = {k: (lib.Strides(*v) if isinstance(v, tuple) else v) for k, v in change.items()}
+    a = _desc(lib, **kw)
+    ws = so.fa_bwd_ex_workspace_size(ctypes.byref(a))
+    if code is None:
+        # padded layout: B * H * ceil(N_q / 128) * 128 rows of 8 + 4 * 64 bytes
+        # (a valid description is never launched here: the addresses are fake)
+        assert ws == 2 * 3 * 256 * (8 + 256)
+        return
+    assert ws == 0
+    assert so.fa_fwd_ex(ctypes.byref(a), A16, A16, A16, A16, A16, None) == code
+    assert so.fa_bwd_ex(ctypes.byref(a), A16, A16, A16, A16, A16, A16, A16, A16, A16, A16,
+                        1 << 30, None) == code
+
+
+def test_general_workspace_size_of_packed_layout(lib):
+    """Packed: H * (ceil(total_q / 128) * 128 + 256 B) rows, each 8 + 4 D bytes."""
+    so = lib.library()
+    a = _desc(lib, cu_seqlens_q=A16, cu_seqlens_k=A16, total_q=1000, total_k=900, head_dim=96)
+    for name in ("q", "k", "v", "o", "dout", "dq", "dk", "dv"):
+        setattr(a, name, lib.Strides(0, 96, 3 * 96))
+    rows = 3 * (1024 + 256 * 2)
+    assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == (rows * (8 + 512) + 255) // 256 * 256
+    assert so.fa_fwd_ex(None, A16, A16, A16, A16, A16, None) == 1
+
+
+def test_qkv_projection_rejects_bad_shapes(lib):
+    so = lib.library()
+    a = A16
+    assert so.fa_qkv_projection(a, a, None, a, a, a, 1, 128, 1, 64, 64, None) == 2  # H d = 64
+    assert so.fa_qkv_projection(a, a, None, a, a, a, 1, 128, 2, 96, 64, None) == 2  # d = 96
+    assert so.fa_qkv_projection(a, a, None, a, a, a, 1, 128, 2, 64, 60, None) == 1  # d_model % 8
+    assert so.fa_qkv_projection(a + 8, a, None, a, a, a, 1, 128, 2, 64, 64, None) == 1
+    assert so.fa_qkv_projection(a, a, a + 2, a, a, a, 1, 128, 2, 64, 64, None) == 1  # bias align

@@ -61,12 +61,45 @@ CASES = [
 
 
 @pytest.mark.parametrize("B,H,N,d,causal,lens,density,p", CASES)
-def test_backward_matches_oracle(lib, B, H, N, d, causal, lens, density, p):
+def test_backward_matches_oracle(lib, parity_record, B, H, N, d, causal, lens, density, p):
     got, ref = run_bwd(lib, B, H, N, d, causal, lens, density, p)
+    errs = {}
     for name, a, r in zip(("dq", "dk", "dv"), got, ref):
         assert np.isfinite(a).all(), name
-        e = rel_l2(a, r)
+        errs[name] = e = rel_l2(a, r)
         assert e <= REL_L2, (name, e)
+    parity_record(**{f"{k}_rel_l2": float(v) for k, v in errs.items()})
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("p", [0.0, 0.1])
+def test_backward_block_mask_without_diagonal(lib, parity_record, d, causal, p):
+    """Block mask with holes in its diagonal, an all-zero block row (query
+    tile 1: rows without keys, so dQ = 0 there) and an all-zero block column
+    (key tile 2: reached by no query tile, so dK = dV = 0 there)."""
+    import torch
+    from test_gpu_fwd import block_mask_with_holes
+    B, H, N = 2, 2, 600
+    q, k, v, do = make_qkvdo(B, H, N, d, 33)
+    bm = block_mask_with_holes(N, 32)
+    scale = d ** -0.5
+    kw = dict(scale=scale, causal=causal, dropout_p=p, seed=6, block_mask=bm)
+    gq, gk, gv, gdo = (x.cuda() for x in (q, k, v, do))
+    o, lse = lib.forward(gq, gk, gv, **kw)
+    dq, dk, dv = lib.backward(gq, gk, gv, o, lse, gdo, **kw)
+    torch.cuda.synchronize()
+    assert lib.last_device_status() == 0
+    ref = attention_backward(f64(q), f64(k), f64(v), f64(do), scale, causal, None, p, 6, bm)
+    got = (f64(dq), f64(dk), f64(dv))
+    errs = {}
+    for name, a, r in zip(("dq", "dk", "dv"), got, ref):
+        assert np.isfinite(a).all(), name
+        errs[name] = e = rel_l2(a, r)
+        assert e <= REL_L2, (name, e)
+    parity_record(**{f"{k}_rel_l2": float(v) for k, v in errs.items()})
+    assert (got[0][:, :, 128:256] == 0).all()                          # empty query rows
+    assert (got[1][:, :, 256:384] == 0).all() and (got[2][:, :, 256:384] == 0).all()
 
 
 def test_backward_is_repeatable_for_dk_dv(lib):

@@ -41,14 +41,26 @@ def run_case(fa, B, H, N, d, causal=False, lens=None, density=None, p=0.0, seed=
     return f64(o), lse.cpu().numpy().astype(np.float64), ro, rl
 
 
-def compare(o, lse, ro, rl):
+def compare(o, lse, ro, rl, record=None):
+    """Checks O and LSE against the oracle.  The strict the benchmark spec bound
+    (max-abs 1e-2) is asserted wherever bf16 storage can meet it (|O_ref| < 2,
+    half an ulp <= 2^-8 |O| < 0.0079); everywhere the bound is
+    1e-2 + 2^-8 |O_ref|.  The strict max-abs error over all elements is
+    returned (and recorded) so the slack actually used is visible."""
     assert np.isfinite(o).all()
     empty = np.isneginf(rl)
     assert np.array_equal(np.isneginf(lse), empty), "rows without keys must have LSE = -inf"
     assert (o[empty] == 0).all()
-    err_o = np.abs(o - ro).max()
-    excess = (np.abs(o - ro) - (O_TOL + 2.0 ** -8 * np.abs(ro))).max()
+    diff = np.abs(o - ro)
+    err_o = diff.max()
+    small = np.abs(ro) < 2.0
+    err_small = diff[small].max() if small.any() else 0.0
+    excess = (diff - (O_TOL + 2.0 ** -8 * np.abs(ro))).max()
     err_l = np.abs(np.where(empty, 0, lse - rl)).max()
+    if record is not None:
+        record(o_max_abs=float(err_o), o_max_abs_where_abs_ref_lt_2=float(err_small),
+               o_max_abs_ref=float(np.abs(ro).max()), lse_max_abs=float(err_l))
+    assert err_small <= O_TOL, ("strict O bound", err_small)
     assert excess <= 0, (err_o, excess)
     assert err_l <= LSE_TOL, err_l
     return err_o, err_l
@@ -77,9 +89,43 @@ CASES = [
 
 
 @pytest.mark.parametrize("B,H,N,d,causal,lens,density,p", CASES)
-def test_forward_matches_oracle(lib, B, H, N, d, causal, lens, density, p):
+def test_forward_matches_oracle(lib, parity_record, B, H, N, d, causal, lens, density, p):
     o, lse, ro, rl = run_case(lib, B, H, N, d, causal, lens, density, p)
-    compare(o, lse, ro, rl)
+    compare(o, lse, ro, rl, parity_record)
+
+
+def block_mask_with_holes(N, seed):
+    """A block mask whose diagonal is not all set: query tile 1 keeps no key
+    block (its rows have no valid key), key tile 2 is kept by no query tile,
+    and the diagonal blocks (0, 0) and (3, 3) are removed.  Legal input; the
+    workload generator never makes it (it always keeps the diagonal)."""
+    bm = make_block_mask(N, 0.5, seed)
+    bm[1, :] = 0
+    bm[:, 2] = 0
+    bm[0, 0] = 0
+    bm[3, 3] = 0
+    bm[4, 4] = 1
+    return bm
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("p", [0.0, 0.1])
+def test_forward_block_mask_without_diagonal(lib, parity_record, d, causal, p):
+    import torch
+    B, H, N = 2, 2, 600
+    q, k, v, _ = make_qkvdo(B, H, N, d, 31)
+    bm = block_mask_with_holes(N, 32)
+    scale = d ** -0.5
+    o, lse = lib.forward(q.cuda(), k.cuda(), v.cuda(), scale=scale, causal=causal, dropout_p=p,
+                         seed=5, block_mask=bm)
+    torch.cuda.synchronize()
+    assert lib.last_device_status() == 0
+    ro, rl = attention_forward(f64(q), f64(k), f64(v), scale, causal, None, p, 5, bm)
+    o, lse = f64(o), lse.cpu().numpy().astype(np.float64)
+    assert np.isneginf(rl[:, :, 128:256]).all()  # query tile 1 is empty
+    compare(o, lse, ro, rl, parity_record)
+    assert (o[:, :, 128:256] == 0).all()
 
 
 def test_forward_long_rows_many_tiles(lib):
