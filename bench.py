@@ -66,6 +66,11 @@ KERNEL_SOURCES = {
     "bwd_main_kernel": ["fa_bwd.cu", "ptx.cuh", "philox.cuh", "kernels.h"],
 }
 SLAB = 256  # rows of one CPU-oracle sample
+PROJ_SHAPES = {
+    # fused QKV projection measurements, name: (B, N, H, d, d_model)
+    "qkv_proj_gpt2": (8, 1024, 12, 64, 768),
+    "qkv_proj_long128": (1, 16384, 16, 128, 2048),
+}
 
 
 def parse_args(argv=None):
@@ -74,9 +79,11 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all"] + sorted(WORKLOADS), default="all",
+    ap.add_argument("--workload", choices=["all"] + sorted(WORKLOADS) + sorted(PROJ_SHAPES),
+                    default="all",
                     help="'all' (default): headline plus every workload in per_config; a name: "
-                         "that workload alone as the headline (profiling)")
+                         "that workload alone as the headline (profiling); a qkv_proj_* name: "
+                         "that fused-projection measurement alone")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch size (single-workload profiling only)")
     ap.add_argument("--seqlen", type=int, default=None,
@@ -96,8 +103,9 @@ def parse_args(argv=None):
                     help="instead of the bench line: fused vs unfused time and peak memory "
                          "for N = 1K..32K (B=1 H=4 d=128 causal)")
     args = ap.parse_args(argv)
-    if args.workload == "all" and (args.batch or args.seqlen or args.dropout is not None):
-        ap.error("--batch/--seqlen/--dropout need a single --workload")
+    if (args.workload == "all" or args.workload in PROJ_SHAPES) and (
+            args.batch or args.seqlen or args.dropout is not None):
+        ap.error("--batch/--seqlen/--dropout need a single attention --workload")
     return args
 
 
@@ -379,8 +387,9 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    name = HEADLINE if args.workload == "all" else args.workload
-    w = selected_workload(name, None if args.workload == "all" else args)
+    single = args.workload in WORKLOADS
+    name = args.workload if single else HEADLINE
+    w = selected_workload(name, args if single else None)
     inp = make_inputs(w, B=1)
     per_head = math.ceil(w.N / SLAB)
     units = [(0, h, s * SLAB) for h in range(w.H) for s in range(per_head)]
@@ -534,13 +543,6 @@ def measure_packed(fa, w, args, rank, dev, flush, stream, world, local, peak):
     del case
     torch.cuda.empty_cache()
     return entry
-
-
-PROJ_SHAPES = {
-    # name: (B, N, H, d, d_model)
-    "qkv_proj_gpt2": (8, 1024, 12, 64, 768),
-    "qkv_proj_long128": (1, 16384, 16, 128, 2048),
-}
 
 
 def measure_projection(fa, name, args, rank, dev, flush, stream, world, local, peak):
@@ -698,6 +700,11 @@ def run_ours(args):
 
     if args.unfused_sweep:
         return run_unfused_sweep(args, fa, dev, flush, stream, world, rank)
+    if args.workload in PROJ_SHAPES:
+        r = measure_projection(fa, args.workload, args, rank, dev, flush, stream, world, local, peak)
+        if rank == 0:
+            print(json.dumps({"workload": args.workload, **r}), flush=True)
+        return 0
 
     single = args.workload != "all"
     head_name = args.workload if single else HEADLINE
