@@ -8,15 +8,18 @@
 // is the pass that would otherwise reorder its [T, 3, H, d] output into three
 // [B, H, N, d] tensors (one read and one write of 6 T H d bytes).
 //
-// One CTA computes a 128-token x 128-column tile of Y (128 columns lie inside
-// one of Q / K / V and cover 128 / d heads, since H d is a multiple of 128):
-//   warp 0      TMA producer: 64-wide K chunks of X and W (128-byte swizzle)
-//               into a ring of kStages stages
-//   warp 1      TMEM allocator (128 columns) and single-thread MMA issuer:
-//               tcgen05.mma kind::f16, both operands K-major, fp32 in TMEM
+// One CTA computes a 128-token x 256-column tile of Y (each 32-column chunk
+// lies inside one head of one of Q / K / V, d being 64 or 128):
+//   warp 0      TMA producer: 64-wide K chunks of X (128 rows) and W (256
+//               rows), 128-byte swizzle, into a ring of kStages stages
+//   warp 1      TMEM allocator (256 columns) and single-thread MMA issuer:
+//               tcgen05.mma kind::f16, M = 128, N = 256, both operands
+//               K-major, fp32 in TMEM
 //   warps 4-7   epilogue: thread = token row; TMEM -> + bias -> bf16 ->
 //               Q / K / V rows at their head-major addresses
 // Two CTAs fit on an SM, so one CTA's epilogue overlaps the other's main loop.
+// The 256-wide tile halves the X bytes every output element costs against a
+// 128-wide one (the operands stream from L2 once per tile).
 // Every wait is bounded (see ptx.cuh).
 #include <cuda_bf16.h>
 
@@ -30,11 +33,13 @@ namespace fa {
 namespace {
 
 constexpr int kProjThreads = 256;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
+constexpr int kBN = 256;                  // output columns per CTA
 constexpr uint32_t kPanel = 128u * 128u;  // 128 rows x 64 bf16, one 128-byte-swizzled panel
+constexpr uint32_t kPanelW = kBN * 128u;  // kBN rows x 64 bf16
 constexpr uint32_t kOffX = 0;
 constexpr uint32_t kOffW = kStages * kPanel;
-constexpr uint32_t kOffBar = 2 * kStages * kPanel;
+constexpr uint32_t kOffBar = kStages * (kPanel + kPanelW);
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarAcc = 2 * kStages, kBarDrain = 2 * kStages + 1;
 constexpr int kNumBars = 2 * kStages + 2;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
@@ -46,7 +51,7 @@ struct ProjParams {
   __nv_bfloat16* ok;
   __nv_bfloat16* ov;
   const __nv_bfloat16* bias;    // bf16 [3 H d] or null
-  int T, N, H, d, kchunks;
+  int T, N, H, d, ncols, kchunks;
   int* status;
   uint64_t timeout_ns;
 };
@@ -66,7 +71,7 @@ __global__ void __launch_bounds__(kProjThreads, 2)
   const WaitGuard g{abort_flag, p.status, p.timeout_ns};
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * 128;  // first output column
+  const int n0 = blockIdx.x * kBN;  // first output column
   const int t0 = blockIdx.y * 128;  // first token
 
   if (threadIdx.x == 0) {
@@ -80,7 +85,7 @@ __global__ void __launch_bounds__(kProjThreads, 2)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_alloc(smem_u32(tmem_slot), kBN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -98,9 +103,9 @@ __global__ void __launch_bounds__(kProjThreads, 2)
         const int s = kc % kStages;
         const uint32_t ph = (kc / kStages) & 1u;
         if (kc >= kStages && !mbar_wait(bar(kBarEmpty + s), ph ^ 1u, g)) break;
-        mbar_arrive_expect_tx(bar(kBarFull + s), 2 * kPanel);
+        mbar_arrive_expect_tx(bar(kBarFull + s), kPanel + kPanelW);
         tma_load_2d(sbase + kOffX + s * kPanel, &tm_x, bar(kBarFull + s), 64 * kc, t0);
-        tma_load_2d(sbase + kOffW + s * kPanel, &tm_w, bar(kBarFull + s), 64 * kc, n0);
+        tma_load_2d(sbase + kOffW + s * kPanelW, &tm_w, bar(kBarFull + s), 64 * kc, n0);
       }
       if (*abort_flag) {  // let the copies already issued land before the CTA exits
         for (int j = max(0, kc - kStages); j < kc; ++j)
@@ -110,12 +115,12 @@ __global__ void __launch_bounds__(kProjThreads, 2)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
-      constexpr uint32_t kId = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t kId = idesc_bf16(128, kBN, false, false);
       for (int kc = 0; kc < p.kchunks; ++kc) {
         const int s = kc % kStages;
         if (!mbar_wait(bar(kBarFull + s), (kc / kStages) & 1u, g)) break;
         tc_fence_after();
-        const uint32_t xa = sbase + kOffX + s * kPanel, wa = sbase + kOffW + s * kPanel;
+        const uint32_t xa = sbase + kOffX + s * kPanel, wa = sbase + kOffW + s * kPanelW;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(tmem, sdesc_sw128(xa + kk * 32, 16, 1024), sdesc_sw128(wa + kk * 32, 16, 1024),
@@ -139,13 +144,14 @@ __global__ void __launch_bounds__(kProjThreads, 2)
       const int hd = p.H * p.d;
       const int b = t / p.N, n = t % p.N;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kBN / 32; ++c) {
         uint32_t acc[32];
         tmem_ld32<0>(lane_addr + 32 * c, acc);
         tmem_wait_ld32<0>(acc);
         const int col = n0 + 32 * c;
+        const bool col_ok = col < p.ncols;  // the last tile may reach past 3 H d
         float bv[32];
-        if (p.bias != nullptr) {
+        if (p.bias != nullptr && col_ok) {
           const uint4* bsrc = reinterpret_cast<const uint4*>(p.bias + col);
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
@@ -162,7 +168,7 @@ __global__ void __launch_bounds__(kProjThreads, 2)
 #pragma unroll
           for (int j = 0; j < 32; ++j) bv[j] = 0.f;
         }
-        if (t < p.T) {
+        if (t < p.T && col_ok) {
           const int which = col / hd;
           const int within = col - which * hd;
           const int h = within / p.d, e0 = within - h * p.d;
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(kProjThreads, 2)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, kBN);
   }
 }
 
@@ -212,6 +218,7 @@ cudaError_t launch_qkv_projection(const void* x, const void* w, const void* bias
   TmapDesc wd = a;
   wd.base = w;
   wd.dims[1] = static_cast<uint64_t>(3) * H * d;
+  wd.box[1] = kBN;  // rows past 3 H d read as zeros
   if (!tmap_cache().encode(a, &tx) || !tmap_cache().encode(wd, &tw)) return cudaErrorInvalidValue;
   ProjParams p;
   p.oq = static_cast<__nv_bfloat16*>(q);
@@ -222,6 +229,7 @@ cudaError_t launch_qkv_projection(const void* x, const void* w, const void* bias
   p.N = N;
   p.H = H;
   p.d = d;
+  p.ncols = 3 * H * d;
   p.kchunks = (d_model + 63) / 64;
   p.status = status;
   p.timeout_ns = timeout_ns;
@@ -231,7 +239,8 @@ cudaError_t launch_qkv_projection(const void* x, const void* w, const void* bias
                                 static_cast<int>(kProjSmem));
   });
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(3 * H * d / 128), static_cast<unsigned>((T + 127) / 128));
+  const dim3 grid(static_cast<unsigned>((3 * H * d + kBN - 1) / kBN),
+                  static_cast<unsigned>((T + 127) / 128));
   qkv_proj_kernel<<<grid, kProjThreads, kProjSmem, stream>>>(tx, tw, p);
   return cudaGetLastError();
 }
