@@ -51,7 +51,10 @@
  *  - stream: a cudaStream_t (NULL = the legacy default stream).  Every call is
  *    asynchronous on that stream; nothing is synchronised and nothing printed.
  *  - Ownership: the caller allocates and frees every buffer.  The library
- *    keeps no device memory of its own apart from a status word per device.
+ *    keeps no device memory of its own apart from a status word per device
+ *    and the fixed 64 MiB array of fa_bwd_noalloc (present on a device once
+ *    that module is loaded there: at its first call under CUDA's default lazy
+ *    loading, at library load with CUDA_MODULE_LOADING=EAGER).
  *  - Errors: arguments are validated before any launch; a failed check
  *    returns FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED and launches nothing.
  *    A failed launch returns FA_ERR_CUDA.  A kernel whose internal pipeline
