@@ -98,6 +98,15 @@ struct BwdLayout {
   // coalesced reductions: there a 64 KB stage of the two-deep Q / dO ring
   // held until the reduce has read it costs more than it saves.
   static constexpr bool TMA_REDUCE = !DQ_T;
+  // d = 128: setmaxnreg moves registers from warpgroup 0 (producer, MMA
+  // issuer) to the dQ warpgroup, which reads the whole transposed dQ tile
+  // (128 values per thread) out of TMEM before it starts the reductions, so
+  // that the TMEM columns it shares with the next tile's dP^T are free early.
+  // 128 * (REGS_CTL + 2 * 128 + REGS_DQ) must equal 512 threads x 128.
+  static constexpr bool SPLIT_REGS = DQ_T;
+  static constexpr uint32_t REGS_CTL = 72;
+  static constexpr uint32_t REGS_DQ = 184;
+  static_assert(REGS_CTL + 2 * 128 + REGS_DQ == 4 * 128, "register split");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(COL_DK + D <= 512, "TMEM budget");
 };
@@ -290,6 +299,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int q_first = w.next(w.qb_begin);
   const bool any_work = q_first < w.nqb;
 
+  if (warp < 4) {
+  if constexpr (L::SPLIT_REGS) setmaxnreg_dec<L::REGS_CTL>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0 && any_work) {
@@ -486,6 +497,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit(bar(L::B_KVDONE));
       mbar_wait_drain(bar(L::B_KVDONE), 0, 1000000000ull);
     }
+  }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------ P / dS warpgroups
     const int wg = (warp - 4) >> 2;
@@ -770,6 +782,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp >= 12) {
     // ------------------------------------------------------- dQ reduction
+    if constexpr (L::SPLIT_REGS) setmaxnreg_inc<L::REGS_DQ>();
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // query row within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
@@ -787,16 +800,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       };
       if constexpr (L::DQ_T) {
         // lane r = feature r; column c = query qb * 128 + c: each warp's
-        // reduction covers 32 consecutive floats of one accumulator row
+        // reduction covers 32 consecutive floats of one accumulator row.
+        // The whole tile comes out of TMEM first and its columns go back to
+        // the MMA warp (for the next tile's dP^T) before the reductions.
         float* dst = p.ws_dq + (w.ws0 + static_cast<long long>(qb) * 128) * D + r;
+        uint32_t a[128];
+        tmem_ld32<0>(lane_addr + L::COL_DQ + 0, a);
+        tmem_ld32<32>(lane_addr + L::COL_DQ + 32, a);
+        tmem_ld32<64>(lane_addr + L::COL_DQ + 64, a);
+        tmem_ld32<96>(lane_addr + L::COL_DQ + 96, a);
+        tmem_wait_ld32<0>(a);
+        tmem_wait_ld32<32>(a);
+        tmem_wait_ld32<64>(a);
+        tmem_wait_ld32<96>(a);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_DQEMPTY));  // the dQ columns of TMEM are free again
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t a[32];
-          tmem_ld32<0>(lane_addr + L::COL_DQ + 32 * c4, a);
-          tmem_wait_ld32<0>(a);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) red_add_f32(dst + (32 * c4 + k) * D, __uint_as_float(a[k]));
-        }
+        for (int k = 0; k < 128; ++k) red_add_f32(dst + k * D, __uint_as_float(a[k]));
       } else {
         // lane r = query r; columns 32 b .. 32 b + 31 = box b
 #pragma unroll
@@ -810,12 +831,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             st_shared_v4(row + ((k ^ (r & 7)) << 4), a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
         }
       }
-      tc_fence_before();
-      if constexpr (L::TMA_REDUCE) fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(L::B_DQEMPTY));  // the dQ columns of TMEM are free again
-        if constexpr (L::TMA_REDUCE) mbar_arrive(bar(L::B_STAGED));
+      if constexpr (!L::DQ_T) {
+        tc_fence_before();
+        if constexpr (L::TMA_REDUCE) fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(L::B_DQEMPTY));  // the dQ columns of TMEM are free again
+          if constexpr (L::TMA_REDUCE) mbar_arrive(bar(L::B_STAGED));
+        }
       }
       if (L::TMA_REDUCE && warp == 12) {
         // one thread reduces the staged tile into the accumulators, then hands
@@ -867,8 +890,16 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           cudaStream_t stream) {
   using L = BwdLayout<D>;
   auto kern = bwd_main_kernel<D, DROPOUT>;
+  // The setmaxnreg split (d = 128) is sized for exactly 128 registers per
+  // thread at launch; with any other count an increase could wait forever.
   static OncePerContext prepared;
-  cudaError_t e = prepared.run([&]() {
+  cudaError_t e = prepared.run([&]() -> cudaError_t {
+    if constexpr (L::SPLIT_REGS) {
+      cudaFuncAttributes attr{};
+      cudaError_t r = cudaFuncGetAttributes(&attr, kern);
+      if (r != cudaSuccess) return r;
+      if (attr.numRegs != 128) return cudaErrorInvalidConfiguration;
+    }
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(L::SMEM));
   });
