@@ -370,6 +370,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
 
+      // dK += dS^T Q   (A = dS^T K-major in shared memory, B = Q MN-major)
+      auto issue_dk = [&](uint32_t q_addr, int it) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::COL_DK, sdesc_sw128(ds_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(q_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+      };
+      // dQ_tile = dS K (A = dS MN-major, B = K MN-major), or at d = 128 its
+      // transpose dQ^T = K^T dS^T (A = K^T MN-major, B = dS^T MN-major)
+      auto issue_dq = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ds_desc = sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024);
+          const uint64_t k_desc = sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024);
+          if constexpr (L::DQ_T)
+            mma_ss(tmem + L::COL_DQ, k_desc, ds_desc, kIdQ, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tmem + L::COL_DQ, ds_desc, k_desc, kIdQ, kk > 0 ? 1u : 0u);
+        }
+      };
+
       int it = 0;
       if (ok) ok = mbar_wait(bar(L::B_QFULL + 0), 0, g);
       if (ok) {
@@ -398,30 +420,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
             issue_sdp(sn, false);
           }
-          // dS of this tile is in shared memory: dK += dS^T Q  (A = dS^T K-major, B = Q MN-major)
+          // dS of this tile is in shared memory: dK and dQ
           if (!mbar_wait(bar(L::B_DSFULL), it & 1u, g)) break;
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + L::COL_DK, sdesc_sw128(ds_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(q_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          // dQ_tile = dS K   (A = dS MN-major, B = K MN-major)
-          if (L::SEPARATE_DQ && it > 0) {
-            // the dQ columns must have been drained by the previous iteration
-            if (!mbar_wait(bar(L::B_DQEMPTY), (it - 1) & 1u, g)) break;
-            tc_fence_after();
+          if constexpr (L::DQ_T) {
+            // d = 128: dQ^T first, so that its drain out of TMEM runs under
+            // the dK MMAs and the next dP^T (same columns) is not kept waiting
+            issue_dq();
+            mma_commit(bar(L::B_DQFULL));
+            issue_dk(q_addr, it);
+          } else {
+            // d = 64: dK first (the dQ warps stage into this tile's Q / dO
+            // stage once the dQ MMAs are done, and dK reads Q from it)
+            issue_dk(q_addr, it);
+            if (L::SEPARATE_DQ && it > 0) {
+              // the dQ columns must have been drained by the previous iteration
+              if (!mbar_wait(bar(L::B_DQEMPTY), (it - 1) & 1u, g)) break;
+              tc_fence_after();
+            }
+            issue_dq();
+            mma_commit(bar(L::B_DQFULL));
           }
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ds_desc = sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024);
-            const uint64_t k_desc = sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024);
-            if constexpr (L::DQ_T)  // dQ^T = K^T dS^T: A = K^T (MN-major), B = dS^T (MN-major)
-              mma_ss(tmem + L::COL_DQ, k_desc, ds_desc, kIdQ, kk > 0 ? 1u : 0u);
-            else
-              mma_ss(tmem + L::COL_DQ, ds_desc, k_desc, kIdQ, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(L::B_DQFULL));
           mma_commit(bar(L::B_DSEMPTY));
           if constexpr (!L::TMA_REDUCE) mma_commit(bar(L::B_QEMPTY + s));
           if (qbn < w.nqb) {
@@ -462,28 +481,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             issue_sdp(sn, false);
             if (L::SEPARATE_DQ) issue_sdp(sn, true);
           }
-          // dK += dS^T Q   (A = dS^T K-major in shared memory, B = Q MN-major)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + L::COL_DK, sdesc_sw128(ds_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(q_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          // dQ_tile = dS K   (A = dS MN-major, B = K MN-major)
-          if (L::SEPARATE_DQ && it > 0) {
-            // the dQ columns must have been drained by the previous iteration
-            if (!mbar_wait(bar(L::B_DQEMPTY), (it - 1) & 1u, g)) break;
-            tc_fence_after();
+          if constexpr (L::DQ_T) {
+            // d = 128: dQ^T first (its drain runs under dK, see above)
+            issue_dq();
+            mma_commit(bar(L::B_DQFULL));
+            issue_dk(q_addr, it);
+          } else {
+            issue_dk(q_addr, it);
+            if (L::SEPARATE_DQ && it > 0) {
+              // the dQ columns must have been drained by the previous iteration
+              if (!mbar_wait(bar(L::B_DQEMPTY), (it - 1) & 1u, g)) break;
+              tc_fence_after();
+            }
+            issue_dq();
+            mma_commit(bar(L::B_DQFULL));
           }
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ds_desc = sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024);
-            const uint64_t k_desc = sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024);
-            if constexpr (L::DQ_T)  // dQ^T = K^T dS^T: A = K^T (MN-major), B = dS^T (MN-major)
-              mma_ss(tmem + L::COL_DQ, k_desc, ds_desc, kIdQ, kk > 0 ? 1u : 0u);
-            else
-              mma_ss(tmem + L::COL_DQ, ds_desc, k_desc, kIdQ, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(L::B_DQFULL));
           mma_commit(bar(L::B_DSEMPTY));
           if constexpr (!L::TMA_REDUCE) mma_commit(bar(L::B_QEMPTY + s));
           if (!L::SEPARATE_DQ && qbn < w.nqb) {
