@@ -27,7 +27,7 @@ LSE = m + ln(l), the (m, l) pair of the online softmax collapsed to one number
 (same page, closing "解决方案" paragraph, whose symbol list is garbled; the
 running max m and row sum l are the readings used here).
 
-Readings taken where the pages are silent (all are repeated in the design doc):
+Readings taken where the pages are silent:
   * scale is a caller-given float applied to Q K^T before masking and the max;
   * causal: query i may attend key j iff j <= i + (N_k - N_q) (0-based; the
     last query is aligned with the last key, "bottom-right"; with N_q = N_k
