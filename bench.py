@@ -7,7 +7,10 @@ already resident in device memory.  Timing: W untimed warm-up steps, then the
 timed steps, each bracketed by CUDA events on the launching stream, with a
 256 MiB write between steps so that no step finds its inputs in the 126 MB
 L2.  A barrier and a device synchronisation bracket the timed steps; the
-reported time is the maximum over ranks.
+reported time is the maximum over ranks.  Nothing is recorded between the
+launches of a timed step (the library's kernels may start launching under
+their predecessor's last wave); the per-launch split comes from a second
+pass of the same steps with an event between every two launches.
 
 The default run times every workload (tiny, GPT-2, BERT, long d=64, long
 d=128, block-sparse) one after the other.  The headline ``value`` is the
@@ -223,15 +226,17 @@ def max_over_ranks(x, world, device):
     return float(t.item())
 
 
-def kernel_summary(w, eff, fwd_ms, pre_ms, main_ms, post_ms, peak, traffic_key=None):
+def kernel_summary(w, eff, fwd_ms, pre_ms, main_ms, post_ms, peak, traffic_key=None,
+                   step_ms=None):
     """Per-kernel and per-pass TFLOP/s (nominal and effective) of one workload
-    and its dominant kernel against the peak (effective count)."""
+    and its dominant kernel against the peak (effective count).  step_ms: the
+    step timed without events between its launches (default: their sum)."""
     f_fwd, f_bwd = attention_flops(w.B, w.H, w.N, w.d, w.causal)
     bwd_ms = pre_ms + main_ms + post_ms
-    tot_ms = fwd_ms + bwd_ms
+    tot_ms = fwd_ms + bwd_ms if step_ms is None else step_ms
     out = {
         "ms": {"fwd": fwd_ms, "bwd_pre": pre_ms, "bwd_main": main_ms, "bwd_post": post_ms,
-               "step": tot_ms},
+               "step": tot_ms, "step_with_events_between_launches": fwd_ms + bwd_ms},
         "nominal_tflops": {"fwd": tflops(f_fwd, fwd_ms), "bwd_main": tflops(f_bwd, main_ms),
                            "bwd": tflops(f_bwd, bwd_ms), "fwd_bwd": tflops(f_fwd + f_bwd, tot_ms)},
         "effective_tflops": {"fwd": tflops(eff * f_fwd, fwd_ms),
@@ -533,10 +538,11 @@ def measure_packed(fa, w, args, rank, dev, flush, stream, world, local, peak):
     entry = {"workload": describe(w) + " packed (fa_fwd_ex / fa_bwd_ex, no padding rows)",
              "steps": steps, "timed_s": total_ms * 1e-3, "clocks": clocks,
              "device_status": fa.last_device_status(),
-             "ms": {"fwd": fwd_ms, "bwd": bwd_ms, "step": fwd_ms + bwd_ms},
+             "ms": {"fwd": fwd_ms, "bwd": bwd_ms, "step": total_ms / steps,
+                    "step_with_events_between_launches": fwd_ms + bwd_ms},
              "flops_per_launch": {"fwd_kernel": f_fwd, "bwd (3 launches)": f_bwd},
              "tflops": {"fwd": tflops(f_fwd, fwd_ms), "bwd": tflops(f_bwd, bwd_ms),
-                        "fwd_bwd": tflops(f_fwd + f_bwd, fwd_ms + bwd_ms)},
+                        "fwd_bwd": tflops(f_fwd + f_bwd, total_ms / steps)},
              "flops": "4 H d sum_b len_b^2 forward, 2.5x backward: every counted pair is valid",
              "tokens": int(case.lens.sum())}
     entry["pct_of_peak"] = {k: 100.0 * v / peak for k, v in entry["tflops"].items()}
@@ -604,24 +610,36 @@ def measure_projection(fa, name, args, rank, dev, flush, stream, world, local, p
 
 
 def timed_region(case, steps, flush, stream, dev, world, clk_index):
-    """Times `steps` steps (events per launch, L2 flushed before each); returns
-    per-launch mean ms (max over ranks) and the clock record."""
+    """Times `steps` steps, L2 flushed before each, in two passes: the steps
+    alone, one event before and one after each (nothing between the launches,
+    which may then start under their predecessor's last wave), for the step
+    time; then again with an event between every two launches, for the
+    per-launch split.  Returns the per-launch means of the second pass, the
+    total of the first (ms, max over ranks) and the first pass's clock record."""
     import torch
     import torch.distributed as dist
+    ends = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(steps)]
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(clk_index) as clk:
-        for i in range(steps):
+        for a, b in ends:
             flush.zero_()
-            case.step(stream, events[i])
+            a.record(stream)
+            case.step(stream)
+            b.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    total = max_over_ranks(sum(a.elapsed_time(b) for a, b in ends), world, dev)
+    for i in range(steps):
+        flush.zero_()
+        case.step(stream, events[i])
+    torch.cuda.synchronize(dev)
     parts = [[e[a].elapsed_time(e[a + 1]) for e in events] for a in range(4)]
     sums = [max_over_ranks(sum(p), world, dev) for p in parts]
-    total = max_over_ranks(sum(e[0].elapsed_time(e[4]) for e in events), world, dev)
     return [s / steps for s in sums], total, clk.summary()
 
 
@@ -726,7 +744,8 @@ def run_ours(args):
     w = w_head
     f_fwd, f_bwd = attention_flops(w.B, w.H, w.N, w.d, w.causal)
     value = job_throughput(world, f_fwd + f_bwd, args.steps, total_ms)
-    summ = kernel_summary(w, case.eff, fwd_ms, pre_ms, main_ms, post_ms, peak)
+    summ = kernel_summary(w, case.eff, fwd_ms, pre_ms, main_ms, post_ms, peak,
+                          step_ms=total_ms / args.steps)
     dom = summ["dominant"]
     roofline = {"bound": "tensor", "kernel": dom["kernel"],
                 "achieved": dom["achieved_effective_tflops"], "peak": peak, "unit": "TFLOP/s",
@@ -877,7 +896,8 @@ def measure_config(fa, w, args, rank, dev, flush, stream, world, local, peak):
     status = fa.last_device_status()
     entry = {"workload": describe(w), "steps": steps, "timed_s": total_ms * 1e-3,
              "clocks": clocks, "device_status": status}
-    entry.update(kernel_summary(w, case.eff, fwd_ms, pre_ms, main_ms, post_ms, peak))
+    entry.update(kernel_summary(w, case.eff, fwd_ms, pre_ms, main_ms, post_ms, peak,
+                                step_ms=total_ms / steps))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         entry["cpu_baseline"] = cpu_baseline(w, case.inp, args.cpu_seconds_per_config)
     if w.name == "tiny":

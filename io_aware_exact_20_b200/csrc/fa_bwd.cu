@@ -145,6 +145,8 @@ constexpr int kRowsPerBlock = 256 / (D / 8);
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   constexpr int G = D / 8;  // threads per row, 8 elements each
+  griddep_wait();
+  griddep_launch_dependents();
   const int bh = blockIdx.y;
   const int b = bh / p.H, h = bh % p.H;
   const Seq sq = seq_of(p.rows, b);
@@ -191,6 +193,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
 template <int D>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
   constexpr int G = D / 8;
+  griddep_wait();
+  griddep_launch_dependents();
   const int bh = blockIdx.y;
   const int b = bh / p.H, h = bh % p.H;
   const Seq sq = seq_of(p.rows, b);
@@ -225,6 +229,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // are the bottleneck and the serialized order lets the keep-bit generation
   // of the next tile hide under that tile's MMAs instead.
   constexpr bool kTwoPhase = !DROPOUT;
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {
@@ -892,8 +898,7 @@ dim3 prepost_grid(const BwdParams& p) {
 
 template <int D>
 cudaError_t launch_pre_t(const BwdParams& p, cudaStream_t stream) {
-  bwd_pre_kernel<D><<<prepost_grid<D>(p), 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_overlapped(bwd_pre_kernel<D>, prepost_grid<D>(p), dim3(256), 0, stream, p);
 }
 
 template <int D, bool DROPOUT>
@@ -918,14 +923,13 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   if (e != cudaSuccess) return e;
   const long long ctas = static_cast<long long>((p.rows.nk + 127) / 128) * p.B * p.H;
   if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(ctas), kBwdThreads, L::SMEM, stream>>>(tq, tk, tv, tdo, tdq, p);
-  return cudaGetLastError();
+  return launch_overlapped(kern, dim3(static_cast<unsigned>(ctas)), dim3(kBwdThreads), L::SMEM,
+                           stream, tq, tk, tv, tdo, tdq, p);
 }
 
 template <int D>
 cudaError_t launch_post_t(const BwdParams& p, cudaStream_t stream) {
-  bwd_post_kernel<D><<<prepost_grid<D>(p), 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_overlapped(bwd_post_kernel<D>, prepost_grid<D>(p), dim3(256), 0, stream, p);
 }
 
 }  // namespace

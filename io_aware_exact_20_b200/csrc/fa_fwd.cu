@@ -154,6 +154,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   using L = FwdLayout<D>;
   using C = FwdCfg<D>;
   constexpr int NQ = C::NQ, NS = C::NS, KS = C::KS, KW = C::KW;
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {  // the swizzled layouts need 1024-byte alignment
@@ -647,8 +649,8 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   const long long ctas =
       static_cast<long long>((p.rows.nq + 128 * C::NQ - 1) / (128 * C::NQ)) * p.B * p.H;
   if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(ctas), C::THREADS, L::SMEM, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  return launch_overlapped(kern, dim3(static_cast<unsigned>(ctas)), dim3(C::THREADS), L::SMEM,
+                           stream, tq, tk, tv, p);
 }
 
 }  // namespace

@@ -64,6 +64,8 @@ struct ProjParams {
 __global__ void __launch_bounds__(kProjThreads, 1)
     qkv_proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                     const ProjParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {
@@ -285,8 +287,8 @@ cudaError_t launch_qkv_projection(const void* x, const void* w, const void* bias
   });
   if (e != cudaSuccess) return e;
   const int grid = p.tiles < sms ? p.tiles : sms;
-  qkv_proj_kernel<<<grid, kProjThreads, kProjSmem, stream>>>(tx, tw, p);
-  return cudaGetLastError();
+  return launch_overlapped(qkv_proj_kernel, dim3(static_cast<unsigned>(grid)), dim3(kProjThreads),
+                           kProjSmem, stream, tx, tw, p);
 }
 
 }  // namespace fa

@@ -10,6 +10,26 @@
 
 namespace fa {
 
+// Launches `kern` on `stream` with programmatic stream serialization: it may
+// start launching while the previous kernel of the stream finishes its last
+// wave (every kernel of the library waits for its predecessor with
+// griddepcontrol.wait before touching global memory, see ptx.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_overlapped(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // Grid order of the forward and backward CTAs.  The 1-D grid walks groups of
 // `group_heads` (b, h) heads one after the other and, inside a group, puts the
 // tile index slowest: every head's heaviest tile first, a longest-processing-

@@ -43,6 +43,24 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 // ----------------------------------------------------------------------------
+// programmatic dependent launch
+// ----------------------------------------------------------------------------
+
+// Waits until the grids this grid depends on (the previous kernel in the
+// stream, when this one was launched with programmatic stream serialization)
+// have completed and their writes are visible.  A no-op for a normal launch.
+// Every kernel of the library calls it before its first global-memory access,
+// so that launching early only overlaps the launch latency and the CTA
+// rasterisation with the previous kernel's last wave.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel in the stream (if launched with programmatic stream
+// serialization) start launching once every CTA of this grid has executed it.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------------
 // mbarrier
 // ----------------------------------------------------------------------------
 
