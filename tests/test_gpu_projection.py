@@ -33,3 +33,33 @@ def test_qkv_projection_matches_oracle(lib, B, N, H, d, dm, bias):
     for got, r in zip((q, k, v), ref):
         err = np.abs(f64(got) - r)
         assert (err <= 2.0 ** -8 * np.abs(r) + 1e-3).all(), err.max()
+
+
+def test_projection_output_feeds_attention_back_to_back(lib):
+    """The projection and the attention forward / backward launched back to
+    back on one stream (each may start launching under its predecessor's last
+    wave, and must wait for it before reading): the attention reads the Q, K,
+    V the projection has just written, and a torch kernel that rewrites V in
+    between is seen by the next call."""
+    import torch
+    from oracle import attention_forward
+    B, N, H, d, dm = 2, 384, 2, 64, 256
+    g = torch.Generator().manual_seed(77)
+    x = torch.randn(B * N, dm, generator=g).to(torch.bfloat16).cuda()
+    w = (torch.randn(3 * H * d, dm, generator=g) / dm ** 0.5).to(torch.bfloat16).cuda()
+    q, k, v = lib.qkv_projection(x, w, None, B, H, d)
+    o1, _ = lib.forward(q, k, v, causal=True)
+    v.mul_(-2.0)                      # a torch kernel between two library calls
+    o2, lse2 = lib.forward(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert lib.last_device_status() == 0
+    rq, rk, rv = qkv_projection(f64(x), f64(w), None, B, H, d)
+    # the oracle on the bf16 values the kernels actually read
+    qb, kb, vb = (f64(t) for t in (q, k, v))
+    ro1, _ = attention_forward(qb, kb, -0.5 * vb, d ** -0.5, True)
+    ro2, rl2 = attention_forward(qb, kb, vb, d ** -0.5, True)
+    assert np.abs(f64(o1) - ro1).max() <= 1e-2 + 2.0 ** -8 * np.abs(ro1).max()
+    assert np.abs(f64(o2) - ro2).max() <= 1e-2 + 2.0 ** -8 * np.abs(ro2).max()
+    assert np.abs(lse2.cpu().numpy() - rl2).max() <= 1e-3
+    for got, r in zip((q, k), (rq, rk)):
+        assert (np.abs(f64(got) - r) <= 2.0 ** -8 * np.abs(r) + 1e-3).all()
