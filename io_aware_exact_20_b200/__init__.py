@@ -295,12 +295,25 @@ def _dims(t, layout):
     return None, t.shape[0], t.shape[1], t.shape[2]
 
 
+# the tensors of a call that have Q's shape; the others (k, v, dk, dv) have K's
+_Q_SIDE = ("q", "o", "dout", "dq")
+
+
 def _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, scale, causal,
           seqlens_k, dropout_p, seed, block_mask, tensors):
     import torch
-    for t in (q, k):
-        if not t.is_cuda or t.dtype != torch.bfloat16:
-            raise ValueError("tensors must be bfloat16 on a CUDA device")
+    if layout not in ("bhsd", "bshd", "thd"):
+        raise ValueError(f"unknown layout {layout!r}")
+    want_dim = 3 if layout == "thd" else 4
+    for name, t in tensors.items():
+        if t.dim() != want_dim:
+            raise ValueError(f"{name}: a {want_dim}-D tensor is expected for layout {layout!r}")
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.device != q.device:
+            raise ValueError(f"{name}: bfloat16 on the device of q is expected")
+        ref = q if name in _Q_SIDE else k
+        if t.shape != ref.shape:
+            raise ValueError(f"{name}: shape {tuple(t.shape)} differs from "
+                             f"{'q' if name in _Q_SIDE else 'k'} {tuple(ref.shape)}")
     Bq, Nq, H, d = _dims(q, layout)
     Bk, Nk, Hk, dk = _dims(k, layout)
     if H != Hk or d != dk:
@@ -355,16 +368,29 @@ def forward_general(q, k, v, *, layout="bhsd", cu_seqlens_q=None, cu_seqlens_k=N
                     causal, seqlens_k, dropout_p, seed, block_mask,
                     dict(q=q, k=k, v=v, o=out))
     if lse is None:
-        if layout == "thd":
-            lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
-        else:
-            B, Nq, H, _ = _dims(q, layout)
-            lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+        lse = torch.empty(_lse_shape(q, layout), dtype=torch.float32, device=q.device)
+    _check_lse(lse, q, layout)
     code = library().fa_fwd_ex(ctypes.byref(a), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                                _stream_ptr(q.device))
     _check(code, "fa_fwd_ex")
     del keep
     return out, lse
+
+
+def _lse_shape(q, layout):
+    """[B, H, N_q] (padded layouts) or [H, T_q] (packed)."""
+    if layout == "thd":
+        return (q.shape[1], q.shape[0])
+    B, Nq, H, _ = _dims(q, layout)
+    return (B, H, Nq)
+
+
+def _check_lse(lse, q, layout):
+    import torch
+    shape = _lse_shape(q, layout)
+    if (lse.dtype != torch.float32 or lse.device != q.device or tuple(lse.shape) != shape
+            or not lse.is_contiguous()):
+        raise ValueError(f"lse: contiguous float32 {shape} on the device of q is expected")
 
 
 def general_workspace_size(q, k, **kw):
@@ -389,10 +415,13 @@ def backward_general(q, k, v, o, lse, dout, *, layout="bhsd", cu_seqlens_q=None,
     a, keep = _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, scale,
                     causal, seqlens_k, dropout_p, seed, block_mask,
                     dict(q=q, k=k, v=v, o=o, dout=dout, dq=dq, dk=dk, dv=dv))
+    _check_lse(lse, q, layout)
     lib = library()
     need = int(lib.fa_bwd_ex_workspace_size(ctypes.byref(a)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    elif not workspace.is_cuda or workspace.device != q.device:
+        raise ValueError("workspace: a tensor on the device of q is expected")
     code = lib.fa_bwd_ex(ctypes.byref(a), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                          _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _stream_ptr(q.device))

@@ -153,3 +153,18 @@ def test_qkv_projection_rejects_bad_shapes(lib):
     assert so.fa_qkv_projection(a, a, None, a, a, a, 1, 128, 2, 64, 60, None) == 1  # d_model % 8
     assert so.fa_qkv_projection(a + 8, a, None, a, a, a, 1, 128, 2, 64, 64, None) == 1
     assert so.fa_qkv_projection(a, a, a + 2, a, a, a, 1, 128, 2, 64, 64, None) == 1  # bias align
+
+
+def test_general_binding_rejects_host_tensors_and_bad_layouts(lib):
+    """The general-layout binding checks its tensors before it marshals a call:
+    host tensors, an unknown layout and a tensor of the wrong rank raise."""
+    import torch
+    q = torch.zeros((1, 2, 128, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="device of q"):
+        lib.forward_general(q, q, q)
+    with pytest.raises(ValueError, match="unknown layout"):
+        lib.forward_general(q, q, q, layout="sbhd")
+    with pytest.raises(ValueError, match="3-D tensor"):
+        lib.forward_general(q, q, q, layout="thd")
+    with pytest.raises(ValueError, match="device of q"):
+        lib.backward_general(q, q, q, q, torch.zeros((1, 2, 128)), q)
