@@ -22,23 +22,28 @@
 namespace fa {
 namespace {
 
-// G threads per row, 8 columns each (G = d / 8 divides 32, so a row's threads
-// sit in one warp).
+// G threads per row; the row's d / 8 chunks of 8 columns are dealt out to them
+// round-robin (thread `part` takes chunks part, part + G, ...).  G is the
+// largest power of two dividing d / 8 (4, 8, 4, 16 for d = 32, 64, 96, 128),
+// so it divides 32 and a row's threads sit in one warp: the row's two LSEs are
+// read once and passed around by shuffles, and the new LSE is written after
+// every thread of the row has read the old one.
 __global__ void __launch_bounds__(256) merge_kernel(float* o_acc, float* lse_acc,
                                                     const __nv_bfloat16* o_part,
-                                                    const float* lse_part, long long rows, int G) {
+                                                    const float* lse_part, long long rows, int d,
+                                                    int G) {
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long row = tid / G;
   const int part = static_cast<int>(tid % G);
   const bool live = row < rows;
   const int lane = threadIdx.x & 31;
-  const int first = lane - part;  // lane of this row's part 0
+  const int first = lane - part;  // lane of this row's part 0, in this warp
   float la = 0.f, lb = 0.f;
   if (live && part == 0) {
     la = lse_acc[row];
     lb = lse_part[row];
   }
-  // every lane of the warp takes part in the shuffles (rows never straddle warps)
+  // every lane of the warp takes part in the shuffles
   la = __shfl_sync(0xffffffffu, la, first);
   lb = __shfl_sync(0xffffffffu, lb, first);
   if (!live) return;
@@ -51,20 +56,22 @@ __global__ void __launch_bounds__(256) merge_kernel(float* o_acc, float* lse_acc
     fb = eb / s;
     lse = m + logf(s);
   }
-  const long long off = row * (8ll * G) + 8 * part;
-  float4* a = reinterpret_cast<float4*>(o_acc + off);
-  const uint4 pb = *reinterpret_cast<const uint4*>(o_part + off);
-  const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&pb);
-  float4 a0 = a[0], a1 = a[1];
-  const float2 b0 = __bfloat1622float2(p2[0]), b1 = __bfloat1622float2(p2[1]);
-  const float2 b2 = __bfloat1622float2(p2[2]), b3 = __bfloat1622float2(p2[3]);
-  // an empty accumulator may hold anything finite; fa = 0 then discards it
-  a0 = make_float4(fa * a0.x + fb * b0.x, fa * a0.y + fb * b0.y, fa * a0.z + fb * b1.x,
-                   fa * a0.w + fb * b1.y);
-  a1 = make_float4(fa * a1.x + fb * b2.x, fa * a1.y + fb * b2.y, fa * a1.z + fb * b3.x,
-                   fa * a1.w + fb * b3.y);
-  a[0] = a0;
-  a[1] = a1;
+  for (int c = part; c < d / 8; c += G) {
+    const long long off = row * d + 8 * c;
+    float4* a = reinterpret_cast<float4*>(o_acc + off);
+    const uint4 pb = *reinterpret_cast<const uint4*>(o_part + off);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&pb);
+    float4 a0 = a[0], a1 = a[1];
+    const float2 b0 = __bfloat1622float2(p2[0]), b1 = __bfloat1622float2(p2[1]);
+    const float2 b2 = __bfloat1622float2(p2[2]), b3 = __bfloat1622float2(p2[3]);
+    // an empty accumulator may hold anything finite; fa = 0 then discards it
+    a0 = make_float4(fa * a0.x + fb * b0.x, fa * a0.y + fb * b0.y, fa * a0.z + fb * b1.x,
+                     fa * a0.w + fb * b1.y);
+    a1 = make_float4(fa * a1.x + fb * b2.x, fa * a1.y + fb * b2.y, fa * a1.z + fb * b3.x,
+                     fa * a1.w + fb * b3.y);
+    a[0] = a0;
+    a[1] = a1;
+  }
   if (part == 0) lse_acc[row] = lse;
 }
 
@@ -110,10 +117,10 @@ fa_status_t fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part,
     return FA_ERR_INVALID_ARG;
   if (d != 32 && d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
   if (rows == 0) return FA_OK;
-  const int G = d / 8;
+  const int G = (d / 8) & -(d / 8);  // largest power of two dividing d / 8
   if (rows * G / 256 >= 0x7FFFFFFFll) return FA_ERR_UNSUPPORTED;
   fa::merge_kernel<<<fa::blocks_for(rows * G), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      o_acc, lse_acc, static_cast<const __nv_bfloat16*>(o_part), lse_part, rows, G);
+      o_acc, lse_acc, static_cast<const __nv_bfloat16*>(o_part), lse_part, rows, d, G);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
