@@ -82,7 +82,12 @@ struct BwdLayout {
   static constexpr int B_STAGED = B_KVDONE + 1;   // dQ tile written to the staging boxes
   static constexpr int NBAR = B_STAGED + 1;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr uint32_t SMEM = OFF_MISC + 16;
+  // block masks at d = 64: bitmask of the query tiles this key tile meets
+  // (up to 32 BIT_WORDS query tiles).  d = 128 keeps the direct walk: its
+  // producer / MMA warps run at 72 registers, which the bitmask walk exceeds.
+  static constexpr int BIT_WORDS = (D == 64) ? 1024 : 0;
+  static constexpr uint32_t OFF_BITS = OFF_MISC + 16;
+  static constexpr uint32_t SMEM = OFF_BITS + BIT_WORDS * 4;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   // d = 64 leaves room for a dQ tile of its own; d = 128 reuses the dP^T
   // columns once dP^T has been consumed.
@@ -116,11 +121,20 @@ struct BwdLayout {
 // sequence's first query / key, tb its batch coordinate and ws0 its first
 // workspace row.  Under the causal mask query i sees key j iff j <= i + off
 // (bottom-right alignment, off = keys - queries of the sequence).
+//
+// Under a block mask the CTA first gathers the query tiles its key tile meets
+// into a bitmask in shared memory (one pass over the mask column); the roles
+// then find their next query tile with a word read and a find-first-set.
+// Kernels launched without a block mask, with columns longer than the
+// bitmask, or at d = 128 are built without it (kBits false) and test the
+// mask's bytes directly.
+template <bool kBits>
 struct BwdWork {
   int b, h, bh, kb, kv_len, nqb, qb_begin, nbk, off, qrow, krow, tb, lk;
   long long ws0;
   bool alive, causal;
   const uint8_t* bm;
+  const uint32_t* bits;  // shared-memory bitmask over the query tiles, or null
 
   __device__ __forceinline__ bool act(int qb) const {
     if (!alive) return false;
@@ -128,6 +142,14 @@ struct BwdWork {
     return true;
   }
   __device__ __forceinline__ int next(int qb) const {
+    if (kBits && bits != nullptr) {
+      while (qb < nqb) {
+        const uint32_t x = bits[qb >> 5] >> (qb & 31);
+        if (x != 0u) return min(qb + __ffs(x) - 1, nqb);
+        qb = (qb | 31) + 1;
+      }
+      return nqb;
+    }
     while (qb < nqb && !act(qb)) ++qb;
     return qb;
   }
@@ -218,7 +240,7 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
 // main kernel
 // ---------------------------------------------------------------------------
 
-template <int D, bool DROPOUT>
+template <int D, bool DROPOUT, bool BITS>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -244,7 +266,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  BwdWork w;
+  BwdWork<BITS> w;
   grid_unit(blockIdx.x, p.B * p.H, (p.rows.nk + 127) / 128, p.group_heads, &w.bh,
             &w.kb);  // key tile 0 is heaviest
   w.b = w.bh / p.H;
@@ -275,6 +297,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   w.nbk = p.nbk;
   w.bm = p.block_mask;
+  w.bits = nullptr;
+  if (BITS && w.bm != nullptr && (w.nqb + 31) / 32 <= L::BIT_WORDS) {
+    // every thread takes part: a warp's lanes test 32 consecutive query tiles
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L::OFF_BITS);
+    const int words = (w.nqb + 31) / 32;
+    for (int wi = warp; wi < words; wi += kBwdThreads / 32) {
+      const int qb = wi * 32 + lane;
+      const uint32_t word = __ballot_sync(0xffffffffu, qb < w.nqb && w.act(qb));
+      if (lane == 0) bits[wi] = word;
+    }
+    w.bits = bits;  // read after the __syncthreads below
+  }
 
   if (threadIdx.x == 0) {
     *abort_flag = 0u;
@@ -901,12 +935,13 @@ cudaError_t launch_pre_t(const BwdParams& p, cudaStream_t stream) {
   return launch_overlapped(bwd_pre_kernel<D>, prepost_grid<D>(p), dim3(256), 0, stream, p);
 }
 
-template <int D, bool DROPOUT>
+template <int D, bool DROPOUT, bool BITS>
 cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdParams& p,
                           cudaStream_t stream) {
   using L = BwdLayout<D>;
-  auto kern = bwd_main_kernel<D, DROPOUT>;
+  static_assert(!BITS || L::BIT_WORDS > 0, "no bitmask at this head dim");
+  auto kern = bwd_main_kernel<D, DROPOUT, BITS>;
   // The setmaxnreg split (d = 128) is sized for exactly 128 registers per
   // thread at launch; with any other count an increase could wait forever.
   static OncePerContext prepared;
@@ -943,10 +978,19 @@ cudaError_t launch_bwd_pre(int d, const BwdParams& p, cudaStream_t stream) {
 cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdq,
                             const BwdParams& p, cudaStream_t stream) {
-  if (d == 64) return dropout ? launch_main_t<64, true>(tq, tk, tv, tdo, tdq, p, stream)
-                              : launch_main_t<64, false>(tq, tk, tv, tdo, tdq, p, stream);
-  if (d == 128) return dropout ? launch_main_t<128, true>(tq, tk, tv, tdo, tdq, p, stream)
-                               : launch_main_t<128, false>(tq, tk, tv, tdo, tdq, p, stream);
+  if (d == 64) {
+    // a block mask whose columns fit the bitmask (the CTAs' query tiles are
+    // below the longest sequence's)
+    const bool bits = p.block_mask != nullptr &&
+                      ((p.rows.nq + 127) / 128 + 31) / 32 <= BwdLayout<64>::BIT_WORDS;
+    if (bits)
+      return dropout ? launch_main_t<64, true, true>(tq, tk, tv, tdo, tdq, p, stream)
+                     : launch_main_t<64, false, true>(tq, tk, tv, tdo, tdq, p, stream);
+    return dropout ? launch_main_t<64, true, false>(tq, tk, tv, tdo, tdq, p, stream)
+                   : launch_main_t<64, false, false>(tq, tk, tv, tdo, tdq, p, stream);
+  }
+  if (d == 128) return dropout ? launch_main_t<128, true, false>(tq, tk, tv, tdo, tdq, p, stream)
+                               : launch_main_t<128, false, false>(tq, tk, tv, tdo, tdq, p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -103,7 +103,11 @@ struct FwdLayout {
   static constexpr int B_DRAIN = B_ODONE + C::NS;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr uint32_t SMEM = OFF_MISC + 16;
+  // block masks: per Q tile a bitmask of the K/V tiles it takes part in
+  // (BIT_WORDS / NQ words each, so up to 32768 / NQ key tiles)
+  static constexpr int BIT_WORDS = 1024;
+  static constexpr uint32_t OFF_BITS = OFF_MISC + 16;
+  static constexpr uint32_t SMEM = OFF_BITS + BIT_WORDS * 4;
   static constexpr uint32_t TMEM_COLS = NQ == 2 ? 512 : 256;
   static constexpr uint32_t O_COL = C::KW * C::NS;
   static_assert(SMEM <= (NQ == 2 ? 232448u : 113u * 1024u), "shared memory budget");
@@ -115,19 +119,34 @@ struct FwdLayout {
 // sequence's first query / key and tb its batch coordinate.  Under the causal
 // mask query i sees key j iff j <= i + off, off = (keys) - (queries) of the
 // sequence (bottom-right alignment).
+//
+// Under a block mask the CTA first gathers, for each of its Q tiles, the K/V
+// tiles below kb_end that take part into a bitmask in shared memory (one
+// coalesced pass over the mask row); every role then finds its next tile with
+// a word read and a find-first-set instead of testing the mask's bytes one by
+// one.  kRows bitmask rows (one per Q tile) of kWpr words each; kernels
+// launched without a block mask, or with rows longer than the bitmask, are
+// built without it (kBits false) and test the mask's bytes directly.
+template <int kRows, int kWpr, bool kBits>
 struct FwdWork {
   int b, h, bh, q0, qb0, lq, kv_len, n_kb, kb_end, nbk, off, qrow, krow, tb;
   bool exists1, causal;
   const uint8_t* bm;
+  const uint32_t* bits;  // shared-memory bitmask rows, or null
 
   // last row of Q tile t that exists in the sequence
   __device__ __forceinline__ int last_row(int t) const { return min(q0 + 128 * t + 127, lq - 1); }
-  __device__ __forceinline__ bool act(int t, int kb) const {
+  __device__ __forceinline__ bool act_direct(int t, int kb) const {
     if (t == 1 && !exists1) return false;
     if (kb >= n_kb) return false;
     if (causal && kb * 128 > last_row(t) + off) return false;
     if (bm != nullptr && bm[static_cast<size_t>(qb0 + t) * nbk + kb] == 0) return false;
     return true;
+  }
+  // kb < kb_end here (every caller walks below kb_end)
+  __device__ __forceinline__ bool act(int t, int kb) const {
+    if (kBits && bits != nullptr) return t < kRows && ((bits[t * kWpr + (kb >> 5)] >> (kb & 31)) & 1u);
+    return act_direct(t, kb);
   }
   // stream (Q tile t, key part hp of kw keys): also skipped when all its keys
   // are past the key length
@@ -136,6 +155,16 @@ struct FwdWork {
   }
   __device__ __forceinline__ bool any(int kb) const { return act(0, kb) || act(1, kb); }
   __device__ __forceinline__ int next(int kb) const {
+    if (kBits && bits != nullptr) {
+      while (kb < kb_end) {
+        uint32_t x = bits[kb >> 5];
+        if (kRows == 2) x |= bits[kWpr + (kb >> 5)];
+        x >>= (kb & 31);
+        if (x != 0u) return min(kb + __ffs(x) - 1, kb_end);
+        kb = (kb | 31) + 1;
+      }
+      return kb_end;
+    }
     while (kb < kb_end && !any(kb)) ++kb;
     return kb;
   }
@@ -147,7 +176,7 @@ __device__ __forceinline__ void named_bar_sync() {
   asm volatile("bar.sync %0, 256;" ::"n"(kId) : "memory");
 }
 
-template <int D, bool DROPOUT>
+template <int D, bool DROPOUT, bool BITS>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -170,7 +199,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  FwdWork w;
+  FwdWork<NQ, L::BIT_WORDS / NQ, BITS> w;
   {
     const int nqp = (p.rows.nq + 128 * NQ - 1) / (128 * NQ);
     int tile = 0;
@@ -203,6 +232,20 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     }
     w.nbk = p.nbk;
     w.bm = p.block_mask;
+    w.bits = nullptr;
+  }
+  constexpr int kWpr = L::BIT_WORDS / NQ;
+  if (BITS && w.bm != nullptr && (w.kb_end + 31) / 32 <= kWpr) {
+    // every thread takes part: a warp's lanes test 32 consecutive K/V tiles
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L::OFF_BITS);
+    const int words = (w.kb_end + 31) / 32;
+    for (int t = 0; t < NQ; ++t)
+      for (int wi = warp; wi < words; wi += C::THREADS / 32) {
+        const int kb = wi * 32 + lane;
+        const uint32_t word = __ballot_sync(0xffffffffu, kb < w.kb_end && w.act_direct(t, kb));
+        if (lane == 0) bits[t * kWpr + wi] = word;
+      }
+    w.bits = bits;  // read after the __syncthreads below
   }
 
   if (threadIdx.x == 0) {
@@ -627,12 +670,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   }
 }
 
-template <int D, bool DROPOUT>
+template <int D, bool DROPOUT, bool BITS>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, cudaStream_t stream) {
   using L = FwdLayout<D>;
   using C = FwdCfg<D>;
-  auto kern = fwd_kernel<D, DROPOUT>;
+  auto kern = fwd_kernel<D, DROPOUT, BITS>;
   // The setmaxnreg split is sized for exactly LAUNCH_REGS registers per thread
   // at launch; with any other count an increase could wait forever.  Checked,
   // with the shared-memory attribute set, once per device and context.
@@ -653,14 +696,30 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                            stream, tq, tk, tv, p);
 }
 
+// A block mask whose rows fit the bitmask (every CTA's K/V tiles are below nbk)
+template <int D>
+bool uses_bits(const FwdParams& p) {
+  return p.block_mask != nullptr && (p.nbk + 31) / 32 <= FwdLayout<D>::BIT_WORDS / FwdCfg<D>::NQ;
+}
+
 }  // namespace
 
 cudaError_t launch_fwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, cudaStream_t stream) {
-  if (d == 64) return dropout ? launch_fwd_t<64, true>(tq, tk, tv, p, stream)
-                              : launch_fwd_t<64, false>(tq, tk, tv, p, stream);
-  if (d == 128) return dropout ? launch_fwd_t<128, true>(tq, tk, tv, p, stream)
-                               : launch_fwd_t<128, false>(tq, tk, tv, p, stream);
+  if (d == 64) {
+    if (uses_bits<64>(p))
+      return dropout ? launch_fwd_t<64, true, true>(tq, tk, tv, p, stream)
+                     : launch_fwd_t<64, false, true>(tq, tk, tv, p, stream);
+    return dropout ? launch_fwd_t<64, true, false>(tq, tk, tv, p, stream)
+                   : launch_fwd_t<64, false, false>(tq, tk, tv, p, stream);
+  }
+  if (d == 128) {
+    if (uses_bits<128>(p))
+      return dropout ? launch_fwd_t<128, true, true>(tq, tk, tv, p, stream)
+                     : launch_fwd_t<128, false, true>(tq, tk, tv, p, stream);
+    return dropout ? launch_fwd_t<128, true, false>(tq, tk, tv, p, stream)
+                   : launch_fwd_t<128, false, false>(tq, tk, tv, p, stream);
+  }
   return cudaErrorInvalidValue;
 }
 
