@@ -276,16 +276,17 @@ cudaError_t launch_qkv_projection(const void* x, const void* w, const void* bias
   p.status = status;
   p.timeout_ns = timeout_ns;
   static OncePerContext prepared;
-  static int sms = 0;
   cudaError_t e = prepared.run([]() {
-    int dev = 0;
-    cudaError_t r = cudaGetDevice(&dev);
-    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (r != cudaSuccess) return r;
     return cudaFuncSetAttribute(qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(kProjSmem));
   });
   if (e != cudaSuccess) return e;
+  // one CTA per SM of the current device (a cheap, cached attribute query)
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (sms < 1) return cudaErrorInvalidValue;
   const int grid = p.tiles < sms ? p.tiles : sms;
   return launch_overlapped(qkv_proj_kernel, dim3(static_cast<unsigned>(grid)), dim3(kProjThreads),
                            kProjSmem, stream, tx, tw, p);
