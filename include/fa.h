@@ -283,6 +283,14 @@ fa_status_t fa_last_device_status(void* stream);
  * below 1e6 are raised to 1e6.  Applies to launches made after the call. */
 void fa_set_wait_timeout_ns(uint64_t ns);
 
+/* Test support: enabled = 0 makes the kernels of later launches walk a
+ * block mask byte by byte instead of through the per-CTA bitmask they build
+ * in shared memory (the walk a mask too long for the bitmask always takes);
+ * 1, the default, restores the bitmask.  Both visit the same tiles in the
+ * same order, so O, LSE, dK and dV come out identical and dQ equal up to the
+ * order of its fp32 reductions. */
+void fa_debug_set_block_mask_bitmap(int enabled);
+
 /* Test support: writes the dropout keep bits (1 = kept) of every (b,h,i,j)
  * into keep (device uint8 [B,H,N,N]) using the same device generator as the
  * attention kernels. */

@@ -23,7 +23,7 @@ __all__ = [
     "FaError", "library", "forward", "backward", "backward_phases", "bwd_workspace_size",
     "forward_general", "backward_general", "general_workspace_size",
     "merge_partial", "accumulate_bf16", "convert_f32_bf16", "qkv_projection",
-    "dropout_mask", "last_device_status", "set_wait_timeout_ns",
+    "dropout_mask", "last_device_status", "set_wait_timeout_ns", "set_block_mask_bitmap",
     "wait_timeout_probe", "STATUS",
 ]
 
@@ -94,6 +94,7 @@ SIGNATURES = {
     "fa_set_wait_timeout_ns": (None, [_u64]),
     "fa_debug_dropout_mask": (_i, [_vp, _i, _i, _i, _f, _u64, _vp]),
     "fa_debug_wait_timeout": (_i, [_vp]),
+    "fa_debug_set_block_mask_bitmap": (None, [_i]),
 }
 
 
@@ -259,6 +260,11 @@ def last_device_status(device=None):
 
 def set_wait_timeout_ns(ns):
     library().fa_set_wait_timeout_ns(int(ns))
+
+
+def set_block_mask_bitmap(enabled):
+    """Test support: False makes later launches walk block masks byte by byte."""
+    library().fa_debug_set_block_mask_bitmap(1 if enabled else 0)
 
 
 def wait_timeout_probe(device=None):

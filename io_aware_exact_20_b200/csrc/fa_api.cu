@@ -22,6 +22,7 @@ __device__ int g_status_word;
 
 fa::SymbolAddressCache g_status_cache;
 std::atomic<uint64_t> g_timeout_ns{4000000000ull};
+std::atomic<int> g_mask_bitmap{1};
 
 // Device address of the status word in the current device's context.
 int* status_word() {
@@ -277,6 +278,7 @@ fa_status_t run_fwd(const Problem& pr, const void* q, const void* k, const void*
   p.seed_hi = static_cast<uint32_t>(pr.seed >> 32);
   p.rk = fa::philox_round_keys(pr.seed);
   p.timeout_ns = g_timeout_ns.load();
+  p.mask_bitmap = g_mask_bitmap.load();
   const cudaError_t e =
       fa::launch_fwd(pr.D, dr.threshold != 0, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -326,6 +328,7 @@ fa_status_t bwd_params(fa::BwdParams* p, const Problem& pr, const void* workspac
   p->seed_hi = static_cast<uint32_t>(pr.seed >> 32);
   p->rk = fa::philox_round_keys(pr.seed);
   p->timeout_ns = g_timeout_ns.load();
+  p->mask_bitmap = g_mask_bitmap.load();
   return FA_OK;
 }
 
@@ -389,6 +392,8 @@ const char* fa_status_string(fa_status_t s) {
 }
 
 void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns < 1000000ull ? 1000000ull : ns); }
+
+void fa_debug_set_block_mask_bitmap(int enabled) { g_mask_bitmap.store(enabled != 0 ? 1 : 0); }
 
 fa_status_t fa_last_device_status(void* stream) {
   int* w = status_word();

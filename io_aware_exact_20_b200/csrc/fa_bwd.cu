@@ -981,7 +981,7 @@ cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CU
   if (d == 64) {
     // a block mask whose columns fit the bitmask (the CTAs' query tiles are
     // below the longest sequence's)
-    const bool bits = p.block_mask != nullptr &&
+    const bool bits = p.block_mask != nullptr && p.mask_bitmap != 0 &&
                       ((p.rows.nq + 127) / 128 + 31) / 32 <= BwdLayout<64>::BIT_WORDS;
     if (bits)
       return dropout ? launch_main_t<64, true, true>(tq, tk, tv, tdo, tdq, p, stream)

@@ -699,7 +699,8 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 // A block mask whose rows fit the bitmask (every CTA's K/V tiles are below nbk)
 template <int D>
 bool uses_bits(const FwdParams& p) {
-  return p.block_mask != nullptr && (p.nbk + 31) / 32 <= FwdLayout<D>::BIT_WORDS / FwdCfg<D>::NQ;
+  return p.block_mask != nullptr && p.mask_bitmap != 0 &&
+         (p.nbk + 31) / 32 <= FwdLayout<D>::BIT_WORDS / FwdCfg<D>::NQ;
 }
 
 }  // namespace

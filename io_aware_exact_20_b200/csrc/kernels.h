@@ -141,6 +141,7 @@ struct FwdParams {
   uint32_t seed_lo, seed_hi;
   PhiloxRoundKeys rk;         // round keys of the dropout generator
   uint64_t timeout_ns;
+  int mask_bitmap;            // block masks: 1 = walk them through a shared-memory bitmask
 };
 
 struct BwdParams {
@@ -177,6 +178,7 @@ struct BwdParams {
   uint32_t seed_lo, seed_hi;
   PhiloxRoundKeys rk;
   uint64_t timeout_ns;
+  int mask_bitmap;            // as in FwdParams
 };
 
 // First workspace row of (b, h); a multiple of 128.  Packed sequences are
