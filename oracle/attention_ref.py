@@ -105,23 +105,28 @@ def dropout_scale(p):
     return 65536.0 / (65536.0 - t)
 
 
-def dropout_keep(seed, p, b, h, rows, n):
-    """Keep bits Z[i, j] (bool) for query rows ``rows`` and keys 0..n-1."""
+def dropout_keep(seed, p, b, h, rows, n, key0=0):
+    """Keep bits Z[i, j] (bool) for query rows ``rows`` and keys key0..key0+n-1
+    (rows and keys are positions in the whole sequence: the bits are keyed by
+    them, whatever slice of the problem a caller evaluates)."""
     t = dropout_threshold(p)
     if t == 0:
         return np.ones((len(rows), n), dtype=bool)
     seed = int(seed) & 0xFFFFFFFFFFFFFFFF
     k0, k1 = seed & 0xFFFFFFFF, seed >> 32
     rows = np.asarray(rows, dtype=np.uint64)[:, None]
-    groups = np.arange((n + 7) // 8, dtype=np.uint64)[None, :]
+    g_first = key0 // 8
+    g_last = (key0 + n + 7) // 8  # one past the last block
+    groups = np.arange(g_first, g_last, dtype=np.uint64)[None, :]
     words = philox4x32_10(groups, rows, np.uint64(h), np.uint64(b), k0, k1)
     # key 8 g + 2 m + s takes half s of word m of block g
     halves = []
     for w in words:
         halves.append(w & np.uint32(0xFFFF))
         halves.append(w >> np.uint32(16))
-    u = np.stack(halves, axis=-1).reshape(len(rows), -1)[:, :n]
-    return u >= np.uint32(t)
+    u = np.stack(halves, axis=-1).reshape(len(rows), -1)
+    start = key0 - 8 * g_first
+    return u[:, start:start + n] >= np.uint32(t)
 
 
 # ----------------------------------------------------------------------------
@@ -273,31 +278,35 @@ def _row_terms(q, k, v, dout, scale, rows, causal, kv_len, block_mask, keep, dro
 
 
 def head_forward_rows(q, k, v, scale, rows, causal=False, kv_len=None, block_mask=None,
-                      dropout_p=0.0, seed=0, b=0, h=0):
-    """O and LSE of the given query rows of one (b, h) (q, k, v: [N, d])."""
+                      dropout_p=0.0, seed=0, b=0, h=0, row0=0, key0=0):
+    """O and LSE of the given query rows of one (b, h) (q, k, v: [N, d]).
+    row0 / key0: sequence positions of q's and k's first rows, where q, k, v
+    are a slice of a larger problem (they place the dropout bits only)."""
     rows = np.asarray(rows, dtype=np.int64)
     p32 = float(np.float32(dropout_p))
     keep, rscale = None, 1.0
     if p32 > 0:
-        keep = dropout_keep(seed, p32, b, h, rows, k.shape[0])
+        keep = dropout_keep(seed, p32, b, h, rows + row0, k.shape[0], key0)
         rscale = dropout_scale(p32)
     return _head_forward(q, k, v, scale, rows, causal, kv_len, block_mask, keep, rscale)
 
 
 def head_backward_rows(q, k, v, dout, scale, rows, causal=False, kv_len=None,
-                       block_mask=None, dropout_p=0.0, seed=0, b=0, h=0):
-    """dQ of the given query rows of one (b, h): scale * dS[rows] K."""
+                       block_mask=None, dropout_p=0.0, seed=0, b=0, h=0, row0=0, key0=0):
+    """dQ of the given query rows of one (b, h): scale * dS[rows] K (row0 /
+    key0 as in head_forward_rows)."""
     rows = np.asarray(rows, dtype=np.int64)
     p32 = float(np.float32(dropout_p))
-    keep = dropout_keep(seed, p32, b, h, rows, k.shape[0]) if p32 > 0 else None
+    keep = dropout_keep(seed, p32, b, h, rows + row0, k.shape[0], key0) if p32 > 0 else None
     _, ds = _row_terms(q, k, v, dout, scale, rows, causal, kv_len, block_mask, keep, p32)
     return scale * (ds @ k)
 
 
 def head_backward_cols(q, k, v, dout, scale, cols, causal=False, kv_len=None,
                        block_mask=None, dropout_p=0.0, seed=0, b=0, h=0, slab=256,
-                       rows=None):
-    """dK and dV of the given key columns of one (b, h).
+                       rows=None, row0=0, key0=0):
+    """dK and dV of the given key columns of one (b, h) (row0 / key0 as in
+    head_forward_rows).
 
     Both are sums over query rows (dV_j = sum_i Pdrop_ij dO_i,
     dK_j = scale sum_i dS_ij Q_i); the rows are visited in slabs of ``slab``
@@ -313,7 +322,7 @@ def head_backward_cols(q, k, v, dout, scale, cols, causal=False, kv_len=None,
     all_rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
     for r0 in range(0, all_rows.size, slab):
         rows = all_rows[r0:r0 + slab]
-        keep = dropout_keep(seed, p32, b, h, rows, n) if p32 > 0 else None
+        keep = dropout_keep(seed, p32, b, h, rows + row0, n, key0) if p32 > 0 else None
         pd, ds = _row_terms(q, k, v, dout, scale, rows, causal, kv_len, block_mask, keep, p32)
         dv += pd[:, cols].T @ dout[rows]
         dk += scale * (ds[:, cols].T @ q[rows])

@@ -870,3 +870,50 @@ def test_qkv_projection_matches_torch_linear():
         assert np.abs(got - ref[i].numpy()).max() < 1e-12
     q0, _, _ = qkv_projection(x, w, None, B, H, d)
     assert np.abs(q0 - (q - bias[:H * d].reshape(1, H, 1, d))).max() < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# sequence offsets of a slice (dropout bits keyed by the absolute (i, j))
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("key0", [0, 5, 13, 256, 4001])
+def test_dropout_keep_with_key_offset_is_the_slice_of_the_whole_row(key0):
+    """Keys key0 .. key0 + n - 1 take the bits those keys have in the whole
+    row, for block-aligned and unaligned offsets alike."""
+    from oracle import dropout_keep
+    rows = np.array([0, 7, 1000, 123457])
+    n = 37
+    whole = dropout_keep(99, 0.3, 2, 5, rows, key0 + n)
+    assert np.array_equal(dropout_keep(99, 0.3, 2, 5, rows, n, key0=key0), whole[:, key0:])
+
+
+def test_row_and_column_helpers_on_a_diagonal_slice_match_the_whole_problem():
+    """Under a block mask that keeps only the diagonal 128 x 128 blocks, a
+    query tile sees only its own key tile: the helpers on that slice, told its
+    sequence offsets, give the whole problem's rows and columns (dropout on)."""
+    from oracle.attention_ref import head_backward_cols, head_backward_rows, head_forward_rows
+    rng = np.random.default_rng(4)
+    N, d, t = 384, 16, 2
+    q, k, v, do = (rng.standard_normal((N, d)) for _ in range(4))
+    bm = np.eye(N // 128, dtype=np.uint8)
+    kw = dict(dropout_p=0.2, seed=17, b=1, h=3)
+    rows = np.array([0, 5, 127])
+    sl = slice(128 * t, 128 * t + 128)
+    full_o, full_l = head_forward_rows(q, k, v, 0.25, rows + 128 * t, block_mask=bm, **kw)
+    part_o, part_l = head_forward_rows(q[sl], k[sl], v[sl], 0.25, rows, row0=128 * t,
+                                       key0=128 * t, **kw)
+    assert np.allclose(full_o, part_o, rtol=0, atol=1e-12)
+    assert np.allclose(full_l, part_l, rtol=0, atol=1e-12)
+    full_dq = head_backward_rows(q, k, v, do, 0.25, rows + 128 * t, block_mask=bm, **kw)
+    part_dq = head_backward_rows(q[sl], k[sl], v[sl], do[sl], 0.25, rows, row0=128 * t,
+                                 key0=128 * t, **kw)
+    assert np.allclose(full_dq, part_dq, rtol=0, atol=1e-12)
+    cols = np.array([1, 64, 126])
+    full_dk, full_dv = head_backward_cols(q, k, v, do, 0.25, cols + 128 * t, block_mask=bm, **kw)
+    part_dk, part_dv = head_backward_cols(q[sl], k[sl], v[sl], do[sl], 0.25, cols,
+                                          row0=128 * t, key0=128 * t, **kw)
+    assert np.allclose(full_dk, part_dk, rtol=0, atol=1e-12)
+    assert np.allclose(full_dv, part_dv, rtol=0, atol=1e-12)
+    # the offsets matter: without them the dropout bits are another draw
+    wrong_o, _ = head_forward_rows(q[sl], k[sl], v[sl], 0.25, rows, **kw)
+    assert not np.allclose(full_o, wrong_o, rtol=0, atol=1e-6)
