@@ -42,7 +42,7 @@ def run_case(fa, B, H, N, d, causal=False, lens=None, density=None, p=0.0, seed=
 
 
 def compare(o, lse, ro, rl, record=None):
-    """Checks O and LSE against the oracle.  The strict the benchmark spec bound
+    """Checks O and LSE against the oracle.  The strict bound on O
     (max-abs 1e-2) is asserted wherever bf16 storage can meet it (|O_ref| < 2,
     half an ulp <= 2^-8 |O| < 0.0079); everywhere the bound is
     1e-2 + 2^-8 |O_ref|.  The strict max-abs error over all elements is
