@@ -29,7 +29,10 @@
  *  - LSE is fp32 [B, H, N], natural logarithm; a row with no valid key has
  *    LSE = -inf and O = 0.
  *  - d is 32, 64, 96 or 128 (32 and 96 run the 64- and 128-wide kernels on
- *    zero-filled columns).  1 <= N <= 2^23; B * H <= 65535 and
+ *    zero-filled columns); the forward also takes 192 and 256 (a 256-wide
+ *    kernel; the backward entry points return FA_ERR_UNSUPPORTED for them,
+ *    since a 128-key tile's dK and dV accumulators would fill the tensor
+ *    memory the backward also needs for S and dP).  1 <= N <= 2^23; B * H <= 65535 and
  *    B * H * ceil(N / 128) <= 2^31 - 1 (one thread block per head and
  *    128-row tile); larger requests return FA_ERR_UNSUPPORTED.
  *  - softmax_scale multiplies Q K^T before masking (typically 1/sqrt(d)).
@@ -162,7 +165,8 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
  * lengths (researchpapers.dev "FlashAttention 详解", section 关键结果); the
  * entry points below take them packed, with no padding rows, as well as
  * token-major ([B, N, H, d]) or any other strided layout whose d is
- * contiguous, different query and key counts, and head dims 32, 64, 96, 128.
+ * contiguous, different query and key counts, and head dims 32, 64, 96, 128
+ * (192 and 256: forward only).
  * The computation is the one above, per batch entry (or packed sequence) b:
  *  - positions i, j are counted inside sequence b (masks, dropout counter);
  *  - causal: query i attends key j iff j <= i + Nk_b - Nq_b, Nq_b / Nk_b the
@@ -182,7 +186,7 @@ typedef struct {
 typedef struct {
   int batch;     /* B: batch entries (padded layout) or packed sequences */
   int heads;     /* H */
-  int head_dim;  /* d: 32, 64, 96 or 128 */
+  int head_dim;  /* d: 32, 64, 96 or 128; 192 or 256 for the forward only */
   /* Padded layout: rows of every batch entry (queries, keys).  Packed layout:
    * an upper bound of every sequence's query / key count (longer sequences
    * are cut to it). */

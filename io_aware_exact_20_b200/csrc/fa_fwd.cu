@@ -59,14 +59,23 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 //            warpgroups per SM either way, but each CTA walks only the K/V
 //            tiles its own Q tile needs (which matters under block masks) and
 //            one CTA's set-up and epilogue hide under the other's main loop.
+//   d = 256 (WIDE, also d = 192 with zero columns): one Q tile per CTA and
+//            one softmax stream; S (128 columns) and O (256) take 384 TMEM
+//            columns and a 64 KB Q tile plus one 128 KB K/V stage most of the
+//            shared memory, so K and V are released separately (K once its S
+//            MMA is done, V once its PV MMA is done) and the next tile's K
+//            loads while this tile's softmax runs.  No register split: the
+//            256 threads can hold 255 registers each.
 template <int D>
 struct FwdCfg {
-  static constexpr int NQ = D == 64 ? 1 : 2;  // Q tiles per CTA
-  static constexpr int KS = D == 64 ? 2 : 1;  // softmax streams per Q tile
-  static constexpr int NS = NQ * KS;          // softmax streams = softmax warpgroups
-  static constexpr int KW = 128 / KS;         // keys per stream per K/V tile
+  static constexpr bool WIDE = D == 256;
+  static constexpr int NQ = D == 128 ? 2 : 1;  // Q tiles per CTA
+  static constexpr int KS = D == 64 ? 2 : 1;   // softmax streams per Q tile
+  static constexpr int NS = NQ * KS;           // softmax streams = softmax warpgroups
+  static constexpr int KW = 128 / KS;          // keys per stream per K/V tile
   static constexpr int THREADS = 128 * (1 + NS);
-  static constexpr int MIN_BLOCKS = NQ == 2 ? 1 : 2;
+  static constexpr int MIN_BLOCKS = D == 64 ? 2 : 1;
+  static constexpr bool SPLIT_REGS = !WIDE;
   // registers per thread at launch (checked before the first launch): the
   // largest multiple of 8 that MIN_BLOCKS CTAs of THREADS threads can hold
   static constexpr int LAUNCH_REGS = (65536 / (THREADS * MIN_BLOCKS)) & ~7;
@@ -74,11 +83,12 @@ struct FwdCfg {
   // softmax warpgroups, within the THREADS x LAUNCH_REGS of the launch
   static constexpr uint32_t REGS_CTL = KS == 1 ? 72 : 32;
   static constexpr uint32_t REGS_SOFTMAX =
-      ((THREADS * LAUNCH_REGS - 128 * REGS_CTL) / (128 * NS)) & ~7u;
+      SPLIT_REGS ? ((THREADS * LAUNCH_REGS - 128 * REGS_CTL) / (128 * NS)) & ~7u : 248u;
   static constexpr int MAX_PARTS = KW == 128 ? 8 : 4;  // max / sum chains per row
-  static_assert(128 * (REGS_CTL + NS * REGS_SOFTMAX) <= THREADS * LAUNCH_REGS,
+  static_assert(!SPLIT_REGS || 128 * (REGS_CTL + NS * REGS_SOFTMAX) <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
-  static_assert(REGS_SOFTMAX <= 256 && REGS_SOFTMAX >= 96, "softmax register budget");
+  static_assert(!SPLIT_REGS || (REGS_SOFTMAX <= 256 && REGS_SOFTMAX >= 96),
+                "softmax register budget");
 };
 
 template <int D>
@@ -88,7 +98,9 @@ struct FwdLayout {
   static constexpr int PANELS = D / 64;                 // 64-column, 128-byte-swizzled panels
   static constexpr uint32_t PANEL = 128u * 128u;        // bytes of one [128 rows][64 cols] panel
   static constexpr uint32_t TILE = PANEL * PANELS;      // bytes of one 128-row tile
-  static constexpr int STAGES = 2;                      // K/V ring depth
+  static constexpr int STAGES = C::WIDE ? 1 : 2;        // K/V ring depth
+  // K and V of a stage released by separate barriers (else one, after PV)
+  static constexpr bool SPLIT_RELEASE = C::WIDE;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_KV = NQ * TILE;
   static constexpr uint32_t OFF_XCH = OFF_KV + STAGES * 2 * TILE;  // [NS][128] (m, l) for the merge
@@ -96,8 +108,9 @@ struct FwdLayout {
   static constexpr int B_QFULL = 0;
   static constexpr int B_KFULL = 2;
   static constexpr int B_VFULL = B_KFULL + STAGES;
-  static constexpr int B_KVEMPTY = B_VFULL + STAGES;
-  static constexpr int B_SFULL = B_KVEMPTY + STAGES;  // per stream
+  static constexpr int B_KVEMPTY = B_VFULL + STAGES;  // with SPLIT_RELEASE: K released
+  static constexpr int B_VEMPTY = B_KVEMPTY + STAGES;  // with SPLIT_RELEASE: V released
+  static constexpr int B_SFULL = B_KVEMPTY + STAGES * (SPLIT_RELEASE ? 2 : 1);  // per stream
   static constexpr int B_PFULL = B_SFULL + C::NS;     // per stream
   static constexpr int B_ODONE = B_PFULL + C::NS;     // per stream
   static constexpr int B_DRAIN = B_ODONE + C::NS;
@@ -108,9 +121,9 @@ struct FwdLayout {
   static constexpr int BIT_WORDS = 1024;
   static constexpr uint32_t OFF_BITS = OFF_MISC + 16;
   static constexpr uint32_t SMEM = OFF_BITS + BIT_WORDS * 4;
-  static constexpr uint32_t TMEM_COLS = NQ == 2 ? 512 : 256;
   static constexpr uint32_t O_COL = C::KW * C::NS;
-  static_assert(SMEM <= (NQ == 2 ? 232448u : 113u * 1024u), "shared memory budget");
+  static constexpr uint32_t TMEM_COLS = O_COL + C::NS * D <= 256 ? 256 : 512;
+  static_assert(SMEM <= (C::MIN_BLOCKS == 1 ? 232448u : 113u * 1024u), "shared memory budget");
   static_assert(O_COL + C::NS * D <= TMEM_COLS, "TMEM budget");
 };
 
@@ -260,6 +273,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       mbar_init(bar(L::B_KFULL + s), 1);
       mbar_init(bar(L::B_VFULL + s), 1);
       mbar_init(bar(L::B_KVEMPTY + s), 1);
+      if constexpr (L::SPLIT_RELEASE) mbar_init(bar(L::B_VEMPTY + s), 1);
     }
     mbar_init(bar(L::B_DRAIN), 1);
     fence_mbar_init();
@@ -276,7 +290,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   // Each role runs inside the branch that sets its register budget, so that
   // the compiler allocates every role's code under its own limit.
   if (warp < 4) {
-  setmaxnreg_dec<C::REGS_CTL>();
+  if constexpr (C::SPLIT_REGS) setmaxnreg_dec<C::REGS_CTL>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
@@ -291,9 +305,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
                       64 * pn, w.qrow + w.q0 + 128 * t, w.h, w.tb);
       }
       int it = 0;
+      bool k_alone = false;  // tile it's K was requested, its V not (a wait gave up)
       for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1), ++it) {
         const int s = it % L::STAGES;
         const uint32_t ph = (it / L::STAGES) & 1u;
+        // the stage's K (SPLIT_RELEASE) or K and V are free again
         if (it >= L::STAGES && !mbar_wait(bar(L::B_KVEMPTY + s), ph ^ 1u, g)) break;
         const uint32_t kdst = sbase + L::OFF_KV + s * 2 * L::TILE;
         const uint32_t vdst = kdst + L::TILE;
@@ -301,6 +317,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         for (int pn = 0; pn < L::PANELS; ++pn)
           tma_load_4d(kdst + pn * L::PANEL, &tm_k, bar(L::B_KFULL + s), 64 * pn, w.krow + kb * 128,
                       w.h, w.tb);
+        if constexpr (L::SPLIT_RELEASE) {
+          if (it >= L::STAGES && !mbar_wait(bar(L::B_VEMPTY + s), ph ^ 1u, g)) {
+            k_alone = true;
+            break;
+          }
+        }
         mbar_arrive_expect_tx(bar(L::B_VFULL + s), L::TILE);
         for (int pn = 0; pn < L::PANELS; ++pn)
           tma_load_4d(vdst + pn * L::PANEL, &tm_v, bar(L::B_VFULL + s), 64 * pn, w.krow + kb * 128,
@@ -313,6 +335,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
           mbar_wait_drain(bar(L::B_KFULL + s), ph, 100000000ull);
           mbar_wait_drain(bar(L::B_VFULL + s), ph, 100000000ull);
         }
+        if (k_alone)
+          mbar_wait_drain(bar(L::B_KFULL + it % L::STAGES), (it / L::STAGES) & 1u, 100000000ull);
         mbar_wait_drain(bar(L::B_QFULL + 0), 0, 100000000ull);
         if (w.exists1) mbar_wait_drain(bar(L::B_QFULL + 1), 0, 100000000ull);
       }
@@ -362,6 +386,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
             issue_s(s, sbase + L::OFF_KV);
           }
         }
+        // SPLIT_RELEASE: the first K tile is free once its S MMAs are done
+        if constexpr (L::SPLIT_RELEASE)
+          if (ok) mma_commit(bar(L::B_KVEMPTY + 0));
       }
       while (ok && kb < w.kb_end) {
         const int st = it % L::STAGES;
@@ -409,7 +436,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
           }
         }
         if (!ok) break;
-        mma_commit(bar(L::B_KVEMPTY + st));
+        if constexpr (L::SPLIT_RELEASE) {
+          // V of this tile once its PV MMAs are done; K of the next tile once
+          // its S MMAs are (both commits track every MMA issued before them)
+          mma_commit(bar(L::B_VEMPTY + st));
+          if (kn_ready) mma_commit(bar(L::B_KVEMPTY + sn));
+        } else {
+          mma_commit(bar(L::B_KVEMPTY + st));
+        }
         kb = kbn;
         ++it;
       }
@@ -422,7 +456,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     }
   }
   } else {
-    setmaxnreg_inc<C::REGS_SOFTMAX>();
+    if constexpr (C::SPLIT_REGS) setmaxnreg_inc<C::REGS_SOFTMAX>();
     // -------------------------------------------------------------- softmax
     const int s = (warp - 4) >> 2;  // stream
     const int t = s / KS;           // Q tile
@@ -681,10 +715,12 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   // with the shared-memory attribute set, once per device and context.
   static OncePerContext prepared;
   cudaError_t e = prepared.run([&]() -> cudaError_t {
-    cudaFuncAttributes attr{};
-    cudaError_t r = cudaFuncGetAttributes(&attr, kern);
-    if (r != cudaSuccess) return r;
-    if (attr.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+    if constexpr (C::SPLIT_REGS) {
+      cudaFuncAttributes attr{};
+      cudaError_t r = cudaFuncGetAttributes(&attr, kern);
+      if (r != cudaSuccess) return r;
+      if (attr.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+    }
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(L::SMEM));
   });
@@ -720,6 +756,13 @@ cudaError_t launch_fwd(int d, bool dropout, const CUtensorMap& tq, const CUtenso
                      : launch_fwd_t<128, false, true>(tq, tk, tv, p, stream);
     return dropout ? launch_fwd_t<128, true, false>(tq, tk, tv, p, stream)
                    : launch_fwd_t<128, false, false>(tq, tk, tv, p, stream);
+  }
+  if (d == 256) {
+    if (uses_bits<256>(p))
+      return dropout ? launch_fwd_t<256, true, true>(tq, tk, tv, p, stream)
+                     : launch_fwd_t<256, false, true>(tq, tk, tv, p, stream);
+    return dropout ? launch_fwd_t<256, true, false>(tq, tk, tv, p, stream)
+                   : launch_fwd_t<256, false, false>(tq, tk, tv, p, stream);
   }
   return cudaErrorInvalidValue;
 }

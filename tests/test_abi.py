@@ -55,7 +55,8 @@ A16 = 1 << 20  # a fake, 16-byte aligned address: validation fails before use
 
 @pytest.mark.parametrize("args,code", [
     (dict(q=0), 1), (dict(k=A16 + 8), 1), (dict(B=0), 1), (dict(N=0), 1),
-    (dict(d=80), 2), (dict(d=256), 2), (dict(scale=0.0), 1), (dict(scale=float("inf")), 1),
+    (dict(d=80), 2), (dict(d=160), 2), (dict(d=512), 2), (dict(scale=0.0), 1),
+    (dict(scale=float("inf")), 1),
     (dict(p=1.0), 1), (dict(p=-0.1), 1), (dict(p=float("nan")), 1),
     (dict(B=300, H=300), 2), (dict(lse=A16 + 2), 1),
     (dict(N=(1 << 23) + 1), 2),                       # N beyond 2^23
@@ -108,7 +109,7 @@ def _desc(lib, **kw):
 
 @pytest.mark.parametrize("change,code", [
     (dict(), None),                                        # valid: workspace size > 0
-    (dict(head_dim=80), 2), (dict(head_dim=256), 2),
+    (dict(head_dim=80), 2), (dict(head_dim=160), 2), (dict(head_dim=512), 2),
     (dict(batch=0), 1), (dict(seqlen_k=0), 1), (dict(dropout_p=1.0), 1),
     (dict(cu_seqlens_q=A16), 1),                           # packed needs both offsets
     (dict(cu_seqlens_q=A16, cu_seqlens_k=A16), 1),          # ... and total_q, total_k >= 1
@@ -168,3 +169,18 @@ def test_general_binding_rejects_host_tensors_and_bad_layouts(lib):
         lib.forward_general(q, q, q, layout="thd")
     with pytest.raises(ValueError, match="device of q"):
         lib.backward_general(q, q, q, q, torch.zeros((1, 2, 128)), q)
+
+
+@pytest.mark.parametrize("d", [192, 256])
+def test_backward_refuses_the_forward_only_head_dims(lib, d):
+    """d = 192 / 256 run the forward only: every backward entry point returns
+    FA_ERR_UNSUPPORTED before any launch and the workspace size is 0.  (No
+    forward call here: with d = 256 the forward is valid and would launch.)"""
+    so = lib.library()
+    assert so.fa_bwd_workspace_size(1, 2, 256, d) == 0
+    a = _desc(lib, head_dim=d)
+    assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == 0
+    assert so.fa_bwd_ex(ctypes.byref(a), A16, A16, A16, A16, A16, A16, A16, A16, A16, A16,
+                        1 << 30, None) == 2
+    assert so.fa_bwd(A16, A16, A16, A16, A16, A16, A16, A16, A16, 1, 2, 256, d, 0.1, 0, None,
+                     0.0, 0, None, A16, 1 << 30, None) == 2
