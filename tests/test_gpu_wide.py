@@ -87,3 +87,25 @@ def test_wide_backward_is_refused(lib):
         lib.backward(q, k, v, o, lse, do)
     torch.cuda.synchronize()
     assert lib.last_device_status() == 0
+
+
+def test_wide_forward_bitmask_walk_equals_byte_walk(lib):
+    """The 256-wide forward walks a block mask through its shared-memory
+    bitmask or byte by byte (test-support switch) with identical O and LSE."""
+    import torch
+    from io_aware_exact_20_b200.workloads import make_block_mask
+    q, k, v, _ = (x.cuda() for x in make_qkvdo(1, 2, 1100, 256, 12))
+    bm = make_block_mask(1100, 0.4, 13)
+    bm[4, :] = 0
+    out = []
+    for bitmap in (True, False):
+        lib.set_block_mask_bitmap(bitmap)
+        try:
+            o, lse = lib.forward(q, k, v, causal=True, dropout_p=0.1, seed=2, block_mask=bm)
+            torch.cuda.synchronize()
+            assert lib.last_device_status() == 0
+        finally:
+            lib.set_block_mask_bitmap(True)
+        out.append((o.float().cpu().numpy(), lse.cpu().numpy()))
+    assert np.array_equal(out[0][0], out[1][0])
+    assert np.array_equal(out[0][1], out[1][1])
