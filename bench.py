@@ -870,9 +870,10 @@ def time_e2e(case, fa, args, dev, world, flops):
     from pinned host memory and every output copied back, inside the timed
     region, as a user streaming batches would run it: two device buffer sets
     alternate, so that one step's Q, K, V, dO travel in (host-to-device copy
-    engine) while the step before computes and the one before that has its O,
-    LSE, dQ, dK, dV copied out (device-to-host engine).  Events order each
-    buffer's reuse.  One region over all steps is timed, from before the first
+    engine) while the step before computes and has its O, LSE, dQ, dK, dV
+    copied out (device-to-host engine).  Events order each buffer's reuse:
+    its inputs are rewritten once the backward that read them has run, its
+    outputs once the copies that read them are done.  One region over all steps is timed, from before the first
     copy in to after the last copy out; no L2 flush, since every step's inputs
     arrive from the host."""
     import torch
@@ -895,13 +896,17 @@ def time_e2e(case, fa, args, dev, world, flops):
         j = i % 2
         with torch.cuda.stream(s_in):
             if used[j]:
-                s_in.wait_event(out_done[j])  # the buffer's last step is on the host
+                # the buffer's inputs are free once its last step's backward ran
+                s_in.wait_event(bwd_done[j])
             b["q"].copy_(hq, non_blocking=True)
             b["k"].copy_(hk, non_blocking=True)
             b["v"].copy_(hv, non_blocking=True)
             b["do"].copy_(hdo, non_blocking=True)
             in_done[j].record(s_in)
         s_comp.wait_event(in_done[j])
+        if used[j]:
+            # its outputs are free once its last step's results are on the host
+            s_comp.wait_event(out_done[j])
         fa.forward(b["q"], b["k"], b["v"], out=b["o"], lse=b["lse"], **case.fkw)
         fwd_done[j].record(s_comp)
         fa.backward(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], workspace=case.ws,
@@ -933,6 +938,9 @@ def time_e2e(case, fa, args, dev, world, flops):
         dist.barrier()
     e_ms = max_over_ranks(start.elapsed_time(end), world, dev)
     nb = case.q.numel() * case.q.element_size()
+    # the pipelined steps must give the resident steps' results: dK and dV
+    # are deterministic, so the last step's copies equal them bit for bit
+    same = bool(torch.equal(hdk, case.dk.cpu()) and torch.equal(hdv, case.dv.cpu()))
     del bufs
     return {"value": job_throughput(world, flops, n_e2e, e_ms), "unit": UNIT,
             "h2d_bytes_per_step": 4 * nb,
@@ -940,7 +948,8 @@ def time_e2e(case, fa, args, dev, world, flops):
             "steps": n_e2e, "ms_per_step": e_ms / n_e2e,
             "schedule": "two device buffer sets; copies in, compute and copies out of "
                         "consecutive steps overlap; every step copies all inputs in and "
-                        "all outputs out"}
+                        "all outputs out",
+            "dk_dv_equal_resident_step": same}
 
 
 def measure_config(fa, w, args, rank, dev, flush, stream, world, local, peak):
