@@ -50,3 +50,37 @@ def test_bitmask_walk_equals_byte_walk(lib, B, H, N, d, causal, lens, density, p
         assert np.array_equal(a, b, equal_nan=True)
     scale = np.abs(dq1).max() + 1e-30
     assert np.abs(dq1 - dq2).max() <= 1e-2 * scale
+
+
+def test_bitmask_walk_equals_byte_walk_packed(lib):
+    """The same for a packed variable-length batch (the mask indexed by tile
+    positions inside each sequence, N_q != N_k, causal, dropout, d = 64)."""
+    import torch
+    lq, lk = [300, 1, 700, 129], [500, 40, 650, 129]
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    g = torch.Generator().manual_seed(21)
+    H, d = 2, 64
+    q, do = (torch.randn(int(cu_q[-1]), H, d, generator=g).to(torch.bfloat16).cuda()
+             for _ in range(2))
+    k, v = (torch.randn(int(cu_k[-1]), H, d, generator=g).to(torch.bfloat16).cuda()
+            for _ in range(2))
+    bm = make_block_mask(700, 0.5, 22)[:, :6]
+    bm[2, :] = 0
+    kw = dict(layout="thd", cu_seqlens_q=cu_q, cu_seqlens_k=cu_k, max_seqlen_q=700,
+              max_seqlen_k=650, causal=True, dropout_p=0.1, seed=5, block_mask=bm)
+    out = []
+    for bitmap in (True, False):
+        lib.set_block_mask_bitmap(bitmap)
+        try:
+            o, lse = lib.forward_general(q, k, v, **kw)
+            dq, dk, dv = lib.backward_general(q, k, v, o, lse, do, **kw)
+            torch.cuda.synchronize()
+            assert lib.last_device_status() == 0
+        finally:
+            lib.set_block_mask_bitmap(True)
+        out.append([x.float().cpu().numpy() for x in (o, lse, dq, dk, dv)])
+    (o1, l1, dq1, dk1, dv1), (o2, l2, dq2, dk2, dv2) = out
+    for a, b in ((o1, o2), (l1, l2), (dk1, dk2), (dv1, dv2)):
+        assert np.array_equal(a, b, equal_nan=True)
+    assert np.abs(dq1 - dq2).max() <= 1e-2 * (np.abs(dq1).max() + 1e-30)
