@@ -110,8 +110,12 @@ struct FwdLayout {
   static constexpr int B_VFULL = B_KFULL + STAGES;
   static constexpr int B_KVEMPTY = B_VFULL + STAGES;  // with SPLIT_RELEASE: K released
   static constexpr int B_VEMPTY = B_KVEMPTY + STAGES;  // with SPLIT_RELEASE: V released
-  static constexpr int B_SFULL = B_KVEMPTY + STAGES * (SPLIT_RELEASE ? 2 : 1);  // per stream
-  static constexpr int B_PFULL = B_SFULL + C::NS;     // per stream
+  // S / P buffers per stream: two in the WIDE kernel, so that the next tile's
+  // S is computed while this tile's softmax runs (its TMEM has room: 2 x 128
+  // S columns + 256 O columns)
+  static constexpr int S_BUFS = C::WIDE ? 2 : 1;
+  static constexpr int B_SFULL = B_KVEMPTY + STAGES * (SPLIT_RELEASE ? 2 : 1);  // per stream, buffer
+  static constexpr int B_PFULL = B_SFULL + C::NS * S_BUFS;  // per stream
   static constexpr int B_ODONE = B_PFULL + C::NS;     // per stream
   static constexpr int B_DRAIN = B_ODONE + C::NS;
   static constexpr int NBAR = B_DRAIN + 1;
@@ -121,7 +125,7 @@ struct FwdLayout {
   static constexpr int BIT_WORDS = 1024;
   static constexpr uint32_t OFF_BITS = OFF_MISC + 16;
   static constexpr uint32_t SMEM = OFF_BITS + BIT_WORDS * 4;
-  static constexpr uint32_t O_COL = C::KW * C::NS;
+  static constexpr uint32_t O_COL = C::KW * C::NS * S_BUFS;
   static constexpr uint32_t TMEM_COLS = O_COL + C::NS * D <= 256 ? 256 : 512;
   static_assert(SMEM <= (C::MIN_BLOCKS == 1 ? 232448u : 113u * 1024u), "shared memory budget");
   static_assert(O_COL + C::NS * D <= TMEM_COLS, "TMEM budget");
@@ -264,8 +268,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   if (threadIdx.x == 0) {
     *abort_flag = 0u;
     for (int t = 0; t < 2; ++t) mbar_init(bar(L::B_QFULL + t), 1);
+    for (int s = 0; s < NS * L::S_BUFS; ++s) mbar_init(bar(L::B_SFULL + s), 1);
     for (int s = 0; s < NS; ++s) {
-      mbar_init(bar(L::B_SFULL + s), 1);
       mbar_init(bar(L::B_PFULL + s), 4);  // one arrival per softmax warp
       mbar_init(bar(L::B_ODONE + s), 1);
     }
@@ -305,11 +309,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
                       64 * pn, w.qrow + w.q0 + 128 * t, w.h, w.tb);
       }
       int it = 0;
-      bool k_alone = false;  // tile it's K was requested, its V not (a wait gave up)
       for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1), ++it) {
         const int s = it % L::STAGES;
         const uint32_t ph = (it / L::STAGES) & 1u;
-        // the stage's K (SPLIT_RELEASE) or K and V are free again
+        // the stage's K (SPLIT_RELEASE: V has its own producer) or K and V
+        // are free again
         if (it >= L::STAGES && !mbar_wait(bar(L::B_KVEMPTY + s), ph ^ 1u, g)) break;
         const uint32_t kdst = sbase + L::OFF_KV + s * 2 * L::TILE;
         const uint32_t vdst = kdst + L::TILE;
@@ -317,28 +321,44 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         for (int pn = 0; pn < L::PANELS; ++pn)
           tma_load_4d(kdst + pn * L::PANEL, &tm_k, bar(L::B_KFULL + s), 64 * pn, w.krow + kb * 128,
                       w.h, w.tb);
-        if constexpr (L::SPLIT_RELEASE) {
-          if (it >= L::STAGES && !mbar_wait(bar(L::B_VEMPTY + s), ph ^ 1u, g)) {
-            k_alone = true;
-            break;
-          }
+        if constexpr (!L::SPLIT_RELEASE) {
+          mbar_arrive_expect_tx(bar(L::B_VFULL + s), L::TILE);
+          for (int pn = 0; pn < L::PANELS; ++pn)
+            tma_load_4d(vdst + pn * L::PANEL, &tm_v, bar(L::B_VFULL + s), 64 * pn,
+                        w.krow + kb * 128, w.h, w.tb);
         }
-        mbar_arrive_expect_tx(bar(L::B_VFULL + s), L::TILE);
-        for (int pn = 0; pn < L::PANELS; ++pn)
-          tma_load_4d(vdst + pn * L::PANEL, &tm_v, bar(L::B_VFULL + s), 64 * pn, w.krow + kb * 128,
-                      w.h, w.tb);
       }
       if (*abort_flag) {  // let the copies already issued land before the CTA exits
         for (int j = max(0, it - L::STAGES); j < it; ++j) {
           const int s = j % L::STAGES;
           const uint32_t ph = (j / L::STAGES) & 1u;
           mbar_wait_drain(bar(L::B_KFULL + s), ph, 100000000ull);
-          mbar_wait_drain(bar(L::B_VFULL + s), ph, 100000000ull);
+          if constexpr (!L::SPLIT_RELEASE) mbar_wait_drain(bar(L::B_VFULL + s), ph, 100000000ull);
         }
-        if (k_alone)
-          mbar_wait_drain(bar(L::B_KFULL + it % L::STAGES), (it / L::STAGES) & 1u, 100000000ull);
         mbar_wait_drain(bar(L::B_QFULL + 0), 0, 100000000ull);
         if (w.exists1) mbar_wait_drain(bar(L::B_QFULL + 1), 0, 100000000ull);
+      }
+    }
+  } else if (L::SPLIT_RELEASE && warp == 2) {
+    // ------------------------------------------------------------ TMA of V
+    // (SPLIT_RELEASE: V tiles have their own producer, so that the next K
+    // never waits behind a V that waits for its PV)
+    if (lane == 0) {
+      tma_prefetch_map(&tm_v);
+      int it = 0;
+      for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1), ++it) {
+        const int s = it % L::STAGES;
+        const uint32_t ph = (it / L::STAGES) & 1u;
+        if (it >= L::STAGES && !mbar_wait(bar(L::B_VEMPTY + s), ph ^ 1u, g)) break;
+        const uint32_t vdst = sbase + L::OFF_KV + s * 2 * L::TILE + L::TILE;
+        mbar_arrive_expect_tx(bar(L::B_VFULL + s), L::TILE);
+        for (int pn = 0; pn < L::PANELS; ++pn)
+          tma_load_4d(vdst + pn * L::PANEL, &tm_v, bar(L::B_VFULL + s), 64 * pn, w.krow + kb * 128,
+                      w.h, w.tb);
+      }
+      if (*abort_flag) {
+        for (int j = max(0, it - L::STAGES); j < it; ++j)
+          mbar_wait_drain(bar(L::B_VFULL + j % L::STAGES), (j / L::STAGES) & 1u, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -373,79 +393,125 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         return true;
       };
 
-      int kb = w.next(0);
-      int it = 0;
-      if (kb < w.kb_end) {
-        ok = mbar_wait(bar(L::B_KFULL + 0), 0, g);
-#pragma unroll(kUnrollS)
-        for (int s = 0; s < NS; ++s) {
-          if (!ok || !w.act_s(s / KS, s % KS, KW, kb)) continue;
-          ok = ensure_q(s / KS);
+      if constexpr (L::S_BUFS == 2) {
+        // One stream, two S / P buffers: tile n's S goes to buffer n & 1, and
+        // S of the tile after next is issued right behind this tile's PV into
+        // the buffer that PV has just read, so the tensor pipe computes it
+        // while the softmax works on the next tile.  One K / V stage: tile n's
+        // K and V are the n-th fills of their barriers (parity n & 1).
+        const uint32_t kaddr = sbase + L::OFF_KV, vaddr = kaddr + L::TILE;
+        auto issue_s_buf = [&](uint32_t buf) {
+          const uint32_t qaddr = sbase + L::OFF_Q;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::PANEL + (kk & 3) * 32;
+            mma_ss(tmem + KW * buf, sdesc_sw128(qaddr + off, 16, 1024),
+                   sdesc_sw128(kaddr + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::B_SFULL + buf));
+          mma_commit(bar(L::B_KVEMPTY));  // the K tile is free once its S is done
+        };
+        int kb = w.next(0);
+        int kb1 = kb < w.kb_end ? w.next(kb + 1) : w.kb_end;
+        if (kb < w.kb_end) {
+          ok = mbar_wait(bar(L::B_KFULL), 0, g) && ensure_q(0);
           if (ok) {
             tc_fence_after();
-            issue_s(s, sbase + L::OFF_KV);
+            issue_s_buf(0);
           }
         }
-        // SPLIT_RELEASE: the first K tile is free once its S MMAs are done
-        if constexpr (L::SPLIT_RELEASE)
-          if (ok) mma_commit(bar(L::B_KVEMPTY + 0));
-      }
-      while (ok && kb < w.kb_end) {
-        const int st = it % L::STAGES;
-        const uint32_t ph = (it / L::STAGES) & 1u;
-        const int kbn = w.next(kb + 1);
-        const int sn = (it + 1) % L::STAGES;
-        const uint32_t phn = ((it + 1) / L::STAGES) & 1u;
-        bool kn_ready = false;
-        if (!mbar_wait(bar(L::B_VFULL + st), ph, g)) break;
-        const uint32_t vaddr = sbase + L::OFF_KV + st * 2 * L::TILE + L::TILE;
-#pragma unroll(kUnrollS)
-        for (int s = 0; s < NS; ++s) {
-          if (!ok) break;
-          if (w.act_s(s / KS, s % KS, KW, kb)) {
-            if (!mbar_wait(bar(L::B_PFULL + s), (p_par >> s) & 1u, g)) {
-              ok = false;
-              break;
-            }
-            p_par ^= 1u << s;
+        if (ok && kb1 < w.kb_end) {
+          ok = mbar_wait(bar(L::B_KFULL), 1, g);
+          if (ok) {
             tc_fence_after();
-            // this stream's keys are rows [KW (s % KS), KW (s % KS) + KW) of the V tile
-            const uint32_t vpart = vaddr + static_cast<uint32_t>((s % KS) * KW) * 128u;
-#pragma unroll
-            for (int kk = 0; kk < KW / 16; ++kk)
-              mma_ts(tmem + L::O_COL + D * s, tmem + KW * s + 8 * kk,
-                     sdesc_sw128(vpart + kk * 2048, L::PANEL, 1024), kIdPV,
-                     (((o_init >> s) & 1u) != 0u || kk > 0) ? 1u : 0u);
-            o_init |= 1u << s;
-            mma_commit(bar(L::B_ODONE + s));
+            issue_s_buf(1);
           }
-          if (kbn < w.kb_end && w.act_s(s / KS, s % KS, KW, kbn)) {
-            if (!kn_ready) {
-              if (!mbar_wait(bar(L::B_KFULL + sn), phn, g)) {
+        }
+        for (int it = 0; ok && kb < w.kb_end; ++it) {
+          const int kb2 = kb1 < w.kb_end ? w.next(kb1 + 1) : w.kb_end;
+          const uint32_t buf = static_cast<uint32_t>(it) & 1u;
+          if (!mbar_wait(bar(L::B_VFULL), buf, g) || !mbar_wait(bar(L::B_PFULL), buf, g)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < KW / 16; ++kk)
+            mma_ts(tmem + L::O_COL, tmem + KW * buf + 8 * kk,
+                   sdesc_sw128(vaddr + kk * 2048, L::PANEL, 1024), kIdPV,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::B_ODONE));
+          mma_commit(bar(L::B_VEMPTY));  // the V tile is free once its PV is done
+          if (kb2 < w.kb_end) {
+            if (!mbar_wait(bar(L::B_KFULL), buf, g)) break;  // tile it + 2: parity it & 1
+            tc_fence_after();
+            issue_s_buf(buf);
+          }
+          kb = kb1;
+          kb1 = kb2;
+        }
+      } else {
+        int kb = w.next(0);
+        int it = 0;
+        if (kb < w.kb_end) {
+          ok = mbar_wait(bar(L::B_KFULL + 0), 0, g);
+  #pragma unroll(kUnrollS)
+          for (int s = 0; s < NS; ++s) {
+            if (!ok || !w.act_s(s / KS, s % KS, KW, kb)) continue;
+            ok = ensure_q(s / KS);
+            if (ok) {
+              tc_fence_after();
+              issue_s(s, sbase + L::OFF_KV);
+            }
+          }
+        }
+        while (ok && kb < w.kb_end) {
+          const int st = it % L::STAGES;
+          const uint32_t ph = (it / L::STAGES) & 1u;
+          const int kbn = w.next(kb + 1);
+          const int sn = (it + 1) % L::STAGES;
+          const uint32_t phn = ((it + 1) / L::STAGES) & 1u;
+          bool kn_ready = false;
+          if (!mbar_wait(bar(L::B_VFULL + st), ph, g)) break;
+          const uint32_t vaddr = sbase + L::OFF_KV + st * 2 * L::TILE + L::TILE;
+  #pragma unroll(kUnrollS)
+          for (int s = 0; s < NS; ++s) {
+            if (!ok) break;
+            if (w.act_s(s / KS, s % KS, KW, kb)) {
+              if (!mbar_wait(bar(L::B_PFULL + s), (p_par >> s) & 1u, g)) {
                 ok = false;
                 break;
               }
-              kn_ready = true;
+              p_par ^= 1u << s;
+              tc_fence_after();
+              // this stream's keys are rows [KW (s % KS), KW (s % KS) + KW) of the V tile
+              const uint32_t vpart = vaddr + static_cast<uint32_t>((s % KS) * KW) * 128u;
+  #pragma unroll
+              for (int kk = 0; kk < KW / 16; ++kk)
+                mma_ts(tmem + L::O_COL + D * s, tmem + KW * s + 8 * kk,
+                       sdesc_sw128(vpart + kk * 2048, L::PANEL, 1024), kIdPV,
+                       (((o_init >> s) & 1u) != 0u || kk > 0) ? 1u : 0u);
+              o_init |= 1u << s;
+              mma_commit(bar(L::B_ODONE + s));
             }
-            if (!ensure_q(s / KS)) {
-              ok = false;
-              break;
+            if (kbn < w.kb_end && w.act_s(s / KS, s % KS, KW, kbn)) {
+              if (!kn_ready) {
+                if (!mbar_wait(bar(L::B_KFULL + sn), phn, g)) {
+                  ok = false;
+                  break;
+                }
+                kn_ready = true;
+              }
+              if (!ensure_q(s / KS)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_s(s, sbase + L::OFF_KV + sn * 2 * L::TILE);
             }
-            tc_fence_after();
-            issue_s(s, sbase + L::OFF_KV + sn * 2 * L::TILE);
           }
-        }
-        if (!ok) break;
-        if constexpr (L::SPLIT_RELEASE) {
-          // V of this tile once its PV MMAs are done; K of the next tile once
-          // its S MMAs are (both commits track every MMA issued before them)
-          mma_commit(bar(L::B_VEMPTY + st));
-          if (kn_ready) mma_commit(bar(L::B_KVEMPTY + sn));
-        } else {
+          if (!ok) break;
           mma_commit(bar(L::B_KVEMPTY + st));
+          kb = kbn;
+          ++it;
         }
-        kb = kbn;
-        ++it;
       }
       // every MMA issued above has completed once this commit arrives
       mma_commit(bar(L::B_DRAIN));
@@ -466,7 +532,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     const int i = w.q0 + 128 * t + r;
     if (t == 0 || w.exists1) {
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-      const uint32_t s_addr = lane_addr + KW * s;
+      const uint32_t s_base = lane_addr + KW * s;
       const uint32_t o_addr = lane_addr + L::O_COL + D * s;
       float m = -INFINITY;  // reference maximum, log2 units of scaled scores
       float l = 0.f;        // row sum of exp2(x - m)
@@ -474,7 +540,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       bool ok = true;
       for (int kb = w.next(0); kb < w.kb_end; kb = w.next(kb + 1)) {
         if (!w.act_s(t, hp, KW, kb)) continue;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + s), cnt & 1u, g));
+        // S / P buffer of this tile (tiles alternate when there are two)
+        const uint32_t buf = L::S_BUFS == 2 ? (cnt & 1u) : 0u;
+        const uint32_t s_addr = s_base + KW * NS * buf;
+        const uint32_t s_par = L::S_BUFS == 2 ? ((cnt >> 1) & 1u) : (cnt & 1u);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + s + NS * buf), s_par, g));
         if (!ok) break;
         tc_fence_after();
         uint32_t sr[KW];
