@@ -1,7 +1,7 @@
 // Forward pass of exact attention on sm_100a.
 //
 // Work unit: one (b, h) and NQ 128-row Q tiles (NQ = 2 at d = 128, 1 at
-// d = 64) that share every K/V tile the CTA loads.  The CTA walks the K/V tiles
+// d = 64 and 256) that share every K/V tile the CTA loads.  The CTA walks the K/V tiles
 // of its head that at least one of its Q tiles needs (tiles that are fully
 // masked by the causal mask, the key lengths or the block mask are neither
 // loaded nor computed).
@@ -25,8 +25,10 @@
 //
 // Roles:
 //   warp 0            TMA producer: Q tiles once, then K/V tiles into a ring
+//                     (d = 256: K tiles only)
 //   warp 1            TMEM allocator and single-thread MMA issuer
-//   warps 2-3         idle
+//   warp 2            d = 256: TMA producer of the V tiles; else idle
+//   warp 3            idle
 //   warpgroup 1 + s   softmax stream s (thread = row, TMEM lanes 0..127)
 //
 // The running maximum m is only moved when a new block raises it by more than
@@ -37,7 +39,8 @@
 //
 // TMEM columns: S/P of stream s at [KW s, KW s + KW) (KW = 128 / KS keys; P
 // packed as bf16 pairs in the first KW / 2 columns), O of stream s at
-// [KW NS + D s, KW NS + D s + D), NS = NQ KS streams.
+// [KW NS + D s, KW NS + D s + D), NS = NQ KS streams.  d = 256: S/P of tile n
+// at [128 (n & 1), 128 (n & 1) + 128) (two buffers), O at [256, 512).
 #include <cuda_bf16.h>
 
 #include "devctx.h"
