@@ -56,7 +56,7 @@ def compare(o, lse, ro, rl, record=None):
     small = np.abs(ro) < 2.0
     err_small = diff[small].max() if small.any() else 0.0
     excess = (diff - (O_TOL + 2.0 ** -8 * np.abs(ro))).max()
-    err_l = np.abs(np.where(empty, 0, lse - rl)).max()
+    err_l = np.abs(lse[~empty] - rl[~empty]).max() if (~empty).any() else 0.0
     if record is not None:
         record(o_max_abs=float(err_o), o_max_abs_where_abs_ref_lt_2=float(err_small),
                o_max_abs_ref=float(np.abs(ro).max()), lse_max_abs=float(err_l))
