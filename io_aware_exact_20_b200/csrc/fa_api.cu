@@ -59,7 +59,7 @@ constexpr int kMaxRows = 1 << 23;
 int kernel_dim(int d) {
   if (d == 32 || d == 64) return 64;
   if (d == 96 || d == 128) return 128;
-  if (d == 192 || d == 256) return 256;  // forward only
+  if (d == 192 || d == 256) return 256;
   return 0;
 }
 
@@ -110,14 +110,15 @@ fa_status_t resolve(const fa_attention_desc_t* a, Problem* p, Uses uses) {
   if (a->seqlens_k != nullptr && !aligned(a->seqlens_k, 4)) return FA_ERR_INVALID_ARG;
   const int D = kernel_dim(a->head_dim);
   if (D == 0) return FA_ERR_UNSUPPORTED;
-  // the backward kernels hold a 128-key tile's dK and dV in TMEM: d <= 128
-  if (uses == kBackward && D > 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(a->batch) * a->heads > 65535) return FA_ERR_UNSUPPORTED;
   if (a->seqlen_q > kMaxRows || a->seqlen_k > kMaxRows) return FA_ERR_UNSUPPORTED;
   // one CTA per (b, h, 128-row tile) in a 1-D grid
   const int64_t tiles = (static_cast<int64_t>(a->seqlen_q > a->seqlen_k ? a->seqlen_q : a->seqlen_k) +
                          127) / 128;
-  if (static_cast<int64_t>(a->batch) * a->heads * tiles > 0x7FFFFFFF) return FA_ERR_UNSUPPORTED;
+  // (the d = 256 backward runs two CTAs per key tile)
+  const int64_t per_tile = (uses == kBackward && D == 256) ? 2 : 1;
+  if (static_cast<int64_t>(a->batch) * a->heads * tiles * per_tile > 0x7FFFFFFF)
+    return FA_ERR_UNSUPPORTED;
   const fa_strides_t* all[8] = {&a->q, &a->k, &a->v, &a->o, &a->dout, &a->dq, &a->dk, &a->dv};
   for (int t = 0; t < (uses == kForward ? 4 : 8); ++t) {
     const fa_strides_t* s = all[t];
@@ -432,7 +433,7 @@ fa_status_t fa_fwd_ex(const fa_attention_desc_t* desc, const void* q, const void
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || kernel_dim(d) == 0 || kernel_dim(d) > 128) return 0;
+  if (B < 1 || H < 1 || N < 1 || kernel_dim(d) == 0) return 0;
   const fa_attention_desc_t a = classic_desc(B, H, N, d, 1.f, 0, nullptr, 0.f, 0, nullptr);
   Problem pr;
   if (resolve(&a, &pr, kBackward) != FA_OK) {  // sizes beyond the kernels' limits: still report the bytes

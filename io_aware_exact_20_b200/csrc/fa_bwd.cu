@@ -60,14 +60,22 @@ struct BwdLayout {
   static constexpr int PANELS = D / 64;
   static constexpr uint32_t PANEL = 128u * 128u;
   static constexpr uint32_t TILE = PANEL * PANELS;
-  static constexpr int STAGES = (D == 64) ? 3 : 2;
+  // d = 256: two CTAs per key tile, each owning HD = 128 of the feature
+  // columns of dK, dV and dQ (both recompute S^T and dP^T over all 256).
+  // K and V stay resident; Q and dO pass through a ring of 64-column panels
+  // in the order the MMAs consume them.
+  static constexpr bool RING = (D == 256);
+  static constexpr int HD = RING ? 128 : D;
+  // Q / dO stages, or (RING) panel slots
+  static constexpr int STAGES = RING ? 4 : (D == 64) ? 3 : 2;
+  static constexpr int LD_STAGES = RING ? 2 : STAGES;
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = TILE;
-  static constexpr uint32_t OFF_Q = 2 * TILE;
-  static constexpr uint32_t OFF_DO = OFF_Q + STAGES * TILE;
-  static constexpr uint32_t OFF_DS = OFF_DO + STAGES * TILE;  // [128 keys][128 queries] bf16
-  static constexpr uint32_t OFF_LD = OFF_DS + 2 * PANEL;      // per stage: -lse2[128], -delta[128]
-  static constexpr uint32_t OFF_BAR = OFF_LD + STAGES * 1024;
+  static constexpr uint32_t OFF_Q = 2 * TILE;  // RING: the panel slots
+  static constexpr uint32_t OFF_DO = OFF_Q + (RING ? STAGES * PANEL : STAGES * TILE);
+  static constexpr uint32_t OFF_DS = OFF_DO + (RING ? 0 : STAGES * TILE);  // [128 keys][128 queries] bf16
+  static constexpr uint32_t OFF_LD = OFF_DS + 2 * PANEL;  // per stage: -lse2[128], -delta[128]
+  static constexpr uint32_t OFF_BAR = OFF_LD + LD_STAGES * 1024;
   static constexpr int B_KV = 0;
   static constexpr int B_QFULL = 1;
   static constexpr int B_QEMPTY = B_QFULL + STAGES;
@@ -80,7 +88,9 @@ struct BwdLayout {
   static constexpr int B_DQEMPTY = B_DQFULL + 1;
   static constexpr int B_KVDONE = B_DQEMPTY + 1;
   static constexpr int B_STAGED = B_KVDONE + 1;   // dQ tile written to the staging boxes
-  static constexpr int NBAR = B_STAGED + 1;
+  static constexpr int B_LDFULL = B_STAGED + 1;   // RING: the LSE / D slices of a query tile
+  static constexpr int B_LDEMPTY = B_LDFULL + 2;
+  static constexpr int NBAR = RING ? B_LDEMPTY + 2 : B_STAGED + 1;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   // block masks at d = 64: bitmask of the query tiles this key tile meets
   // (up to 32 BIT_WORDS query tiles).  d = 128 keeps the direct walk: its
@@ -88,23 +98,24 @@ struct BwdLayout {
   static constexpr int BIT_WORDS = (D == 64) ? 1024 : 0;
   static constexpr uint32_t OFF_BITS = OFF_MISC + 16;
   static constexpr uint32_t SMEM = OFF_BITS + BIT_WORDS * 4;
-  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-  // d = 64 leaves room for a dQ tile of its own; d = 128 reuses the dP^T
-  // columns once dP^T has been consumed.
-  static constexpr bool SEPARATE_DQ = (COL_DK + D + D <= 512);
-  static constexpr uint32_t COL_DQ = SEPARATE_DQ ? COL_DK + D : COL_DP;
-  // d = 128: the dQ tile is computed transposed (dQ^T = K^T dS^T, TMEM lane =
-  // feature c, column = query) so that each warp's reduction into the fp32
-  // accumulators covers 32 consecutive floats of one row: one 128-byte line.
-  static constexpr bool DQ_T = (D == 128);
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + HD;
+  // d = 64 leaves room for a dQ tile of its own; d = 128 and 256 reuse the
+  // dP^T columns once dP^T has been consumed.
+  static constexpr bool SEPARATE_DQ = (COL_DK + HD + HD <= 512);
+  static constexpr uint32_t COL_DQ = SEPARATE_DQ ? COL_DK + HD : COL_DP;
+  // d = 128 / 256: the dQ tile (its HD columns) is computed transposed
+  // (dQ^T = K^T dS^T, TMEM lane = feature c, column = query) so that each
+  // warp's reduction into the fp32 accumulators covers 32 consecutive floats
+  // of one row: one 128-byte line.
+  static constexpr bool DQ_T = (D == 128 || RING);
   // d = 64: the dQ tile is staged in the just-consumed Q / dO stage and added
   // into the accumulators by TMA bulk reduce-adds (the dQ warps then hand the
   // stage back to the producer).  d = 128 keeps the transposed tile and its
   // coalesced reductions: there a 64 KB stage of the two-deep Q / dO ring
   // held until the reduce has read it costs more than it saves.
   static constexpr bool TMA_REDUCE = !DQ_T;
-  // d = 128: setmaxnreg moves registers from warpgroup 0 (producer, MMA
-  // issuer) to the dQ warpgroup, which reads the whole transposed dQ tile
+  // d = 128 / 256: setmaxnreg moves registers from warpgroup 0 (producer,
+  // MMA issuer) to the dQ warpgroup, which reads the whole transposed dQ tile
   // (128 values per thread) out of TMEM before it starts the reductions, so
   // that the TMEM columns it shares with the next tile's dP^T are free early.
   // 128 * (REGS_CTL + 2 * 128 + REGS_DQ) must equal 512 threads x 128.
@@ -113,7 +124,8 @@ struct BwdLayout {
   static constexpr uint32_t REGS_DQ = 184;
   static_assert(REGS_CTL + 2 * 128 + REGS_DQ == 4 * 128, "register split");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(COL_DK + D <= 512, "TMEM budget");
+  static_assert(COL_DK + HD <= 512, "TMEM budget");
+  static_assert(!RING || BIT_WORDS == 0, "no room for the bitmask next to the ring");
 };
 
 // The key tile of this CTA and the query tiles that meet it.  Rows and keys
@@ -267,7 +279,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
 
   BwdWork<BITS> w;
-  grid_unit(blockIdx.x, p.B * p.H, (p.rows.nk + 127) / 128, p.group_heads, &w.bh,
+  // d = 256: CTAs 2u and 2u + 1 take the two column halves of unit u
+  const int hf = L::RING ? static_cast<int>(blockIdx.x & 1u) : 0;
+  const long long unit = L::RING ? static_cast<long long>(blockIdx.x >> 1) : blockIdx.x;
+  grid_unit(unit, p.B * p.H, (p.rows.nk + 127) / 128, p.group_heads, &w.bh,
             &w.kb);  // key tile 0 is heaviest
   w.b = w.bh / p.H;
   w.h = w.bh % p.H;
@@ -326,6 +341,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(L::B_DQEMPTY), 4);   // one arrival per dQ warp
     mbar_init(bar(L::B_KVDONE), 1);
     mbar_init(bar(L::B_STAGED), 4);    // one arrival per dQ warp
+    if constexpr (L::RING) {
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(bar(L::B_LDFULL + s), 1);
+        mbar_init(bar(L::B_LDEMPTY + s), 8);  // one arrival per P / dS warp
+      }
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -355,6 +376,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_4d(sbase + L::OFF_V + pn * L::PANEL, &tm_v, bar(L::B_KV), 64 * pn,
                     w.krow + w.kb * 128, w.h, w.tb);
       }
+      if constexpr (L::RING) {
+        // Panels in the order the MMA warp consumes them: Q(first), dO(first)
+        // for the first S^T / dP^T, then per query tile n: this CTA's two dO
+        // panels (dV), Q(n + 1) (next S^T), this CTA's two Q panels (dK),
+        // dO(n + 1) (next dP^T).  A tile adds 12 panels (4 for the last), a
+        // multiple of the 4 slots, so the pairs for dV and dK always sit in
+        // the adjacent slots 0, 1 and 2, 3.
+        int t = 0, nld = 0;
+        auto panel = [&](const CUtensorMap* m, int pn, int qb) -> bool {
+          const int s = t % L::STAGES;
+          if (t >= L::STAGES && !mbar_wait(bar(L::B_QEMPTY + s), ((t / L::STAGES) & 1u) ^ 1u, g))
+            return false;
+          mbar_arrive_expect_tx(bar(L::B_QFULL + s), L::PANEL);
+          tma_load_4d(sbase + L::OFF_Q + s * L::PANEL, m, bar(L::B_QFULL + s), 64 * pn,
+                      w.qrow + qb * 128, w.h, w.tb);
+          ++t;
+          return true;
+        };
+        auto tile4 = [&](const CUtensorMap* m, int qb) -> bool {
+          for (int pn = 0; pn < L::PANELS; ++pn)
+            if (!panel(m, pn, qb)) return false;
+          return true;
+        };
+        auto ld = [&](int qb) -> bool {  // -LSE log2e and -D of the tile's rows
+          const int s = nld & 1;
+          if (nld >= 2 && !mbar_wait(bar(L::B_LDEMPTY + s), ((nld >> 1) & 1u) ^ 1u, g)) return false;
+          mbar_arrive_expect_tx(bar(L::B_LDFULL + s), 1024);
+          const long long roff = w.ws0 + static_cast<long long>(qb) * 128;
+          bulk_load(sbase + L::OFF_LD + s * 1024, p.ws_lse2 + roff, 512, bar(L::B_LDFULL + s));
+          bulk_load(sbase + L::OFF_LD + s * 1024 + 512, p.ws_delta + roff, 512,
+                    bar(L::B_LDFULL + s));
+          ++nld;
+          return true;
+        };
+        bool ok = ld(q_first) && tile4(&tm_q, q_first) && tile4(&tm_do, q_first);
+        for (int qb = q_first; ok && qb < w.nqb;) {
+          const int qbn = w.next(qb + 1);
+          ok = panel(&tm_do, 2 * hf, qb) && panel(&tm_do, 2 * hf + 1, qb);
+          if (ok && qbn < w.nqb) ok = ld(qbn) && tile4(&tm_q, qbn);
+          if (ok) ok = panel(&tm_q, 2 * hf, qb) && panel(&tm_q, 2 * hf + 1, qb);
+          if (ok && qbn < w.nqb) ok = tile4(&tm_do, qbn);
+          qb = qbn;
+        }
+        if (*abort_flag) {
+          for (int j = max(0, t - L::STAGES); j < t; ++j)
+            mbar_wait_drain(bar(L::B_QFULL + j % L::STAGES), (j / L::STAGES) & 1u, 100000000ull);
+          for (int j = max(0, nld - 2); j < nld; ++j)
+            mbar_wait_drain(bar(L::B_LDFULL + (j & 1)), (j >> 1) & 1u, 100000000ull);
+          mbar_wait_drain(bar(L::B_KV), 0, 100000000ull);
+        }
+      } else {
       int it = 0;
       for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
         const int s = it % L::STAGES;
@@ -376,15 +448,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mbar_wait_drain(bar(L::B_QFULL + j % L::STAGES), (j / L::STAGES) & 1u, 100000000ull);
         mbar_wait_drain(bar(L::B_KV), 0, 100000000ull);
       }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0 && any_work) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t kIdKQ = idesc_bf16(128, D, false, true);  // dV, dK
-      constexpr uint32_t kIdQ = L::DQ_T ? idesc_bf16(D, 128, true, true)   // dQ^T
-                                        : idesc_bf16(128, D, true, true);  // dQ
+      constexpr uint32_t kIdKQ = idesc_bf16(128, L::HD, false, true);  // dV, dK
+      constexpr uint32_t kIdQ = L::DQ_T ? idesc_bf16(L::HD, 128, true, true)  // dQ^T
+                                        : idesc_bf16(128, D, true, true);     // dQ
       const uint32_t k_addr = sbase + L::OFF_K, v_addr = sbase + L::OFF_V;
+      // the K panels of this CTA's dQ columns
+      const uint32_t kh_addr = k_addr + static_cast<uint32_t>(2 * hf) * L::PANEL;
       const uint32_t ds_addr = sbase + L::OFF_DS;
       bool ok = mbar_wait(bar(L::B_KV), 0, g);
 
@@ -424,7 +499,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t ds_desc = sdesc_sw128(ds_addr + kk * 2048, L::PANEL, 1024);
-          const uint64_t k_desc = sdesc_sw128(k_addr + kk * 2048, L::PANEL, 1024);
+          const uint64_t k_desc = sdesc_sw128(kh_addr + kk * 2048, L::PANEL, 1024);
           if constexpr (L::DQ_T)
             mma_ss(tmem + L::COL_DQ, k_desc, ds_desc, kIdQ, kk > 0 ? 1u : 0u);
           else
@@ -432,6 +507,89 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
 
+      if constexpr (L::RING) {
+        int c = 0;  // panels taken from the ring
+        auto slot = [&](int s) -> uint32_t { return sbase + L::OFF_Q + s * L::PANEL; };
+        // the slot of the next panel, or -1 once a wait has given up
+        auto take = [&]() -> int {
+          const int s = c % L::STAGES;
+          if (!mbar_wait(bar(L::B_QFULL + s), (c / L::STAGES) & 1u, g)) return -1;
+          tc_fence_after();
+          ++c;
+          return s;
+        };
+        // this CTA's two panels of dO (for dV) or Q (for dK), in the adjacent
+        // slots s, s + 1 (the producer's panel counts keep pairs at even slots)
+        auto take_pair = [&]() -> int {
+          const int s = take();
+          if (s < 0) return -1;
+          if ((s & 1) != 0) {
+            if (p.status) atomicExch(p.status, kStatusInternal);
+            *abort_flag = 1u;
+            return -1;
+          }
+          return take() < 0 ? -1 : s;
+        };
+        // S^T = K Q^T (dp: dP^T = V dO^T) over the tile's four panels, each
+        // slot handed back once its MMAs are done
+        auto ring_sdp = [&](bool dp) -> bool {
+          const uint32_t a_addr = dp ? v_addr : k_addr;
+          const uint32_t col = dp ? L::COL_DP : L::COL_S;
+          for (int pn = 0; pn < L::PANELS; ++pn) {
+            const int s = take();
+            if (s < 0) return false;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem + col, sdesc_sw128(a_addr + pn * L::PANEL + kk * 32, 16, 1024),
+                     sdesc_sw128(slot(s) + kk * 32, 16, 1024), kIdS, (pn > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar(L::B_QEMPTY + s));
+          }
+          mma_commit(bar(dp ? L::B_DPFULL : L::B_SFULL));
+          return true;
+        };
+        // Per query tile: dV, the next tile's S^T (it overwrites S^T / P only
+        // after the dV MMAs), then once dS is in shared memory dQ^T (its
+        // drain runs under dK) and dK, and the next tile's dP^T once the dQ^T
+        // tile has left its columns.  Both P / dS orders (two phases, or one
+        // under dropout) take the same steps here; without the two phases PFULL
+        // already means dS is ready.
+        int it = 0;
+        if (ok) ok = ring_sdp(false) && ring_sdp(true);
+        for (int qb = q_first; ok && qb < w.nqb; ++it) {
+          const int qbn = w.next(qb + 1);
+          if (!mbar_wait(bar(L::B_PFULL), it & 1u, g)) break;
+          tc_fence_after();
+          const int sd = take_pair();
+          if (sd < 0) break;
+          // dV += P^T dO   (A = P from TMEM, B = dO's two panels MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + L::COL_DV, tmem + L::COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
+                   sdesc_sw128(slot(sd) + kk * 2048, L::PANEL, 1024), kIdKQ,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::B_QEMPTY + sd));
+          mma_commit(bar(L::B_QEMPTY + sd + 1));
+          if (qbn < w.nqb && !ring_sdp(false)) break;
+          if constexpr (kTwoPhase) {
+            if (!mbar_wait(bar(L::B_DSFULL), it & 1u, g)) break;
+            tc_fence_after();
+          }
+          issue_dq();
+          mma_commit(bar(L::B_DQFULL));
+          const int sq = take_pair();
+          if (sq < 0) break;
+          issue_dk(slot(sq), it);
+          mma_commit(bar(L::B_QEMPTY + sq));
+          mma_commit(bar(L::B_QEMPTY + sq + 1));
+          mma_commit(bar(L::B_DSEMPTY));
+          if (qbn < w.nqb) {
+            if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
+            tc_fence_after();
+            if (!ring_sdp(true)) break;
+          }
+          qb = qbn;
+        }
+      } else {
       int it = 0;
       if (ok) ok = mbar_wait(bar(L::B_QFULL + 0), 0, g);
       if (ok) {
@@ -546,6 +704,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           qb = qbn;
         }
       }
+      }
       mma_commit(bar(L::B_KVDONE));
       mbar_wait_drain(bar(L::B_KVDONE), 0, 1000000000ull);
     }
@@ -594,10 +753,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             kw[c][r] = __shfl_sync(0xffffffffu, own, (lane & ~7) | r) >> (lane & 7);
         }
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + s), (it / L::STAGES) & 1u, g));
+      // the LSE / D slices come with the Q / dO stage, or (ring) on their own
+      const int ls = L::RING ? (it & 1) : s;
+      if constexpr (L::RING)
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_LDFULL + ls), (it >> 1) & 1u, g));
+      else
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + s), (it / L::STAGES) & 1u, g));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL), it & 1u, g));
       // -LSE log2e and -D of the tile's 128 queries
-      const float* nlse = reinterpret_cast<const float*>(smem + L::OFF_LD + s * 1024);
+      const float* nlse = reinterpret_cast<const float*>(smem + L::OFF_LD + ls * 1024);
       const float* ndlt = nlse + 128;
       // causal: query q of this tile sees this thread's key iff q >= qmin
       const bool diag = w.causal && (w.kb * 128 + 127 > qb * 128 + w.off);
@@ -721,7 +885,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_DSFULL));
+        if (lane == 0) {
+          mbar_arrive(bar(L::B_DSFULL));
+          if constexpr (L::RING) mbar_arrive(bar(L::B_LDEMPTY + ls));  // LSE / D read
+        }
       } else {
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_DPFULL), it & 1u, g));
         if (ok && it > 0)
@@ -787,7 +954,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_PFULL));
+        if (lane == 0) {
+          mbar_arrive(bar(L::B_PFULL));
+          if constexpr (L::RING) mbar_arrive(bar(L::B_LDEMPTY + ls));  // LSE / D read
+        }
       }
     }
 
@@ -799,12 +969,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool row_ok = jg < w.lk;
       const long long kr = w.krow + jg;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        const int col = wg * (D / 2) + 32 * c;
+      for (int c = 0; c < L::HD / 64; ++c) {
+        const int tcol = wg * (L::HD / 2) + 32 * c;  // TMEM column of this CTA's slice
+        const int col = L::HD * hf + tcol;            // feature column
         uint32_t a[32], bk[32];
         if (any_work && n_it > 0) {
-          tmem_ld32<0>(lane_addr + L::COL_DV + col, a);
-          tmem_ld32<0>(lane_addr + L::COL_DK + col, bk);
+          tmem_ld32<0>(lane_addr + L::COL_DV + tcol, a);
+          tmem_ld32<0>(lane_addr + L::COL_DK + tcol, bk);
           tmem_wait_ld32<0>(a);
           tmem_wait_ld32<0>(bk);
         } else {
@@ -851,11 +1022,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                              : sbase + L::OFF_DO + s * L::TILE + (b - L::PANELS) * L::PANEL;
       };
       if constexpr (L::DQ_T) {
-        // lane r = feature r; column c = query qb * 128 + c: each warp's
-        // reduction covers 32 consecutive floats of one accumulator row.
-        // The whole tile comes out of TMEM first and its columns go back to
-        // the MMA warp (for the next tile's dP^T) before the reductions.
-        float* dst = p.ws_dq + (w.ws0 + static_cast<long long>(qb) * 128) * D + r;
+        // lane r = feature HD hf + r; column c = query qb * 128 + c: each
+        // warp's reduction covers 32 consecutive floats of one accumulator
+        // row.  The whole tile comes out of TMEM first and its columns go back
+        // to the MMA warp (for the next tile's dP^T) before the reductions.
+        const int feat = L::HD * hf + r;
+        float* dst = p.ws_dq + (w.ws0 + static_cast<long long>(qb) * 128) * D + feat;
         uint32_t a[128];
         tmem_ld32<0>(lane_addr + L::COL_DQ + 0, a);
         tmem_ld32<32>(lane_addr + L::COL_DQ + 32, a);
@@ -868,8 +1040,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::B_DQEMPTY));  // the dQ columns of TMEM are free again
+        // features past d (zero columns of d = 96 / 192) are left out, whole
+        // warps at a time (d is a multiple of 32)
+        if (feat < p.d_real) {
 #pragma unroll
-        for (int k = 0; k < 128; ++k) red_add_f32(dst + k * D, __uint_as_float(a[k]));
+          for (int k = 0; k < 128; ++k) red_add_f32(dst + k * D, __uint_as_float(a[k]));
+        }
       } else {
         // lane r = query r; columns 32 b .. 32 b + 31 = box b
 #pragma unroll
@@ -956,7 +1132,9 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                                 static_cast<int>(L::SMEM));
   });
   if (e != cudaSuccess) return e;
-  const long long ctas = static_cast<long long>((p.rows.nk + 127) / 128) * p.B * p.H;
+  // d = 256: two CTAs (column halves) per key tile
+  const long long ctas =
+      static_cast<long long>((p.rows.nk + 127) / 128) * p.B * p.H * (L::RING ? 2 : 1);
   if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   return launch_overlapped(kern, dim3(static_cast<unsigned>(ctas)), dim3(kBwdThreads), L::SMEM,
                            stream, tq, tk, tv, tdo, tdq, p);
@@ -972,6 +1150,7 @@ cudaError_t launch_post_t(const BwdParams& p, cudaStream_t stream) {
 cudaError_t launch_bwd_pre(int d, const BwdParams& p, cudaStream_t stream) {
   if (d == 64) return launch_pre_t<64>(p, stream);
   if (d == 128) return launch_pre_t<128>(p, stream);
+  if (d == 256) return launch_pre_t<256>(p, stream);
   return cudaErrorInvalidValue;
 }
 
@@ -991,12 +1170,15 @@ cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CU
   }
   if (d == 128) return dropout ? launch_main_t<128, true, false>(tq, tk, tv, tdo, tdq, p, stream)
                                : launch_main_t<128, false, false>(tq, tk, tv, tdo, tdq, p, stream);
+  if (d == 256) return dropout ? launch_main_t<256, true, false>(tq, tk, tv, tdo, tdq, p, stream)
+                               : launch_main_t<256, false, false>(tq, tk, tv, tdo, tdq, p, stream);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_bwd_post(int d, const BwdParams& p, cudaStream_t stream) {
   if (d == 64) return launch_post_t<64>(p, stream);
   if (d == 128) return launch_post_t<128>(p, stream);
+  if (d == 256) return launch_post_t<256>(p, stream);
   return cudaErrorInvalidValue;
 }
 

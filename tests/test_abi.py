@@ -171,16 +171,21 @@ def test_general_binding_rejects_host_tensors_and_bad_layouts(lib):
         lib.backward_general(q, q, q, q, torch.zeros((1, 2, 128)), q)
 
 
-@pytest.mark.parametrize("d", [192, 256])
-def test_backward_refuses_the_forward_only_head_dims(lib, d):
-    """d = 192 / 256 run the forward only: every backward entry point returns
-    FA_ERR_UNSUPPORTED before any launch and the workspace size is 0.  (No
-    forward call here: with d = 256 the forward is valid and would launch.)"""
+def test_backward_at_width_256(lib):
+    """d = 192 / 256 run the 256-wide backward (two CTAs per key tile): the
+    workspace holds 256 accumulators per row, and a grid that fits one CTA
+    per key tile but not two is refused (FA_ERR_UNSUPPORTED) before any
+    launch, where d = 128 at the same size passes that check and stops at the
+    workspace (FA_ERR_WORKSPACE), also before any launch."""
     so = lib.library()
-    assert so.fa_bwd_workspace_size(1, 2, 256, d) == 0
-    a = _desc(lib, head_dim=d)
-    assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == 0
-    assert so.fa_bwd_ex(ctypes.byref(a), A16, A16, A16, A16, A16, A16, A16, A16, A16, A16,
-                        1 << 30, None) == 2
-    assert so.fa_bwd(A16, A16, A16, A16, A16, A16, A16, A16, A16, 1, 2, 256, d, 0.1, 0, None,
-                     0.0, 0, None, A16, 1 << 30, None) == 2
+    assert so.fa_bwd_workspace_size(1, 1, 128, 256) == 128 * (8 + 1024)
+    assert so.fa_bwd_workspace_size(1, 1, 128, 192) == 128 * (8 + 1024)
+    assert so.fa_bwd_workspace_size(2, 3, 300, 256) == 2 * 3 * 384 * (8 + 1024)
+    st, sk = lib.Strides(3 * 256 * 256, 256 * 256, 256), lib.Strides(3 * 384 * 256, 384 * 256, 256)
+    a = _desc(lib, head_dim=256, q=st, o=st, dout=st, dq=st, k=sk, v=sk, dk=sk, dv=sk)
+    assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == a.batch * a.heads * 256 * (8 + 1024)
+    # 65535 x 32768 key tiles < 2^31 - 1 < twice that
+    big = (65535, 1, 1 << 22)
+    for d, code in ((256, 2), (192, 2), (128, 5)):
+        assert so.fa_bwd(A16, A16, A16, A16, A16, A16, A16, A16, A16, *big, d, 0.1, 0, None,
+                         0.0, 0, None, A16, 1 << 30, None) == code, d

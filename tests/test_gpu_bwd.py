@@ -57,6 +57,11 @@ CASES = [
     (2, 2, 256, 64, True, None, None, 0.1),
     (2, 2, 384, 128, False, (100, 384), None, 0.2),
     (1, 3, 700, 64, True, (500, 700), 0.4, 0.3),
+    # the 256-wide backward (two CTAs per key tile, each with half the columns)
+    (1, 2, 128, 256, False, None, None, 0.0),
+    (2, 2, 300, 256, True, None, None, 0.1),
+    (1, 2, 1000, 192, True, (300, 1000), 0.5, 0.0),
+    (2, 1, 777, 256, False, (100, 777), 0.4, 0.2),
 ]
 
 
@@ -71,7 +76,7 @@ def test_backward_matches_oracle(lib, parity_record, B, H, N, d, causal, lens, d
     parity_record(**{f"{k}_rel_l2": float(v) for k, v in errs.items()})
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("p", [0.0, 0.1])
 def test_backward_block_mask_without_diagonal(lib, parity_record, d, causal, p):
@@ -102,10 +107,11 @@ def test_backward_block_mask_without_diagonal(lib, parity_record, d, causal, p):
     assert (got[1][:, :, 256:384] == 0).all() and (got[2][:, :, 256:384] == 0).all()
 
 
-def test_backward_is_repeatable_for_dk_dv(lib):
+@pytest.mark.parametrize("d", [64, 256])
+def test_backward_is_repeatable_for_dk_dv(lib, d):
     """dK and dV involve no atomics: two runs give identical bits."""
     import torch
-    q, k, v, do = (x.cuda() for x in make_qkvdo(1, 2, 512, 64, 9))
+    q, k, v, do = (x.cuda() for x in make_qkvdo(1, 2, 512, d, 9))
     o, lse = lib.forward(q, k, v, causal=True, dropout_p=0.1, seed=3)
     a = lib.backward(q, k, v, o, lse, do, causal=True, dropout_p=0.1, seed=3)
     b = lib.backward(q, k, v, o, lse, do, causal=True, dropout_p=0.1, seed=3)
@@ -114,7 +120,7 @@ def test_backward_is_repeatable_for_dk_dv(lib):
     assert (a[0].float() - b[0].float()).abs().max().item() < 1e-2
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_backward_kernel_dropout_bits_exact(lib, d):
     """Q = 0 gives P = 1/N; dO rows one-hot over a window of d queries give
     dV[j, c] = keep(i0 + c, j) / (N q), q the keep probability: every keep bit the backward

@@ -2,8 +2,8 @@
 the float64 oracle.  The hand-picked parity cases each vary one or two
 features; here every case draws all of them at once, so that combinations no
 one wrote down get exercised: the layout (classic [B, H, N, d], token-major
-[B, N, H, d], packed variable-length), every head dim (the backward for
-d <= 128, the 256-wide forward alone for 192 / 256), N_q != N_k with the
+[B, N, H, d], packed variable-length), every head dim (32 to 256, the
+forward and the backward), N_q != N_k with the
 bottom-right causal alignment, ragged tails, sequences up to 3000 rows, key
 padding, block masks with whole tile rows and columns removed, dropout, and a
 scale other than d^-1/2.
@@ -97,10 +97,10 @@ def rel_l2(a, ref):
 
 
 def test_sweep_covers_every_feature():
-    """The drawn cases reach every layout, head dim and mask kind, and both
-    the backward and the forward-only dims (checked without a device)."""
-    seen = {(c["layout"], c["d"] <= 128) for c in CASES}
-    assert len(seen) == 6, seen
+    """The drawn cases reach every layout, head dim and mask kind, and the
+    64-, 128- and 256-wide kernels in every layout (checked without a device)."""
+    seen = {(c["layout"], min(w for w in (64, 128, 256) if c["d"] <= w)) for c in CASES}
+    assert len(seen) == 9, seen
     assert {c["d"] for c in CASES} == set(HEAD_DIMS)
     assert any(c["nq"] != c["nk"] and c["layout"] != "thd" for c in CASES)
     assert any(c["mask"] is not None and c["causal"] for c in CASES)
@@ -120,7 +120,6 @@ def test_random_case_matches_oracle(lib, parity_record, c):
     kv_pad = None if c["kv_pad"] is None else np.array(c["kv_pad"], dtype=np.int32)
     kw = dict(layout=layout, scale=c["scale"], causal=c["causal"], seqlens_k=kv_pad,
               dropout_p=c["p"], seed=c["seed"], block_mask=bm)
-    backward = d <= 128
 
     def rnd(*shape):
         return torch.randn(*shape, generator=g).to(torch.bfloat16)
@@ -147,7 +146,7 @@ def test_random_case_matches_oracle(lib, parity_record, c):
 
     q, k, v, do = (to_dev(x) for x in (hq, hk, hv, hdo))
     o, lse = lib.forward_general(q, k, v, **kw)
-    grads = lib.backward_general(q, k, v, o, lse, do, **kw) if backward else None
+    grads = lib.backward_general(q, k, v, o, lse, do, **kw)
     torch.cuda.synchronize()
     assert lib.last_device_status() == 0
 
@@ -161,8 +160,6 @@ def test_random_case_matches_oracle(lib, parity_record, c):
     else:
         ro, rl = attention_forward(f64(hq), f64(hk), f64(hv), *ref_args)
         compare(to_host(o), lse.cpu().numpy().astype(np.float64), ro, rl, parity_record)
-    if not backward:
-        return
 
     if layout == "thd":
         rg = attention_backward_varlen(f64(hq), f64(hk), f64(hv), f64(hdo), cu_q, cu_k, *ref_args)

@@ -1,7 +1,10 @@
-"""The 256-wide forward (head dims 192 and 256, forward only) against the
-float64 oracle: the classic layout, strided and packed layouts, every mask,
+"""The 256-wide kernels (head dims 192 and 256) against the float64 oracle:
+the forward in the classic layout, strided and packed layouts, every mask,
 dropout, rows long enough that the single K/V stage is refilled many times
-(K and V released separately), and the backward's refusal of these dims."""
+(K and V released separately); the backward (two CTAs per key tile, each
+owning half of dK / dV / dQ's columns, Q and dO through a ring of 64-column
+panels) in the same layouts and over enough query tiles to cycle the ring
+many times.  Bounds as in the other parity tests."""
 
 import numpy as np
 import pytest
@@ -77,16 +80,74 @@ def test_wide_forward_general_layouts(lib, parity_record):
             parity_record)
 
 
-def test_wide_backward_is_refused(lib):
-    """The backward entry points refuse d = 256 (no launch, FA_ERR_UNSUPPORTED)."""
+def _rel_l2(a, r):
+    n = np.linalg.norm(r)
+    return np.linalg.norm(a - r) / n if n > 0 else np.linalg.norm(a)
+
+
+def _check_grads(got, ref, record):
+    errs = {}
+    for name, a, r in zip(("dq", "dk", "dv"), got, ref):
+        assert np.isfinite(a).all(), name
+        errs[name] = _rel_l2(a, r)
+    record(**{f"{k}_rel_l2": float(v) for k, v in errs.items()})
+    for name, e in errs.items():
+        assert e <= 2e-2, (name, e)
+
+
+@pytest.mark.parametrize("N,d,causal,p", [
+    (4096, 256, True, 0.0),    # 32 query tiles for the first key tile: the ring turns 96 times
+    (2176, 192, False, 0.1),   # 17 x 128 rows, dropout (the one-pass P / dS order)
+])
+def test_wide_backward_long_rows(lib, parity_record, N, d, causal, p):
     import torch
-    q, k, v, do = (x.cuda() for x in make_qkvdo(1, 1, 128, 256, 3))
-    o, lse = lib.forward(q, k, v)
-    torch.cuda.synchronize()
-    with pytest.raises(lib.FaError):
-        lib.backward(q, k, v, o, lse, do)
+    from oracle import attention_backward
+    q, k, v, do = make_qkvdo(1, 2, N, d, 14)
+    kw = dict(causal=causal, dropout_p=p, seed=15)
+    gq, gk, gv, gdo = (x.cuda() for x in (q, k, v, do))
+    o, lse = lib.forward(gq, gk, gv, **kw)
+    grads = lib.backward(gq, gk, gv, o, lse, gdo, **kw)
     torch.cuda.synchronize()
     assert lib.last_device_status() == 0
+    ref = attention_backward(f64(q), f64(k), f64(v), f64(do), d ** -0.5, causal, None, p, 15)
+    _check_grads(tuple(f64(x) for x in grads), ref, parity_record)
+
+
+def test_wide_backward_general_layouts(lib, parity_record):
+    """Token-major strides with N_q != N_k (bottom-right causal) and a packed
+    variable-length batch with an empty sequence, at d = 256."""
+    import torch
+    from oracle import attention_backward
+    from oracle.varlen_ref import attention_backward_varlen
+    B, H, Nq, Nk, d = 2, 2, 200, 520, 256
+    qh, doh = make_qkvdo(B, H, Nq, d, 16)[0], make_qkvdo(B, H, Nq, d, 17)[3]
+    _, kh, vh, _ = make_qkvdo(B, H, Nk, d, 18)
+    t = lambda x: x.transpose(1, 2).contiguous().cuda()  # noqa: E731  [B, N, H, d]
+    kw = dict(layout="bshd", causal=True, dropout_p=0.1, seed=19)
+    q, k, v, do = t(qh), t(kh), t(vh), t(doh)
+    o, lse = lib.forward_general(q, k, v, **kw)
+    grads = lib.backward_general(q, k, v, o, lse, do, **kw)
+    torch.cuda.synchronize()
+    assert lib.last_device_status() == 0
+    ref = attention_backward(f64(qh), f64(kh), f64(vh), f64(doh), d ** -0.5, True, None, 0.1, 19)
+    _check_grads(tuple(f64(x.transpose(1, 2)) for x in grads), ref, parity_record)
+
+    lq, lk = [129, 0, 300], [200, 5, 300]
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    g = torch.Generator().manual_seed(20)
+    pq, pdo = (torch.randn(int(cu_q[-1]), H, d, generator=g).to(torch.bfloat16) for _ in range(2))
+    pk, pv = (torch.randn(int(cu_k[-1]), H, d, generator=g).to(torch.bfloat16) for _ in range(2))
+    kw = dict(layout="thd", cu_seqlens_q=cu_q, cu_seqlens_k=cu_k, max_seqlen_q=300,
+              max_seqlen_k=300, causal=True, dropout_p=0.1, seed=21)
+    q, k, v, do = (x.cuda() for x in (pq, pk, pv, pdo))
+    o, lse = lib.forward_general(q, k, v, **kw)
+    grads = lib.backward_general(q, k, v, o, lse, do, **kw)
+    torch.cuda.synchronize()
+    assert lib.last_device_status() == 0
+    ref = attention_backward_varlen(f64(pq), f64(pk), f64(pv), f64(pdo), cu_q, cu_k, d ** -0.5,
+                                    True, None, 0.1, 21)
+    _check_grads(tuple(f64(x) for x in grads), ref, parity_record)
 
 
 def test_wide_forward_bitmask_walk_equals_byte_walk(lib):
