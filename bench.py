@@ -13,7 +13,7 @@ their predecessor's last wave); the per-launch split comes from a second
 pass of the same steps with an event between every two launches.
 
 The default run times every workload (tiny, GPT-2, BERT, long d=64, long
-d=128, block-sparse) one after the other.  The headline ``value`` is the
+d=128, long d=256, block-sparse) one after the other.  The headline ``value`` is the
 dense long-sequence case (B=1 H=16 N=16384 d=128 causal) timed over exactly
 K steps; ``per_config`` holds each workload (that one included, timed again
 for at least half a second so the clock record has many samples) with its
@@ -59,7 +59,7 @@ from io_aware_exact_20_b200.workloads import WORKLOADS, attention_flops, make_in
 METRIC = "attention fwd+bwd TFLOP/s (bf16, N=512–64K) and % of B200 dense BF16 peak"
 UNIT = "TFLOP/s"
 HEADLINE = "long128"
-ORDER = ["tiny", "gpt2", "bert", "long64", "long128", "sparse"]
+ORDER = ["tiny", "gpt2", "bert", "long64", "long128", "long256", "sparse"]
 UNFUSED_CONFIGS = ("gpt2", "long128")
 FLUSH_BYTES = 256 << 20
 DATASHEET_BF16_TFLOPS = 2250.0
@@ -74,10 +74,6 @@ PROJ_SHAPES = {
     "qkv_proj_gpt2": (8, 1024, 12, 64, 768),
     "qkv_proj_long128": (1, 16384, 16, 128, 2048),
 }
-FWD_ONLY_SHAPES = {
-    # forward-only head dims (no backward kernel), name: (B, H, N, d, causal)
-    "fwd_long256": (1, 16, 16384, 256, True),
-}
 
 
 def parse_args(argv=None):
@@ -86,8 +82,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all"] + sorted(WORKLOADS) + sorted(PROJ_SHAPES)
-                    + sorted(FWD_ONLY_SHAPES),
+    ap.add_argument("--workload", choices=["all"] + sorted(WORKLOADS) + sorted(PROJ_SHAPES),
                     default="all",
                     help="'all' (default): headline plus every workload in per_config; a name: "
                          "that workload alone as the headline (profiling); a qkv_proj_* name: "
@@ -111,8 +106,7 @@ def parse_args(argv=None):
                     help="instead of the bench line: fused vs unfused time and peak memory "
                          "for N = 1K..32K (B=1 H=4 d=128 causal)")
     args = ap.parse_args(argv)
-    if (args.workload == "all" or args.workload in PROJ_SHAPES
-            or args.workload in FWD_ONLY_SHAPES) and (
+    if (args.workload == "all" or args.workload in PROJ_SHAPES) and (
             args.batch or args.seqlen or args.dropout is not None):
         ap.error("--batch/--seqlen/--dropout need a single attention --workload")
     return args
@@ -615,50 +609,6 @@ def measure_projection(fa, name, args, rank, dev, flush, stream, world, local, p
                         "fused_speedup": ms_u / ms}}
 
 
-def measure_forward_only(fa, name, args, rank, dev, flush, stream, world, local, peak):
-    """The forward at a head dim that has no backward kernel (256): the same
-    timing rules as the other entries, L2 flushed before each launch."""
-    import torch
-    from io_aware_exact_20_b200.workloads import make_qkvdo
-    B, H, N, d, causal = FWD_ONLY_SHAPES[name]
-    q, k, v = (x.to(dev) for x in make_qkvdo(B, H, N, d, 17)[:3])
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-
-    def fwd():
-        fa.forward(q, k, v, causal=causal, out=o, lse=lse)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        fwd()
-    torch.cuda.synchronize(dev)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    fwd()
-    b.record(stream)
-    torch.cuda.synchronize(dev)
-    n = int(min(5000, max(args.steps, math.ceil(args.min_seconds * 1e3 /
-                                               max(a.elapsed_time(b) + 0.05, 1e-3)))))
-    n = int(max_over_ranks(n, world, dev))
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(n)]
-    with ClockSampler(local) as clk:
-        for e0, e1 in ev:
-            flush.zero_()
-            e0.record(stream)
-            fwd()
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-    ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / n, world, dev)
-    f_fwd, _ = attention_flops(B, H, N, d, causal)
-    ach = tflops(f_fwd, ms)
-    return {"shape": f"forward only: B={B} H={H} N={N} d={d}" + (" causal" if causal else ""),
-            "steps": n, "ms": ms, "tflops": ach,
-            "roofline": {"bound": "tensor", "kernel": "fwd_kernel", "achieved": ach,
-                         "peak": peak, "frac": ach / peak},
-            "clocks": clk.summary(), "device_status": fa.last_device_status()}
-
-
 def timed_region(case, steps, flush, stream, dev, world, clk_index):
     """Times `steps` steps, L2 flushed before each, in two passes: the steps
     alone, one event before and one after each (nothing between the launches,
@@ -768,9 +718,9 @@ def run_ours(args):
 
     if args.unfused_sweep:
         return run_unfused_sweep(args, fa, dev, flush, stream, world, rank)
-    if args.workload in PROJ_SHAPES or args.workload in FWD_ONLY_SHAPES:
-        fn = measure_projection if args.workload in PROJ_SHAPES else measure_forward_only
-        r = fn(fa, args.workload, args, rank, dev, flush, stream, world, local, peak)
+    if args.workload in PROJ_SHAPES:
+        r = measure_projection(fa, args.workload, args, rank, dev, flush, stream, world, local,
+                               peak)
         if rank == 0:
             print(json.dumps({"workload": args.workload, **r}), flush=True)
         return 0
@@ -829,8 +779,6 @@ def run_ours(args):
                 jobs.append(("bert_packed", measure_packed, WORKLOADS[name]))
         for name in PROJ_SHAPES:
             jobs.append((name, measure_projection, name))
-        for name in FWD_ONLY_SHAPES:
-            jobs.append((name, measure_forward_only, name))
         for name, fn, wl in jobs:
             try:
                 per_config[name] = fn(fa, wl, args, rank, dev, flush, stream, world, local, peak)

@@ -379,10 +379,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if constexpr (L::RING) {
         // Panels in the order the MMA warp consumes them: Q(first), dO(first)
         // for the first S^T / dP^T, then per query tile n: this CTA's two dO
-        // panels (dV), Q(n + 1) (next S^T), this CTA's two Q panels (dK),
-        // dO(n + 1) (next dP^T).  A tile adds 12 panels (4 for the last), a
+        // panels (dV), Q(n + 1) (next S^T), dO(n + 1) (next dP^T), this CTA's
+        // two Q panels (dK).  A tile adds 12 panels (4 for the last), a
         // multiple of the 4 slots, so the pairs for dV and dK always sit in
-        // the adjacent slots 0, 1 and 2, 3.
+        // the adjacent slots 0, 1 and 2, 3.  dO(n + 1) takes the slots the
+        // next S^T frees early and is resident by the time dP^T(n + 1) can
+        // start; the reload of the Q pair waits for dP^T(n + 1) instead, off
+        // the path from one tile's dS to the next tile's dP^T.
         int t = 0, nld = 0;
         auto panel = [&](const CUtensorMap* m, int pn, int qb) -> bool {
           const int s = t % L::STAGES;
@@ -414,9 +417,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int qb = q_first; ok && qb < w.nqb;) {
           const int qbn = w.next(qb + 1);
           ok = panel(&tm_do, 2 * hf, qb) && panel(&tm_do, 2 * hf + 1, qb);
-          if (ok && qbn < w.nqb) ok = ld(qbn) && tile4(&tm_q, qbn);
+          if (ok && qbn < w.nqb) ok = ld(qbn) && tile4(&tm_q, qbn) && tile4(&tm_do, qbn);
           if (ok) ok = panel(&tm_q, 2 * hf, qb) && panel(&tm_q, 2 * hf + 1, qb);
-          if (ok && qbn < w.nqb) ok = tile4(&tm_do, qbn);
           qb = qbn;
         }
         if (*abort_flag) {
@@ -548,11 +550,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           return true;
         };
         // Per query tile: dV, the next tile's S^T (it overwrites S^T / P only
-        // after the dV MMAs), then once dS is in shared memory dQ^T (its
-        // drain runs under dK) and dK, and the next tile's dP^T once the dQ^T
-        // tile has left its columns.  Both P / dS orders (two phases, or one
-        // under dropout) take the same steps here; without the two phases PFULL
-        // already means dS is ready.
+        // after the dV MMAs), then once dS is in shared memory dQ^T, the next
+        // tile's dP^T once the dQ^T tile has left its columns, and dK.  Both
+        // P / dS orders (two phases, or one under dropout) take the same steps
+        // here; without the two phases PFULL already means dS is ready.
         int it = 0;
         if (ok) ok = ring_sdp(false) && ring_sdp(true);
         for (int qb = q_first; ok && qb < w.nqb; ++it) {
@@ -576,17 +577,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           issue_dq();
           mma_commit(bar(L::B_DQFULL));
+          if (qbn < w.nqb) {
+            if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
+            tc_fence_after();
+            if (!ring_sdp(true)) break;
+          }
           const int sq = take_pair();
           if (sq < 0) break;
           issue_dk(slot(sq), it);
           mma_commit(bar(L::B_QEMPTY + sq));
           mma_commit(bar(L::B_QEMPTY + sq + 1));
           mma_commit(bar(L::B_DSEMPTY));
-          if (qbn < w.nqb) {
-            if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
-            tc_fence_after();
-            if (!ring_sdp(true)) break;
-          }
           qb = qbn;
         }
       } else {

@@ -55,14 +55,15 @@ def _wl(k, name, B, H, N, d, **kw):
 
 
 # The five workloads: tiny exact case, GPT-2-small-shaped causal with dropout,
-# BERT-large-shaped key-padded with dropout, long causal sequence (d 64 and
-# 128), and the 64K block-sparse case.
+# BERT-large-shaped key-padded with dropout, long causal sequence (d 64, 128
+# and 256), and the 64K block-sparse case.
 WORKLOADS = {
     "tiny": _wl(1, "tiny", 1, 2, 128, 64),
     "gpt2": _wl(2, "gpt2", 8, 12, 1024, 64, causal=True, dropout_p=0.1),
     "bert": _wl(3, "bert", 16, 16, 512, 64, dropout_p=0.1, seqlen_range=(256, 512)),
     "long64": _wl(4, "long64", 1, 16, 16384, 64, causal=True),
     "long128": _wl(4, "long128", 1, 16, 16384, 128, causal=True),
+    "long256": _wl(4, "long256", 1, 16, 16384, 256, causal=True),
     "sparse": _wl(5, "sparse", 1, 8, 65536, 64, block_density=1.0 / 8.0),
 }
 
