@@ -28,13 +28,13 @@
  *    (row-major, d fastest), in device memory, 16-byte aligned.
  *  - LSE is fp32 [B, H, N], natural logarithm; a row with no valid key has
  *    LSE = -inf and O = 0.
- *  - d is 32, 64, 96 or 128 (32 and 96 run the 64- and 128-wide kernels on
- *    zero-filled columns); the forward also takes 192 and 256 (a 256-wide
- *    kernel; the backward entry points return FA_ERR_UNSUPPORTED for them,
- *    since a 128-key tile's dK and dV accumulators would fill the tensor
- *    memory the backward also needs for S and dP).  1 <= N <= 2^23; B * H <= 65535 and
+ *  - d is 32, 64, 96, 128, 192 or 256 (32, 96 and 192 run the 64-, 128-
+ *    and 256-wide kernels on zero-filled columns; the 256-wide backward runs
+ *    two thread blocks per 128-key tile, each owning half of dK, dV and dQ's
+ *    columns).  1 <= N <= 2^23; B * H <= 65535 and
  *    B * H * ceil(N / 128) <= 2^31 - 1 (one thread block per head and
- *    128-row tile); larger requests return FA_ERR_UNSUPPORTED.
+ *    128-row tile; the 256-wide backward needs twice that product within the
+ *    bound); larger requests return FA_ERR_UNSUPPORTED.
  *  - softmax_scale multiplies Q K^T before masking (typically 1/sqrt(d)).
  *  - causal != 0: query i attends key j only if j <= i.
  *  - seqlens: NULL, or device int32[B]; keys j >= seqlens[b] are masked for
@@ -77,7 +77,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, p out of range */
-  FA_ERR_UNSUPPORTED = 2, /* valid request the kernels do not cover (d not 32/64/96/128, sizes too large) */
+  FA_ERR_UNSUPPORTED = 2, /* valid request the kernels do not cover (d not 32/64/96/128/192/256, sizes too large) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed */
   FA_ERR_TIMEOUT = 4,     /* a kernel gave up on a pipeline wait (reported by fa_last_device_status) */
   FA_ERR_WORKSPACE = 5    /* workspace missing or smaller than fa_bwd_workspace_size() */
@@ -92,7 +92,7 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
 /* Bytes of device workspace fa_bwd needs for these sizes: per (b, h) and per
  * query row rounded up to a multiple of 128, one fp32 -LSE_i * log2(e), one
  * fp32 -D_i = -sum_c dO_ic O_ic and D fp32 dQ accumulators (D = 64 for
- * d <= 64, else 128).  0 on bad sizes. */
+ * d <= 64, 128 for d = 96 / 128, 256 for d = 192 / 256).  0 on bad sizes. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /* Backward pass.  Given the forward inputs, its outputs o and lse, and dout
@@ -165,8 +165,8 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
  * lengths (researchpapers.dev "FlashAttention 详解", section 关键结果); the
  * entry points below take them packed, with no padding rows, as well as
  * token-major ([B, N, H, d]) or any other strided layout whose d is
- * contiguous, different query and key counts, and head dims 32, 64, 96, 128
- * (192 and 256: forward only).
+ * contiguous, different query and key counts, and head dims 32, 64, 96, 128,
+ * 192 and 256.
  * The computation is the one above, per batch entry (or packed sequence) b:
  *  - positions i, j are counted inside sequence b (masks, dropout counter);
  *  - causal: query i attends key j iff j <= i + Nk_b - Nq_b, Nq_b / Nk_b the
@@ -186,7 +186,7 @@ typedef struct {
 typedef struct {
   int batch;     /* B: batch entries (padded layout) or packed sequences */
   int heads;     /* H */
-  int head_dim;  /* d: 32, 64, 96 or 128; 192 or 256 for the forward only */
+  int head_dim;  /* d: 32, 64, 96, 128, 192 or 256 */
   /* Padded layout: rows of every batch entry (queries, keys).  Packed layout:
    * an upper bound of every sequence's query / key count (longer sequences
    * are cut to it). */
