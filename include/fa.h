@@ -245,7 +245,7 @@ fa_status_t fa_bwd_ex(const fa_attention_desc_t* desc, const void* q, const void
  * fa_merge_partial: o_acc (fp32 [rows, d], 16-byte aligned) and lse_acc
  *   (fp32 [rows]) hold the result so far (start: any finite o_acc, lse_acc =
  *   -inf); merges in o_part (bf16 [rows, d], contiguous) with lse_part.
- *   d in {32, 64, 96, 128}.  A part or accumulator with LSE = -inf adds
+ *   d in {32, 64, 96, 128, 192, 256}.  A part or accumulator with LSE = -inf adds
  *   nothing; both empty gives O = 0, LSE = -inf.
  * fa_accumulate_bf16: acc[i] += part[i] for i < n (fp32 += bf16), n a multiple
  *   of 8, both 16-byte aligned: sums of gradient parts over key / query blocks.

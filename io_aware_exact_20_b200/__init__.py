@@ -99,13 +99,16 @@ SIGNATURES = {
 
 
 def library():
-    """The loaded C library (raises if it has not been built)."""
+    """The loaded C library (raises if it has not been built).  The
+    environment variable FA_B200_LIBRARY may name another build of it (one of
+    the checking variants of `build.build_variant`)."""
     global _LIB
     if _LIB is None:
-        if not os.path.exists(LIB_PATH):
+        path = os.environ.get("FA_B200_LIBRARY") or LIB_PATH
+        if not os.path.exists(path):
             raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with `python -m io_aware_exact_20_b200.build`")
-        lib = ctypes.CDLL(LIB_PATH)
+                f"{path} is missing: build it with `python -m io_aware_exact_20_b200.build`")
+        lib = ctypes.CDLL(path)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(lib, name)
             fn.restype = res

@@ -24,7 +24,8 @@ namespace {
 
 // G threads per row; the row's d / 8 chunks of 8 columns are dealt out to them
 // round-robin (thread `part` takes chunks part, part + G, ...).  G is the
-// largest power of two dividing d / 8 (4, 8, 4, 16 for d = 32, 64, 96, 128),
+// largest power of two dividing d / 8 (4, 8, 4, 16, 8, 32 for d = 32, 64, 96,
+// 128, 192, 256),
 // so it divides 32 and a row's threads sit in one warp: the row's two LSEs are
 // read once and passed around by shuffles, and the new LSE is written after
 // every thread of the row has read the old one.
@@ -115,7 +116,7 @@ fa_status_t fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part,
   if (!fa::aligned16(o_acc) || !fa::aligned16(o_part) || lse_acc == nullptr ||
       lse_part == nullptr || rows < 0)
     return FA_ERR_INVALID_ARG;
-  if (d != 32 && d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 32 && d != 64 && d != 96 && d != 128 && d != 192 && d != 256) return FA_ERR_UNSUPPORTED;
   if (rows == 0) return FA_OK;
   const int G = (d / 8) & -(d / 8);  // largest power of two dividing d / 8
   if (rows * G / 256 >= 0x7FFFFFFFll) return FA_ERR_UNSUPPORTED;

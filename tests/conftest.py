@@ -44,8 +44,10 @@ def has_gpu():
 
 @pytest.fixture(scope="session")
 def lib():
-    """The C-ABI library, built in-tree if it is missing or stale."""
+    """The C-ABI library, built in-tree if it is missing or stale (unless
+    FA_B200_LIBRARY names another build to load)."""
     from io_aware_exact_20_b200 import build as _build
-    _build.ensure_built()
+    if not os.environ.get("FA_B200_LIBRARY"):
+        _build.ensure_built()
     import io_aware_exact_20_b200 as fa
     return fa

@@ -189,3 +189,12 @@ def test_backward_at_width_256(lib):
     for d, code in ((256, 2), (192, 2), (128, 5)):
         assert so.fa_bwd(A16, A16, A16, A16, A16, A16, A16, A16, A16, *big, d, 0.1, 0, None,
                          0.0, 0, None, A16, 1 << 30, None) == code, d
+
+def test_merge_partial_head_dims(lib):
+    """fa_merge_partial takes every head dim of the attention kernels (32 to
+    256) and refuses others before any launch; zero rows launch nothing."""
+    so = lib.library()
+    for d in (32, 64, 96, 128, 192, 256):
+        assert so.fa_merge_partial(A16, A16, A16, A16, 0, d, None) == 0, d
+    for d in (16, 80, 160, 320, 512):
+        assert so.fa_merge_partial(A16, A16, A16, A16, 5, d, None) == 2, d

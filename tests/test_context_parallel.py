@@ -153,7 +153,8 @@ def test_emulated_ring_with_oracle_kernels_on_cpu(world):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("world", [2, 4])
-@pytest.mark.parametrize("d,causal", [(64, True), (96, True), (128, False), (128, True)])
+@pytest.mark.parametrize("d,causal", [(64, True), (96, True), (128, False), (128, True),
+                                      (192, False), (256, True)])
 def test_ring_with_library_kernels_on_one_gpu(lib, parity_record, world, d, causal):
     """The ring with the library's kernels (fa_fwd_ex, fa_bwd_ex, merge and
     accumulate kernels), W ranks emulated on one device, against the oracle

@@ -14,7 +14,7 @@ def _lse(rng, rows, empty_frac):
     return lse
 
 
-@pytest.mark.parametrize("d", [32, 64, 96, 128])
+@pytest.mark.parametrize("d", [32, 64, 96, 128, 192, 256])
 @pytest.mark.parametrize("rows", [1, 31, 777])
 def test_merge_partial_matches_the_oracle(lib, d, rows):
     """Each row of O_acc / LSE_acc merged with its part, empty parts (LSE = -inf)
