@@ -80,7 +80,9 @@ typedef enum {
   FA_ERR_UNSUPPORTED = 2, /* valid request the kernels do not cover (d not 32/64/96/128/192/256, sizes too large) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed */
   FA_ERR_TIMEOUT = 4,     /* a kernel gave up on a pipeline wait (reported by fa_last_device_status) */
-  FA_ERR_WORKSPACE = 5    /* workspace missing or smaller than fa_bwd_workspace_size() */
+  FA_ERR_WORKSPACE = 5,   /* workspace missing or smaller than fa_bwd_workspace_size() */
+  FA_ERR_BOUNDS = 6       /* only the FA_DEBUG_BOUNDS build: a kernel skipped a global-memory
+                             access outside its buffer (reported by fa_last_device_status) */
 } fa_status_t;
 
 /* Forward pass.  Writes O (bf16 [B,H,N,d]) and LSE (fp32 [B,H,N]).
@@ -294,6 +296,11 @@ void fa_set_wait_timeout_ns(uint64_t ns);
  * same order, so O, LSE, dK and dV come out identical and dQ equal up to the
  * order of its fp32 reductions. */
 void fa_debug_set_block_mask_bitmap(int enabled);
+
+/* 1 in the bounds-checking build (FA_DEBUG_BOUNDS: every global-memory access
+ * the kernels make outside TMA is checked against its buffer's extent, an
+ * out-of-range one skipped and FA_ERR_BOUNDS recorded), 0 otherwise. */
+int fa_debug_bounds_checking(void);
 
 /* Test support: writes the dropout keep bits (1 = kept) of every (b,h,i,j)
  * into keep (device uint8 [B,H,N,N]) using the same device generator as the

@@ -95,6 +95,7 @@ SIGNATURES = {
     "fa_debug_dropout_mask": (_i, [_vp, _i, _i, _i, _f, _u64, _vp]),
     "fa_debug_wait_timeout": (_i, [_vp]),
     "fa_debug_set_block_mask_bitmap": (None, [_i]),
+    "fa_debug_bounds_checking": (_i, []),
 }
 
 

@@ -248,6 +248,32 @@ size_t workspace_bytes_of(const Problem& p) {
   return static_cast<size_t>((bytes + 255) / 256 * 256);
 }
 
+#ifdef FA_DEBUG_BOUNDS
+// Elements from a tensor's base to one past the last element a call may touch.
+long long span(const fa_strides_t& s, int tb, int H, long long rows, int d) {
+  return (tb - 1) * s.batch + (H - 1) * s.head + (rows - 1) * s.row + d;
+}
+
+// Extents of the buffers the kernels address directly, and the rows' offsets.
+void set_extents(const Problem& pr, int* status, fa::Extents* e, fa::Rows* rows) {
+  const int tb = pr.tb();
+  e->o = span(pr.o, tb, pr.H, pr.rows_q(), pr.d);
+  e->dout = span(pr.dout, tb, pr.H, pr.rows_q(), pr.d);
+  e->dq = span(pr.dq, tb, pr.H, pr.rows_q(), pr.d);
+  e->dk = span(pr.dk, tb, pr.H, pr.rows_k(), pr.d);
+  e->dv = span(pr.dv, tb, pr.H, pr.rows_k(), pr.d);
+  long long sb = 0, sh = 0;
+  lse_strides(pr, &sb, &sh);
+  e->lse = (tb - 1) * sb + (pr.H - 1) * sh + pr.rows_q();
+  e->mask = pr.block_mask != nullptr
+                ? static_cast<long long>((pr.nq + 127) / 128) * ((pr.nk + 127) / 128)
+                : 0;
+  e->seqlens = pr.seqlens != nullptr ? pr.B : 0;
+  rows->n_cu = pr.packed ? pr.B + 1 : 0;
+  rows->status = status;
+}
+#endif
+
 fa_status_t run_fwd(const Problem& pr, const void* q, const void* k, const void* v, void* o,
                     float* lse, void* stream) {
   if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(o)) return FA_ERR_INVALID_ARG;
@@ -283,6 +309,9 @@ fa_status_t run_fwd(const Problem& pr, const void* q, const void* k, const void*
   p.rk = fa::philox_round_keys(pr.seed);
   p.timeout_ns = g_timeout_ns.load();
   p.mask_bitmap = g_mask_bitmap.load();
+#ifdef FA_DEBUG_BOUNDS
+  set_extents(pr, status, &p.ext, &p.rows);
+#endif
   const cudaError_t e =
       fa::launch_fwd(pr.D, dr.threshold != 0, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -333,6 +362,9 @@ fa_status_t bwd_params(fa::BwdParams* p, const Problem& pr, const void* workspac
   p->rk = fa::philox_round_keys(pr.seed);
   p->timeout_ns = g_timeout_ns.load();
   p->mask_bitmap = g_mask_bitmap.load();
+#ifdef FA_DEBUG_BOUNDS
+  set_extents(pr, status, &p->ext, &p->rows);
+#endif
   return FA_OK;
 }
 
@@ -391,6 +423,7 @@ const char* fa_status_string(fa_status_t s) {
     case FA_ERR_CUDA: return "CUDA error";
     case FA_ERR_TIMEOUT: return "kernel pipeline wait timed out";
     case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_BOUNDS: return "a kernel index was out of bounds (bounds-checking build)";
   }
   return "unknown status";
 }
@@ -398,6 +431,14 @@ const char* fa_status_string(fa_status_t s) {
 void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns < 1000000ull ? 1000000ull : ns); }
 
 void fa_debug_set_block_mask_bitmap(int enabled) { g_mask_bitmap.store(enabled != 0 ? 1 : 0); }
+
+int fa_debug_bounds_checking(void) {
+#ifdef FA_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 fa_status_t fa_last_device_status(void* stream) {
   int* w = status_word();

@@ -147,10 +147,17 @@ struct BwdWork {
   bool alive, causal;
   const uint8_t* bm;
   const uint32_t* bits;  // shared-memory bitmask over the query tiles, or null
+#ifdef FA_DEBUG_BOUNDS
+  int* status;
+  long long ext_mask;
+#endif
 
   __device__ __forceinline__ bool act(int qb) const {
     if (!alive) return false;
-    if (bm != nullptr && bm[static_cast<size_t>(qb) * nbk + kb] == 0) return false;
+    if (bm != nullptr) {
+      const long long mi = static_cast<long long>(qb) * nbk + kb;
+      if (!FA_IN_BOUNDS(status, mi, 1, ext_mask) || bm[mi] == 0) return false;
+    }
     return true;
   }
   __device__ __forceinline__ int next(int qb) const {
@@ -190,13 +197,13 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   // the bound is a multiple of the block's rows, so whole blocks leave
   if (blockIdx.x * kRowsPerBlock<D> >= (sq.lq + 127) / 128 * 128) return;
   float acc = 0.f;
-  if (i < sq.lq && part * 8 < p.d_real) {
-    const long long r = sq.q0 + i;
-    const uint4 ov = *reinterpret_cast<const uint4*>(
-        static_cast<const __nv_bfloat16*>(p.o) + sq.tb * p.so.b + h * p.so.h + r * p.so.r + part * 8);
-    const uint4 gv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) +
-                                                     sq.tb * p.sdo.b + h * p.sdo.h + r * p.sdo.r +
-                                                     part * 8);
+  const long long r = sq.q0 + i;
+  const long long o_off = sq.tb * p.so.b + h * p.so.h + r * p.so.r + part * 8;
+  const long long do_off = sq.tb * p.sdo.b + h * p.sdo.h + r * p.sdo.r + part * 8;
+  if (i < sq.lq && part * 8 < p.d_real && FA_IN_BOUNDS(p.status, o_off, 8, p.ext.o) &&
+      FA_IN_BOUNDS(p.status, do_off, 8, p.ext.dout)) {
+    const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + o_off);
+    const uint4 gv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + do_off);
     const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
     const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
 #pragma unroll
@@ -210,18 +217,21 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
 #pragma unroll
   for (int m = G / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
   const long long row = ws_row0(p, b, h, sq.q0) + i;
-  if (part == 0) {
+  if (part == 0 && FA_IN_BOUNDS(p.status, row, 1, p.ws_rows)) {
     p.ws_delta[row] = (i < sq.lq) ? -acc : 0.f;
     float nl2 = -INFINITY;
-    if (i < sq.lq) {
-      const float l = p.lse[sq.tb * p.lse_sb + h * p.lse_sh + sq.q0 + i];
+    const long long lse_off = sq.tb * p.lse_sb + h * p.lse_sh + sq.q0 + i;
+    if (i < sq.lq && FA_IN_BOUNDS(p.status, lse_off, 1, p.ext.lse)) {
+      const float l = p.lse[lse_off];
       if (l != -INFINITY) nl2 = -l * kLog2e;
     }
     p.ws_lse2[row] = nl2;
   }
-  float4* dq = reinterpret_cast<float4*>(p.ws_dq + row * D + part * 8);
-  dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-  dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (FA_IN_BOUNDS(p.status, row * D + part * 8, 8, p.ws_rows * D)) {
+    float4* dq = reinterpret_cast<float4*>(p.ws_dq + row * D + part * 8);
+    dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 template <int D>
@@ -235,8 +245,13 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
   const int i = blockIdx.x * kRowsPerBlock<D> + static_cast<int>(threadIdx.x) / G;
   const int part = static_cast<int>(threadIdx.x) % G;
   if (i >= sq.lq || part * 8 >= p.d_real) return;
-  const float4* src = reinterpret_cast<const float4*>(
-      p.ws_dq + (ws_row0(p, b, h, sq.q0) + i) * D + part * 8);
+  const long long acc_off = (ws_row0(p, b, h, sq.q0) + i) * D + part * 8;
+  const long long dq_off = sq.tb * p.sdq.b + h * p.sdq.h + static_cast<long long>(sq.q0 + i) * p.sdq.r +
+                           part * 8;
+  if (!FA_IN_BOUNDS(p.status, acc_off, 8, p.ws_rows * D) ||
+      !FA_IN_BOUNDS(p.status, dq_off, 8, p.ext.dq))
+    return;
+  const float4* src = reinterpret_cast<const float4*>(p.ws_dq + acc_off);
   const float4 a = src[0], c = src[1];
   const float s = p.scale;
   uint4 out;
@@ -244,8 +259,7 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
   out.y = pack_bf16(a.z * s, a.w * s);
   out.z = pack_bf16(c.x * s, c.y * s);
   out.w = pack_bf16(c.z * s, c.w * s);
-  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dq) + sq.tb * p.sdq.b + h * p.sdq.h +
-                            static_cast<long long>(sq.q0 + i) * p.sdq.r + part * 8) = out;
+  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dq) + dq_off) = out;
 }
 
 // ---------------------------------------------------------------------------
@@ -292,7 +306,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // any set-up (the whole CTA takes this branch)
     if (w.kb * 128 >= sq.lk) return;
     int kv = sq.lk;
-    if (p.seqlens != nullptr) kv = max(0, min(p.seqlens[w.b], sq.lk));
+    if (p.seqlens != nullptr && FA_IN_BOUNDS(p.status, w.b, 1, p.ext.seqlens))
+      kv = max(0, min(p.seqlens[w.b], sq.lk));
     w.kv_len = kv;
     w.lk = sq.lk;
     w.qrow = sq.q0;
@@ -313,6 +328,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   w.nbk = p.nbk;
   w.bm = p.block_mask;
   w.bits = nullptr;
+#ifdef FA_DEBUG_BOUNDS
+  w.status = p.status;
+  w.ext_mask = p.ext.mask;
+#endif
   if (BITS && w.bm != nullptr && (w.nqb + 31) / 32 <= L::BIT_WORDS) {
     // every thread takes part: a warp's lanes test 32 consecutive query tiles
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L::OFF_BITS);
@@ -406,7 +425,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int s = nld & 1;
           if (nld >= 2 && !mbar_wait(bar(L::B_LDEMPTY + s), ((nld >> 1) & 1u) ^ 1u, g)) return false;
           mbar_arrive_expect_tx(bar(L::B_LDFULL + s), 1024);
-          const long long roff = w.ws0 + static_cast<long long>(qb) * 128;
+          long long roff = w.ws0 + static_cast<long long>(qb) * 128;
+          if (!FA_IN_BOUNDS(p.status, roff, 128, p.ws_rows)) roff = 0;
           bulk_load(sbase + L::OFF_LD + s * 1024, p.ws_lse2 + roff, 512, bar(L::B_LDFULL + s));
           bulk_load(sbase + L::OFF_LD + s * 1024 + 512, p.ws_delta + roff, 512,
                     bar(L::B_LDFULL + s));
@@ -441,7 +461,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_4d(sbase + L::OFF_DO + s * L::TILE + pn * L::PANEL, &tm_do, bar(L::B_QFULL + s),
                       64 * pn, w.qrow + qb * 128, w.h, w.tb);
         }
-        const long long roff = w.ws0 + static_cast<long long>(qb) * 128;
+        long long roff = w.ws0 + static_cast<long long>(qb) * 128;
+        if (!FA_IN_BOUNDS(p.status, roff, 128, p.ws_rows)) roff = 0;
         bulk_load(sbase + L::OFF_LD + s * 1024, p.ws_lse2 + roff, 512, bar(L::B_QFULL + s));
         bulk_load(sbase + L::OFF_LD + s * 1024 + 512, p.ws_delta + roff, 512, bar(L::B_QFULL + s));
       }
@@ -983,11 +1004,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) a[k] = bk[k] = 0u;
         }
-        if (row_ok && col < p.d_real) {
-          uint4* dvp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + w.tb * p.sdv.b +
-                                                w.h * p.sdv.h + kr * p.sdv.r + col);
-          uint4* dkp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + w.tb * p.sdk.b +
-                                                w.h * p.sdk.h + kr * p.sdk.r + col);
+        const long long dv_off = w.tb * p.sdv.b + w.h * p.sdv.h + kr * p.sdv.r + col;
+        const long long dk_off = w.tb * p.sdk.b + w.h * p.sdk.h + kr * p.sdk.r + col;
+        if (row_ok && col < p.d_real && FA_IN_BOUNDS(p.status, dv_off, 32, p.ext.dv) &&
+            FA_IN_BOUNDS(p.status, dk_off, 32, p.ext.dk)) {
+          uint4* dvp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + dv_off);
+          uint4* dkp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + dk_off);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             uint32_t vv[4], kk4[4];
@@ -1043,7 +1065,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0) mbar_arrive(bar(L::B_DQEMPTY));  // the dQ columns of TMEM are free again
         // features past d (zero columns of d = 96 / 192) are left out, whole
         // warps at a time (d is a multiple of 32)
-        if (feat < p.d_real) {
+        // (the tile's rows are consecutive: its first and last accumulator
+        // element bound every one it touches)
+        const long long acc0 = (w.ws0 + static_cast<long long>(qb) * 128) * D + feat;
+        if (feat < p.d_real && FA_IN_BOUNDS(p.status, acc0, 127ll * D + 1, p.ws_rows * D)) {
 #pragma unroll
           for (int k = 0; k < 128; ++k) red_add_f32(dst + k * D, __uint_as_float(a[k]));
         }

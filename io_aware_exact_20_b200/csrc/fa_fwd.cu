@@ -153,6 +153,10 @@ struct FwdWork {
   bool exists1, causal;
   const uint8_t* bm;
   const uint32_t* bits;  // shared-memory bitmask rows, or null
+#ifdef FA_DEBUG_BOUNDS
+  int* status;
+  long long ext_mask;
+#endif
 
   // last row of Q tile t that exists in the sequence
   __device__ __forceinline__ int last_row(int t) const { return min(q0 + 128 * t + 127, lq - 1); }
@@ -160,7 +164,10 @@ struct FwdWork {
     if (t == 1 && !exists1) return false;
     if (kb >= n_kb) return false;
     if (causal && kb * 128 > last_row(t) + off) return false;
-    if (bm != nullptr && bm[static_cast<size_t>(qb0 + t) * nbk + kb] == 0) return false;
+    if (bm != nullptr && (!FA_IN_BOUNDS(status, static_cast<long long>(qb0 + t) * nbk + kb, 1,
+                                        ext_mask) ||
+                          bm[static_cast<size_t>(qb0 + t) * nbk + kb] == 0))
+      return false;
     return true;
   }
   // kb < kb_end here (every caller walks below kb_end)
@@ -240,7 +247,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     w.off = sq.lk - sq.lq;
     w.exists1 = NQ == 2 && (w.q0 + 128) < sq.lq;
     int kv = sq.lk;
-    if (p.seqlens != nullptr) kv = max(0, min(p.seqlens[w.b], sq.lk));
+    if (p.seqlens != nullptr && FA_IN_BOUNDS(p.status, w.b, 1, p.ext.seqlens))
+      kv = max(0, min(p.seqlens[w.b], sq.lk));
     w.kv_len = kv;
     w.n_kb = (kv + 127) / 128;
     w.causal = p.causal != 0;
@@ -253,6 +261,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     w.nbk = p.nbk;
     w.bm = p.block_mask;
     w.bits = nullptr;
+#ifdef FA_DEBUG_BOUNDS
+    w.status = p.status;
+    w.ext_mask = p.ext.mask;
+#endif
   }
   constexpr int kWpr = L::BIT_WORDS / NQ;
   if (BITS && w.bm != nullptr && (w.kb_end + 31) / 32 <= kWpr) {
@@ -680,6 +692,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + w.tb * p.so.b +
                             w.h * p.so.h + static_cast<long long>(w.qrow + i) * p.so.r;
       float* lse_out = p.lse + w.tb * p.lse_sb + w.h * p.lse_sh + w.qrow + i;
+#ifdef FA_DEBUG_BOUNDS
+      const long long o_row = orow - reinterpret_cast<__nv_bfloat16*>(p.o);
+      const long long lse_off = lse_out - p.lse;
+#endif
       if constexpr (KS == 1) {
         if (ok) {
           tc_fence_after();
@@ -701,14 +717,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
                                      make_float2(inv, inv));
               ob[k] = pack_bf16(o2.x, o2.y);
             }
-            if (row_ok && 32 * c < p.d_real) {
+            if (row_ok && 32 * c < p.d_real &&
+                FA_IN_BOUNDS(p.status, o_row + 32 * c, 32, p.ext.o)) {
               uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 dst[k] = make_uint4(ob[4 * k], ob[4 * k + 1], ob[4 * k + 2], ob[4 * k + 3]);
             }
           }
-          if (row_ok) *lse_out = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+          if (row_ok && FA_IN_BOUNDS(p.status, lse_off, 1, p.ext.lse))
+            *lse_out = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
         }
       } else {
         // Merge the two streams of this Q tile.  A stream that processed no
@@ -755,14 +773,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
               const float2 o2 = fma2(x1, g1, mul2(x0, g0));
               ob[k] = pack_bf16(o2.x, o2.y);
             }
-            if (row_ok && (D / 2) * hp + 32 * c < p.d_real) {
+            if (row_ok && (D / 2) * hp + 32 * c < p.d_real &&
+                FA_IN_BOUNDS(p.status, o_row + (D / 2) * hp + 32 * c, 32, p.ext.o)) {
               uint4* dst = reinterpret_cast<uint4*>(orow + (D / 2) * hp + 32 * c);
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 dst[k] = make_uint4(ob[4 * k], ob[4 * k + 1], ob[4 * k + 2], ob[4 * k + 3]);
             }
           }
-          if (row_ok && hp == 0) *lse_out = (lt > 0.f) ? (mref + log2f(lt)) * kLn2 : -INFINITY;
+          if (row_ok && hp == 0 && FA_IN_BOUNDS(p.status, lse_off, 1, p.ext.lse))
+            *lse_out = (lt > 0.f) ? (mref + log2f(lt)) * kLn2 : -INFINITY;
         }
       }
     }

@@ -74,7 +74,28 @@ __host__ __device__ inline void grid_unit(long long u, int bh_total, int tiles, 
 }
 
 // Device status codes written to the per-device status word.
-enum : int { kStatusOk = 0, kStatusInternal = 3, kStatusTimeout = 4 };
+enum : int { kStatusOk = 0, kStatusInternal = 3, kStatusTimeout = 4, kStatusBounds = 6 };
+
+// Builds with FA_DEBUG_BOUNDS check every global-memory access the kernels
+// make outside TMA (tensor maps clip by themselves) against the extent of its
+// buffer: elements from the base pointer to one past the last element the call
+// may touch, computed on the host from the call's sizes and strides.  An access
+// out of range is skipped and kStatusBounds is recorded in the status word.
+// Other builds compile the checks away (the macro drops its arguments).
+#ifdef FA_DEBUG_BOUNDS
+struct Extents {
+  long long o, lse, dout, dq, dk, dv, mask, seqlens;
+};
+__device__ __forceinline__ bool in_bounds(int* status, long long off, long long width,
+                                          long long extent) {
+  if (off >= 0 && width >= 0 && off + width <= extent) return true;
+  if (status != nullptr) atomicExch(status, kStatusBounds);
+  return false;
+}
+#define FA_IN_BOUNDS(status, off, width, extent) ::fa::in_bounds((status), (off), (width), (extent))
+#else
+#define FA_IN_BOUNDS(status, off, width, extent) true
+#endif
 
 // Element strides of a [batch, head, row, d] view (d is contiguous).
 struct Strides {
@@ -91,6 +112,10 @@ struct Rows {
   const int32_t* cu_k;
   int nq, nk;
   int total_q, total_k;
+#ifdef FA_DEBUG_BOUNDS
+  long long n_cu;  // entries of cu_q and cu_k (B + 1)
+  int* status;
+#endif
 };
 
 // One batch entry resolved: first row and length of its queries and keys, and
@@ -109,6 +134,7 @@ __device__ __forceinline__ Seq seq_of(const Rows& r, int b) {
     s.lk = r.nk;
     s.tb = b;
   } else {
+    if (!FA_IN_BOUNDS(r.status, b, 2, r.n_cu)) return Seq{0, 0, 0, 0, 0};
     const int a0 = min(max(r.cu_q[b], 0), r.total_q);
     const int a1 = min(max(r.cu_q[b + 1], a0), r.total_q);
     const int c0 = min(max(r.cu_k[b], 0), r.total_k);
@@ -142,6 +168,9 @@ struct FwdParams {
   PhiloxRoundKeys rk;         // round keys of the dropout generator
   uint64_t timeout_ns;
   int mask_bitmap;            // block masks: 1 = walk them through a shared-memory bitmask
+#ifdef FA_DEBUG_BOUNDS
+  Extents ext;
+#endif
 };
 
 struct BwdParams {
@@ -179,6 +208,9 @@ struct BwdParams {
   PhiloxRoundKeys rk;
   uint64_t timeout_ns;
   int mask_bitmap;            // as in FwdParams
+#ifdef FA_DEBUG_BOUNDS
+  Extents ext;
+#endif
 };
 
 // First workspace row of (b, h); a multiple of 128.  Packed sequences are

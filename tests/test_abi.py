@@ -33,6 +33,10 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_status_strings(lib):
     so = lib.library()
+    assert so.fa_status_string(6).startswith(b"a kernel index was out of bounds")
+    # the default library is the production build (no bounds checks)
+    if not os.environ.get("FA_B200_LIBRARY"):
+        assert so.fa_debug_bounds_checking() == 0
     assert so.fa_status_string(0) == b"ok"
     assert so.fa_status_string(5).startswith(b"workspace")
     assert so.fa_status_string(99) == b"unknown status"
