@@ -15,6 +15,7 @@ tensors of layout [B, H, N, d].
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 from .build import LIB_PATH
@@ -24,7 +25,7 @@ __all__ = [
     "forward_general", "backward_general", "general_workspace_size",
     "merge_partial", "accumulate_bf16", "convert_f32_bf16", "qkv_projection",
     "dropout_mask", "last_device_status", "set_wait_timeout_ns", "set_block_mask_bitmap",
-    "wait_timeout_probe", "STATUS",
+    "wait_timeout_probe", "set_nvtx", "STATUS",
 ]
 
 STATUS = {
@@ -34,7 +35,36 @@ STATUS = {
     3: "FA_ERR_CUDA",
     4: "FA_ERR_TIMEOUT",
     5: "FA_ERR_WORKSPACE",
+    6: "FA_ERR_BOUNDS",
 }
+
+
+# NVTX ranges around the entry points below, for timeline profilers: off unless
+# FA_NVTX is set to a non-zero value or set_nvtx(True) is called.
+_NVTX = os.environ.get("FA_NVTX", "0") not in ("", "0")
+
+
+def set_nvtx(enabled):
+    """Marks each call of the entry points with an NVTX range ("fa.forward",
+    "fa.backward", ...) when enabled."""
+    global _NVTX
+    _NVTX = bool(enabled)
+
+
+def _nvtx(name):
+    def deco(fn):
+        @functools.wraps(fn)
+        def wrapped(*args, **kwargs):
+            if not _NVTX:
+                return fn(*args, **kwargs)
+            import torch
+            torch.cuda.nvtx.range_push(name)
+            try:
+                return fn(*args, **kwargs)
+            finally:
+                torch.cuda.nvtx.range_pop()
+        return wrapped
+    return deco
 
 
 class FaError(RuntimeError):
@@ -159,6 +189,7 @@ def _masks(seqlens, block_mask, device):
     return sl, bm
 
 
+@_nvtx("fa.forward")
 def forward(q, k, v, scale=None, causal=False, seqlens=None, dropout_p=0.0, seed=0,
             block_mask=None, out=None, lse=None):
     """O, LSE = attention(q, k, v) for bf16 CUDA tensors [B, H, N, d]."""
@@ -183,6 +214,7 @@ def bwd_workspace_size(B, H, N, d):
     return int(library().fa_bwd_workspace_size(B, H, N, d))
 
 
+@_nvtx("fa.backward")
 def backward(q, k, v, o, lse, dout, scale=None, causal=False, seqlens=None, dropout_p=0.0,
              seed=0, block_mask=None, workspace=None, dq=None, dk=None, dv=None):
     """dQ, dK, dV of attention for bf16 CUDA tensors [B, H, N, d]."""
@@ -208,6 +240,7 @@ def backward(q, k, v, o, lse, dout, scale=None, causal=False, seqlens=None, drop
     return dq, dk, dv
 
 
+@_nvtx("fa.backward_phases")
 def backward_phases(q, k, v, o, lse, dout, scale=None, causal=False, seqlens=None,
                     dropout_p=0.0, seed=0, block_mask=None, workspace=None, dq=None, dk=None,
                     dv=None):
@@ -360,6 +393,7 @@ def _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, 
     return a, keep
 
 
+@_nvtx("fa.forward_general")
 def forward_general(q, k, v, *, layout="bhsd", cu_seqlens_q=None, cu_seqlens_k=None,
                     max_seqlen_q=None, max_seqlen_k=None, scale=None, causal=False,
                     seqlens_k=None, dropout_p=0.0, seed=0, block_mask=None, out=None, lse=None):
@@ -413,6 +447,7 @@ def general_workspace_size(q, k, **kw):
     return int(library().fa_bwd_ex_workspace_size(ctypes.byref(a)))
 
 
+@_nvtx("fa.backward_general")
 def backward_general(q, k, v, o, lse, dout, *, layout="bhsd", cu_seqlens_q=None,
                      cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None, scale=None,
                      causal=False, seqlens_k=None, dropout_p=0.0, seed=0, block_mask=None,
@@ -444,6 +479,7 @@ def backward_general(q, k, v, o, lse, dout, *, layout="bhsd", cu_seqlens_q=None,
 # combining partial results (context-parallel attention)
 # ---------------------------------------------------------------------------
 
+@_nvtx("fa.merge_partial")
 def merge_partial(o_acc, lse_acc, o_part, lse_part):
     """o_acc (fp32 [..., d]), lse_acc (fp32 [...]) <- merge with the partial
     result o_part (bf16 [..., d]), lse_part (fp32 [...]); in place."""
@@ -460,6 +496,7 @@ def merge_partial(o_acc, lse_acc, o_part, lse_part):
                                       rows, d, _stream_ptr(o_acc.device)), "fa_merge_partial")
 
 
+@_nvtx("fa.accumulate_bf16")
 def accumulate_bf16(acc, part):
     """acc (fp32) += part (bf16), elementwise, in place."""
     import torch
@@ -471,6 +508,7 @@ def accumulate_bf16(acc, part):
                                         _stream_ptr(acc.device)), "fa_accumulate_bf16")
 
 
+@_nvtx("fa.convert_f32_bf16")
 def convert_f32_bf16(src, out=None):
     """bf16 copy of an fp32 tensor (round to nearest even)."""
     import torch
@@ -486,6 +524,7 @@ def convert_f32_bf16(src, out=None):
 # fused QKV projection
 # ---------------------------------------------------------------------------
 
+@_nvtx("fa.qkv_projection")
 def qkv_projection(x, weight, bias, batch, heads, head_dim, q=None, k=None, v=None):
     """Q, K, V [B, H, N, d] = split_heads(x @ weight.T + bias) in one kernel.
 

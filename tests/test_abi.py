@@ -202,3 +202,26 @@ def test_merge_partial_head_dims(lib):
         assert so.fa_merge_partial(A16, A16, A16, A16, 0, d, None) == 0, d
     for d in (16, 80, 160, 320, 512):
         assert so.fa_merge_partial(A16, A16, A16, A16, 5, d, None) == 2, d
+
+
+def test_nvtx_ranges_wrap_the_entry_points(lib, monkeypatch):
+    """With NVTX on, an entry point runs inside a range named after it, popped
+    even when the call raises; off (the default), no range is pushed."""
+    import torch
+    calls = []
+    monkeypatch.setattr(torch.cuda.nvtx, "range_push", lambda name: calls.append(("push", name)))
+    monkeypatch.setattr(torch.cuda.nvtx, "range_pop", lambda: calls.append(("pop",)))
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)  # host tensors: refused before any launch
+    lib.set_nvtx(True)
+    try:
+        with pytest.raises(ValueError):
+            lib.forward(q, q, q)
+        with pytest.raises(ValueError):
+            lib.forward_general(q, q, q)
+    finally:
+        lib.set_nvtx(False)
+    assert calls == [("push", "fa.forward"), ("pop",), ("push", "fa.forward_general"), ("pop",)]
+    calls.clear()
+    with pytest.raises(ValueError):
+        lib.forward(q, q, q)
+    assert calls == []
