@@ -355,7 +355,7 @@ def merge_partials(o_a, lse_a, o_b, lse_b):
 
 
 def head_backward_block(q, k, v, dout, lse, delta, scale, causal=False, n_q=None, n_k=None,
-                        q0=0, k0=0):
+                        q0=0, k0=0, dropout_p=0.0, seed=0, b=0, h=0):
     """The part of one head's backward that comes from one block of keys,
     given the softmax statistics of the full row (its LSE and
     D_i = sum_c dO_ic O_ic over all keys): with P = exp(scale Q K_blk^T - LSE),
@@ -367,7 +367,10 @@ def head_backward_block(q, k, v, dout, lse, delta, scale, causal=False, n_q=None
     of the pages needs only LSE and D per row: suanlizi.com summary, 重计算).
     q, dout: [R, d] rows q0 .. of a sequence of n_q queries; k, v: [C, d] keys
     k0 .. of n_k keys; causal (bottom-right): key j valid iff j <= i + n_k - n_q.
-    No dropout."""
+    Dropout (the inverted dropout of attention_forward, keep bits Z keyed by the
+    rows' and keys' positions in the sequence, q0 + i and k0 + j, of (b, h)):
+    dV_blk = (P Z / q)^T dO and dP = (dO V_blk^T) Z / q, q the keep
+    probability, while dS = P (dP - D) keeps the undropped P."""
     q, k, v, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
     rows = q0 + np.arange(q.shape[0])[:, None]
     cols = k0 + np.arange(k.shape[0])[None, :]
@@ -379,6 +382,11 @@ def head_backward_block(q, k, v, dout, lse, delta, scale, causal=False, n_q=None
     with np.errstate(invalid="ignore"):
         p = np.where(valid & np.isfinite(lse), np.exp(s - np.where(np.isfinite(lse), lse, 0.0)),
                      0.0)
-    dp = dout @ v.T
+    p32 = float(np.float32(dropout_p))
+    z, rscale = 1.0, 1.0
+    if p32 > 0:
+        z = dropout_keep(seed, p32, b, h, q0 + np.arange(q.shape[0]), k.shape[0], k0)
+        z, rscale = z.astype(np.float64), dropout_scale(p32)
+    dp = (dout @ v.T) * z * rscale
     ds = p * (dp - np.asarray(delta, dtype=np.float64)[:, None])
-    return scale * (ds @ k), scale * (ds.T @ q), p.T @ dout
+    return scale * (ds @ k), scale * (ds.T @ q), (p * z * rscale).T @ dout

@@ -800,19 +800,24 @@ def test_merge_with_empty_parts():
     assert (o4 == 0).all() and np.isneginf(l4).all()
 
 
-@pytest.mark.parametrize("causal", [False, True])
-def test_block_backward_sums_to_the_full_backward(causal):
+@pytest.mark.parametrize("causal,p", [(False, 0.0), (True, 0.0), (False, 0.2), (True, 0.3)])
+def test_block_backward_sums_to_the_full_backward(causal, p):
     """The per-key-block backward given the full rows' LSE and D, summed over
     blocks (query blocks x key blocks), equals the full backward: the
-    decomposition a context-parallel ring uses.  Dropping the D term, using
-    the block's own LSE or a wrong causal offset fails."""
-    from oracle import head_backward_block
+    decomposition a context-parallel ring uses, with dropout too (each block
+    keys its bits by the rows' and keys' positions in the sequence).  Dropping
+    the D term, using the block's own LSE, a wrong causal offset or bits keyed
+    by positions inside the block fails."""
+    from oracle import attention_backward, head_backward_block
     rng = np.random.default_rng(63)
-    W, n, d, scale = 3, 40, 8, 0.45
+    W, n, d, scale, seed = 3, 40, 8, 0.45, 0x5EED
     N = W * n
     q, k, v, do = (_rand((N, d), rng) for _ in range(4))
-    dq, dk, dv, _ = head_backward(q, k, v, do, scale, causal)
-    o, lse = attention_forward(q[None, None], k[None, None], v[None, None], scale, causal)
+    o, lse = attention_forward(q[None, None], k[None, None], v[None, None], scale, causal,
+                               dropout_p=p, seed=seed)
+    full = attention_backward(q[None, None], k[None, None], v[None, None], do[None, None], scale,
+                              causal, None, p, seed)
+    dq, dk, dv = (x[0, 0] for x in full)
     delta = (do * o[0, 0]).sum(axis=1)
     gq, gk, gv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     for r in range(W):
@@ -820,7 +825,7 @@ def test_block_backward_sums_to_the_full_backward(causal):
         for c in range(W):
             cs = slice(c * n, (c + 1) * n)
             a, b, e = head_backward_block(q[rs], k[cs], v[cs], do[rs], lse[0, 0, rs], delta[rs],
-                                          scale, causal, N, N, r * n, c * n)
+                                          scale, causal, N, N, r * n, c * n, p, seed)
             gq[rs] += a
             gk[cs] += b
             gv[cs] += e
