@@ -209,6 +209,14 @@ typedef struct {
   uint64_t seed;
   const uint8_t* block_mask;
   fa_strides_t q, k, v, o, dout, dq, dk, dv;
+  /* Dropout positions: this call's query rows are rows dropout_row0 .. and its
+   * keys keys dropout_key0 .. of the sequence the keep bits are keyed by (the
+   * call evaluates one block of a longer sequence, as in a context-parallel
+   * ring); 0, 0 for a whole sequence.  Both >= 0, dropout_key0 a multiple of
+   * 8 (one Philox call covers 8 keys), dropout_row0 + seqlen_q and
+   * dropout_key0 + seqlen_k at most 2^31 - 1; otherwise FA_ERR_INVALID_ARG.
+   * The masks are not moved: they stay relative to the call's own rows. */
+  int64_t dropout_row0, dropout_key0;
 } fa_attention_desc_t;
 
 /* Forward pass for a general layout.  LSE is fp32 [B, H, seqlen_q]
@@ -220,8 +228,8 @@ fa_status_t fa_fwd_ex(const fa_attention_desc_t* desc, const void* q, const void
 
 /* Workspace bytes of fa_bwd_ex: padded layout B * H * ceil(seqlen_q / 128) * 128
  * rows, packed layout H * (ceil(total_q / 128) * 128 + 256 B) rows, each of
- * 8 + 4 D bytes (D = 64 for d <= 64, else 128).  0 if the description is
- * invalid. */
+ * 8 + 4 D bytes (D = 64 for d <= 64, 128 for d = 96 / 128, 256 for d = 192 /
+ * 256).  0 if the description is invalid. */
 size_t fa_bwd_ex_workspace_size(const fa_attention_desc_t* desc);
 
 /* Backward pass for a general layout (dQ like Q, dK / dV like K / V; the

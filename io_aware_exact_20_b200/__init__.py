@@ -95,6 +95,7 @@ class AttentionDesc(ctypes.Structure):
         ("block_mask", ctypes.c_void_p),
         ("q", Strides), ("k", Strides), ("v", Strides), ("o", Strides), ("dout", Strides),
         ("dq", Strides), ("dk", Strides), ("dv", Strides),
+        ("dropout_row0", ctypes.c_int64), ("dropout_key0", ctypes.c_int64),
     ]
 
 
@@ -343,7 +344,7 @@ _Q_SIDE = ("q", "o", "dout", "dq")
 
 
 def _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, scale, causal,
-          seqlens_k, dropout_p, seed, block_mask, tensors):
+          seqlens_k, dropout_p, seed, block_mask, tensors, dropout_pos=(0, 0)):
     import torch
     if layout not in ("bhsd", "bshd", "thd"):
         raise ValueError(f"unknown layout {layout!r}")
@@ -388,6 +389,7 @@ def _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, 
     a.causal = int(bool(causal))
     a.dropout_p = float(dropout_p)
     a.seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+    a.dropout_row0, a.dropout_key0 = (int(x) for x in dropout_pos)
     for name, t in tensors.items():
         setattr(a, name, _strides(t, layout))
     return a, keep
@@ -396,7 +398,8 @@ def _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, 
 @_nvtx("fa.forward_general")
 def forward_general(q, k, v, *, layout="bhsd", cu_seqlens_q=None, cu_seqlens_k=None,
                     max_seqlen_q=None, max_seqlen_k=None, scale=None, causal=False,
-                    seqlens_k=None, dropout_p=0.0, seed=0, block_mask=None, out=None, lse=None):
+                    seqlens_k=None, dropout_p=0.0, seed=0, block_mask=None, out=None, lse=None,
+                    dropout_row0=0, dropout_key0=0):
     """O, LSE for a general layout (fa_fwd_ex).
 
     layout "bhsd": q [B, H, N_q, d], k / v [B, H, N_k, d]; "bshd": q [B, N_q, H, d],
@@ -404,13 +407,16 @@ def forward_general(q, k, v, *, layout="bhsd", cu_seqlens_q=None, cu_seqlens_k=N
     offsets cu_seqlens_q / cu_seqlens_k ([B + 1]) and the longest lengths.  Any
     strides with d contiguous (multiples of 8 elements).  The causal mask is
     bottom-right aligned per sequence.  LSE: [B, H, N_q] or [H, T_q] (packed).
+    dropout_row0 / dropout_key0: positions of the call's first query row and
+    first key in the sequence the dropout bits are keyed by (a block of a
+    longer sequence); the key position a multiple of 8.
     """
     import torch
     if out is None:
         out = torch.empty_like(q)
     a, keep = _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, scale,
                     causal, seqlens_k, dropout_p, seed, block_mask,
-                    dict(q=q, k=k, v=v, o=out))
+                    dict(q=q, k=k, v=v, o=out), (dropout_row0, dropout_key0))
     if lse is None:
         lse = torch.empty(_lse_shape(q, layout), dtype=torch.float32, device=q.device)
     _check_lse(lse, q, layout)
@@ -451,7 +457,7 @@ def general_workspace_size(q, k, **kw):
 def backward_general(q, k, v, o, lse, dout, *, layout="bhsd", cu_seqlens_q=None,
                      cu_seqlens_k=None, max_seqlen_q=None, max_seqlen_k=None, scale=None,
                      causal=False, seqlens_k=None, dropout_p=0.0, seed=0, block_mask=None,
-                     workspace=None, dq=None, dk=None, dv=None):
+                     workspace=None, dq=None, dk=None, dv=None, dropout_row0=0, dropout_key0=0):
     """dQ, dK, dV for a general layout (fa_bwd_ex); arguments as forward_general."""
     import torch
     dq = torch.empty_like(q) if dq is None else dq
@@ -459,7 +465,8 @@ def backward_general(q, k, v, o, lse, dout, *, layout="bhsd", cu_seqlens_q=None,
     dv = torch.empty_like(v) if dv is None else dv
     a, keep = _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, scale,
                     causal, seqlens_k, dropout_p, seed, block_mask,
-                    dict(q=q, k=k, v=v, o=o, dout=dout, dq=dq, dk=dk, dv=dv))
+                    dict(q=q, k=k, v=v, o=o, dout=dout, dq=dq, dk=dk, dv=dv),
+                    (dropout_row0, dropout_key0))
     _check_lse(lse, q, layout)
     lib = library()
     need = int(lib.fa_bwd_ex_workspace_size(ctypes.byref(a)))

@@ -18,9 +18,11 @@ computed on), so that every rank meets every chunk once:
 
 Under the causal mask chunk c is skipped by rank r when c > r (every pair
 masked) and computed with the causal mask when c = r (equal chunk sizes, so
-the bottom-right alignment is the usual one); c < r is unmasked.  Dropout is
-not offered here: its keep bits are keyed by positions inside the sequence and
-the kernels see chunk positions.
+the bottom-right alignment is the usual one); c < r is unmasked.  Dropout keys
+its bits by positions in the whole sequence: every call tells the kernels the
+positions of its first query row (r N / W) and first key (c N / W), so the
+ring draws exactly the bits of the unsplit attention (the chunk length must
+then be a multiple of 8, the keys of one generator call).
 
 Every arithmetic step runs in the library's kernels (fa_fwd_ex, fa_bwd_ex,
 fa_merge_partial, fa_accumulate_bf16, fa_convert_f32_bf16); torch supplies the
@@ -44,11 +46,16 @@ class LibraryKernels:
             import io_aware_exact_20_b200 as fa
         self.fa = fa
 
-    def forward(self, q, k, v, scale, causal):
-        return self.fa.forward_general(q, k, v, scale=scale, causal=causal)
+    def forward(self, q, k, v, scale, causal, drop=None):
+        """drop: None, or (dropout_p, seed, position of q's first row, of k's first key)."""
+        kw = {} if drop is None else dict(dropout_p=drop[0], seed=drop[1], dropout_row0=drop[2],
+                                          dropout_key0=drop[3])
+        return self.fa.forward_general(q, k, v, scale=scale, causal=causal, **kw)
 
-    def backward(self, q, k, v, o, lse, do, scale, causal):
-        return self.fa.backward_general(q, k, v, o, lse, do, scale=scale, causal=causal)
+    def backward(self, q, k, v, o, lse, do, scale, causal, drop=None):
+        kw = {} if drop is None else dict(dropout_p=drop[0], seed=drop[1], dropout_row0=drop[2],
+                                          dropout_key0=drop[3])
+        return self.fa.backward_general(q, k, v, o, lse, do, scale=scale, causal=causal, **kw)
 
     def zeros_acc(self, like):
         import torch
@@ -68,10 +75,20 @@ class LibraryKernels:
         return self.fa.convert_f32_bf16(acc)
 
 
-def ring_forward(rank, world, q, k, v, scale, causal, kern):
+def _drop(dropout_p, seed, rank, c, n):
+    """The kernels' dropout argument for queries of chunk `rank`, keys of chunk c."""
+    if not dropout_p:
+        return None
+    if n % 8:
+        raise ValueError("dropout in the ring needs a chunk length that is a multiple of 8")
+    return (dropout_p, seed, rank * n, c * n)
+
+
+def ring_forward(rank, world, q, k, v, scale, causal, kern, dropout_p=0.0, seed=0):
     """Generator of one rank's forward.  Yields ("start", tensors): send them to
     rank + 1 and answer with same-shaped buffers that will receive rank - 1's;
     then ("wait",): answer once those have arrived.  Returns (O, LSE)."""
+    n = q.shape[-2]
     o_acc = kern.zeros_acc(q)
     lse_acc = kern.empty_lse(q)
     cur = [k, v]
@@ -80,7 +97,8 @@ def ring_forward(rank, world, q, k, v, scale, causal, kern):
         last = s + 1 == world
         nxt = None if last else (yield ("start", cur))
         if not causal or c <= rank:
-            o_p, l_p = kern.forward(q, cur[0], cur[1], scale, causal and c == rank)
+            o_p, l_p = kern.forward(q, cur[0], cur[1], scale, causal and c == rank,
+                                    _drop(dropout_p, seed, rank, c, n))
             kern.merge(o_acc, lse_acc, o_p, l_p)
         if not last:
             yield ("wait",)
@@ -88,9 +106,10 @@ def ring_forward(rank, world, q, k, v, scale, causal, kern):
     return kern.finish(o_acc), lse_acc
 
 
-def ring_backward(rank, world, q, k, v, o, lse, do, scale, causal, kern):
+def ring_backward(rank, world, q, k, v, o, lse, do, scale, causal, kern, dropout_p=0.0, seed=0):
     """Generator of one rank's backward (same protocol as ring_forward).
     Returns (dQ, dK, dV) of this rank's chunk."""
+    n = q.shape[-2]
     dq_acc = kern.zeros_acc(q)
     acc = [kern.zeros_acc(k), kern.zeros_acc(v)]  # dK, dV of the chunk held now
     cur = [k, v]
@@ -100,7 +119,8 @@ def ring_backward(rank, world, q, k, v, o, lse, do, scale, causal, kern):
         nxt = None if last else (yield ("start", cur))
         if not causal or c <= rank:
             dq_p, dk_p, dv_p = kern.backward(q, cur[0], cur[1], o, lse, do, scale,
-                                             causal and c == rank)
+                                             causal and c == rank,
+                                             _drop(dropout_p, seed, rank, c, n))
             kern.accumulate(dq_acc, dq_p)
             kern.accumulate(acc[0], dk_p)
             kern.accumulate(acc[1], dv_p)
@@ -175,19 +195,22 @@ def run_emulated(gens):
     return results
 
 
-def attention_forward(q, k, v, scale=None, causal=False, group=None, kern=None):
+def attention_forward(q, k, v, scale=None, causal=False, group=None, kern=None, dropout_p=0.0,
+                      seed=0):
     """This rank's chunk of O and LSE: q, k, v are its [B, H, N / W, d] chunks."""
     import torch.distributed as dist
     kern = kern or LibraryKernels()
     scale = q.shape[-1] ** -0.5 if scale is None else scale
     return run_ring(ring_forward(dist.get_rank(group), dist.get_world_size(group), q, k, v,
-                                 scale, causal, kern), group)
+                                 scale, causal, kern, dropout_p, seed), group)
 
 
-def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, group=None, kern=None):
-    """This rank's chunk of dQ, dK, dV (O, LSE from attention_forward)."""
+def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, group=None, kern=None,
+                       dropout_p=0.0, seed=0):
+    """This rank's chunk of dQ, dK, dV (O, LSE from attention_forward; the
+    same dropout_p and seed)."""
     import torch.distributed as dist
     kern = kern or LibraryKernels()
     scale = q.shape[-1] ** -0.5 if scale is None else scale
     return run_ring(ring_backward(dist.get_rank(group), dist.get_world_size(group), q, k, v, o,
-                                  lse, do, scale, causal, kern), group)
+                                  lse, do, scale, causal, kern, dropout_p, seed), group)

@@ -78,6 +78,7 @@ struct Problem {
   uint64_t seed;
   const uint8_t* block_mask;
   fa_strides_t q, k, v, o, dout, dq, dk, dv;
+  int64_t drop_row0, drop_key0;  // dropout positions of the first query row and key
 
   int rows_q() const { return packed ? total_q : nq; }
   int rows_k() const { return packed ? total_k : nk; }
@@ -128,6 +129,12 @@ fa_status_t resolve(const fa_attention_desc_t* a, Problem* p, Uses uses) {
         s->row == 0)
       return FA_ERR_INVALID_ARG;
   }
+  // dropout positions: counter words are 32-bit, keys go in groups of 8
+  if (a->dropout_row0 < 0 || a->dropout_key0 < 0 || a->dropout_key0 % 8 != 0 ||
+      a->dropout_row0 > 0x7FFFFFFFll - a->seqlen_q || a->dropout_key0 > 0x7FFFFFFFll - a->seqlen_k)
+    return FA_ERR_INVALID_ARG;
+  p->drop_row0 = a->dropout_row0;
+  p->drop_key0 = a->dropout_key0;
   p->B = a->batch;
   p->H = a->heads;
   p->d = a->head_dim;
@@ -307,6 +314,8 @@ fa_status_t run_fwd(const Problem& pr, const void* q, const void* k, const void*
   p.seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
   p.seed_hi = static_cast<uint32_t>(pr.seed >> 32);
   p.rk = fa::philox_round_keys(pr.seed);
+  p.drop_row0 = static_cast<uint32_t>(pr.drop_row0);
+  p.drop_kgrp0 = static_cast<uint32_t>(pr.drop_key0 / 8);
   p.timeout_ns = g_timeout_ns.load();
   p.mask_bitmap = g_mask_bitmap.load();
 #ifdef FA_DEBUG_BOUNDS
@@ -360,6 +369,8 @@ fa_status_t bwd_params(fa::BwdParams* p, const Problem& pr, const void* workspac
   p->seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
   p->seed_hi = static_cast<uint32_t>(pr.seed >> 32);
   p->rk = fa::philox_round_keys(pr.seed);
+  p->drop_row0 = static_cast<uint32_t>(pr.drop_row0);
+  p->drop_kgrp0 = static_cast<uint32_t>(pr.drop_key0 / 8);
   p->timeout_ns = g_timeout_ns.load();
   p->mask_bitmap = g_mask_bitmap.load();
 #ifdef FA_DEBUG_BOUNDS

@@ -266,7 +266,9 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
 // main kernel
 // ---------------------------------------------------------------------------
 
-template <int D, bool DROPOUT, bool BITS>
+// POS as in the forward kernel: dropout counters offset by the call's row /
+// key positions (instantiated only with dropout and the direct mask walk).
+template <int D, bool DROPOUT, bool BITS, bool POS = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -764,8 +766,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t own = 0u;
 #pragma unroll
           for (int gq = 0; gq < 4; ++gq) {
-            const uint32_t qg = static_cast<uint32_t>(qb * 128 + qoff + 8 * gq + (lane & 7));
-            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>(jg >> 3), qg,
+            const uint32_t qg = (POS ? p.drop_row0 : 0u) +
+                                static_cast<uint32_t>(qb * 128 + qoff + 8 * gq + (lane & 7));
+            const Philox4 rnd = philox4x32_10((POS ? p.drop_kgrp0 : 0u) + static_cast<uint32_t>(jg >> 3), qg,
                                               static_cast<uint32_t>(w.h), static_cast<uint32_t>(w.b),
                                               p.rk);
             own |= keep_byte(rnd, thr) << (8 * gq);
@@ -1137,13 +1140,13 @@ cudaError_t launch_pre_t(const BwdParams& p, cudaStream_t stream) {
   return launch_overlapped(bwd_pre_kernel<D>, prepost_grid<D>(p), dim3(256), 0, stream, p);
 }
 
-template <int D, bool DROPOUT, bool BITS>
+template <int D, bool DROPOUT, bool BITS, bool POS = false>
 cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdParams& p,
                           cudaStream_t stream) {
   using L = BwdLayout<D>;
   static_assert(!BITS || L::BIT_WORDS > 0, "no bitmask at this head dim");
-  auto kern = bwd_main_kernel<D, DROPOUT, BITS>;
+  auto kern = bwd_main_kernel<D, DROPOUT, BITS, POS>;
   // The setmaxnreg split (d = 128) is sized for exactly 128 registers per
   // thread at launch; with any other count an increase could wait forever.
   static OncePerContext prepared;
@@ -1183,6 +1186,12 @@ cudaError_t launch_bwd_pre(int d, const BwdParams& p, cudaStream_t stream) {
 cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdq,
                             const BwdParams& p, cudaStream_t stream) {
+  if (dropout && (p.drop_row0 != 0u || p.drop_kgrp0 != 0u)) {  // a block of a longer sequence
+    if (d == 64) return launch_main_t<64, true, false, true>(tq, tk, tv, tdo, tdq, p, stream);
+    if (d == 128) return launch_main_t<128, true, false, true>(tq, tk, tv, tdo, tdq, p, stream);
+    if (d == 256) return launch_main_t<256, true, false, true>(tq, tk, tv, tdo, tdq, p, stream);
+    return cudaErrorInvalidValue;
+  }
   if (d == 64) {
     // a block mask whose columns fit the bitmask (the CTAs' query tiles are
     // below the longest sequence's)

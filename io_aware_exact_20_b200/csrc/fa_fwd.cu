@@ -203,7 +203,10 @@ __device__ __forceinline__ void named_bar_sync() {
   asm volatile("bar.sync %0, 256;" ::"n"(kId) : "memory");
 }
 
-template <int D, bool DROPOUT, bool BITS>
+// POS: the dropout counter is offset by the call's row / key positions in a
+// longer sequence (instantiated only with dropout and the direct mask walk; the
+// other instances see compile-time zeros).
+template <int D, bool DROPOUT, bool BITS, bool POS = false>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -636,9 +639,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
           const uint32_t thr_hi = thr << 16;
 #pragma unroll
           for (int gq = 0; gq < KW / 8; ++gq) {
-            const Philox4 rnd = philox4x32_10(static_cast<uint32_t>((j0 >> 3) + gq),
-                                              static_cast<uint32_t>(i), static_cast<uint32_t>(w.h),
-                                              static_cast<uint32_t>(w.b), p.rk);
+            const Philox4 rnd = philox4x32_10(
+                (POS ? p.drop_kgrp0 : 0u) + static_cast<uint32_t>((j0 >> 3) + gq),
+                (POS ? p.drop_row0 : 0u) + static_cast<uint32_t>(i), static_cast<uint32_t>(w.h),
+                static_cast<uint32_t>(w.b), p.rk);
             const uint32_t wv[4] = {rnd.w0, rnd.w1, rnd.w2, rnd.w3};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -797,12 +801,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   }
 }
 
-template <int D, bool DROPOUT, bool BITS>
+template <int D, bool DROPOUT, bool BITS, bool POS = false>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, cudaStream_t stream) {
   using L = FwdLayout<D>;
   using C = FwdCfg<D>;
-  auto kern = fwd_kernel<D, DROPOUT, BITS>;
+  auto kern = fwd_kernel<D, DROPOUT, BITS, POS>;
   // The setmaxnreg split is sized for exactly LAUNCH_REGS registers per thread
   // at launch; with any other count an increase could wait forever.  Checked,
   // with the shared-memory attribute set, once per device and context.
@@ -836,6 +840,12 @@ bool uses_bits(const FwdParams& p) {
 
 cudaError_t launch_fwd(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const FwdParams& p, cudaStream_t stream) {
+  if (dropout && (p.drop_row0 != 0u || p.drop_kgrp0 != 0u)) {  // a block of a longer sequence
+    if (d == 64) return launch_fwd_t<64, true, false, true>(tq, tk, tv, p, stream);
+    if (d == 128) return launch_fwd_t<128, true, false, true>(tq, tk, tv, p, stream);
+    if (d == 256) return launch_fwd_t<256, true, false, true>(tq, tk, tv, p, stream);
+    return cudaErrorInvalidValue;
+  }
   if (d == 64) {
     if (uses_bits<64>(p))
       return dropout ? launch_fwd_t<64, true, true>(tq, tk, tv, p, stream)

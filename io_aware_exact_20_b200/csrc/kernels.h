@@ -166,6 +166,8 @@ struct FwdParams {
   float drop_rscale;          // 1 / (1 - p)
   uint32_t seed_lo, seed_hi;
   PhiloxRoundKeys rk;         // round keys of the dropout generator
+  uint32_t drop_row0;         // dropout counter: position of the call's row 0 ...
+  uint32_t drop_kgrp0;        // ... and 8-key group of its key 0 in the keyed sequence
   uint64_t timeout_ns;
   int mask_bitmap;            // block masks: 1 = walk them through a shared-memory bitmask
 #ifdef FA_DEBUG_BOUNDS
@@ -206,6 +208,7 @@ struct BwdParams {
   float drop_rscale;
   uint32_t seed_lo, seed_hi;
   PhiloxRoundKeys rk;
+  uint32_t drop_row0, drop_kgrp0;  // as in FwdParams
   uint64_t timeout_ns;
   int mask_bitmap;            // as in FwdParams
 #ifdef FA_DEBUG_BOUNDS

@@ -122,6 +122,11 @@ def _desc(lib, **kw):
     (dict(k=(3 * 384 * 64, 0, 64)), 1),                     # heads sharing memory
     (dict(o=(0, 256 * 64, 64)), 1),                         # batch entries sharing memory
     (dict(seqlen_q=(1 << 23) + 1), 2),
+    (dict(dropout_row0=128, dropout_key0=64), None),       # valid dropout positions
+    (dict(dropout_key0=4), 1),                             # not a multiple of 8
+    (dict(dropout_row0=-1), 1), (dict(dropout_key0=-8), 1),
+    (dict(dropout_row0=(1 << 31) - 256), 1),               # row0 + seqlen_q past 2^31 - 1
+    (dict(dropout_key0=(1 << 40)), 1),
 ])
 def test_general_entry_points_validate_before_launching(lib, change, code):
     so = lib.library()

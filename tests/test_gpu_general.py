@@ -229,3 +229,37 @@ def test_packed_equals_padded_with_key_lengths(lib):
     assert (pack(o_pad) - o).abs().max().item() == 0.0  # same tiles, same arithmetic
     assert rel_l2(f64(pack(dk_pad)), f64(dk)) < 1e-2
     assert rel_l2(f64(pack(dv_pad)), f64(dv)) < 1e-2
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_dropout_positions_of_a_block(lib, parity_record, d):
+    """A call that evaluates one block of a longer sequence (queries at
+    positions 256.., keys at 128..) with dropout keys its bits by those
+    positions: O, LSE and the gradients equal the oracle's for the same
+    block with the same positions (its own softmax over the block's keys)."""
+    import torch
+    from oracle import head_backward_block, head_forward_rows
+    B, H, Nq, Nk, row0, key0, p, seed = 1, 2, 200, 328, 256, 128, 0.2, 0x5EED0099
+    qh, doh = randn((B, H, Nq, d), 31), randn((B, H, Nq, d), 32)
+    kh, vh = randn((B, H, Nk, d), 33), randn((B, H, Nk, d), 34)
+    scale = d ** -0.5
+    kw = dict(scale=scale, dropout_p=p, seed=seed, dropout_row0=row0, dropout_key0=key0)
+    q, k, v, do = (x.cuda() for x in (qh, kh, vh, doh))
+    o, lse = lib.forward_general(q, k, v, **kw)
+    dq, dk, dv = lib.backward_general(q, k, v, o, lse, do, **kw)
+    torch.cuda.synchronize()
+    assert lib.last_device_status() == 0
+    ro, rl = np.zeros((B, H, Nq, d)), np.zeros((B, H, Nq))
+    rg = [np.zeros((B, H, Nq, d)), np.zeros((B, H, Nk, d)), np.zeros((B, H, Nk, d))]
+    for h in range(H):
+        a = [f64(x)[0, h] for x in (qh, kh, vh, doh)]
+        ro[0, h], rl[0, h] = head_forward_rows(a[0], a[1], a[2], scale, np.arange(Nq),
+                                               dropout_p=p, seed=seed, b=0, h=h, row0=row0,
+                                               key0=key0)
+        delta = (a[3] * ro[0, h]).sum(-1)
+        g = head_backward_block(a[0], a[1], a[2], a[3], rl[0, h], delta, scale, False, Nq, Nk,
+                                row0, key0, p, seed, 0, h)
+        for i in range(3):
+            rg[i][0, h] = g[i]
+    compare(f64(o), f64(lse), ro, rl, parity_record)
+    check_grads((f64(dq), f64(dk), f64(dv)), rg, parity_record)
