@@ -40,6 +40,16 @@
 // warpgroup; dP^T [128,256); dV [256, 256 + D); dK [256 + D, 256 + 2 D); the
 // dQ tile in [384, 448) for d = 64; for d = 128 its transpose dQ^T (lane =
 // feature, column = query) in the dP^T columns once dP^T has been consumed.
+//
+// d = 256 (and 192): the dK, dV accumulators of a key tile would fill TMEM on
+// their own, so two CTAs share the tile, CTA h owning feature columns
+// [128 h, 128 h + 128) of dK, dV and dQ; both compute the full S^T and dP^T.
+// Each then has the d = 128 TMEM map (dV and dK halves of 128 columns, the dQ^T
+// half in the dP^T columns) and the same roles; K and V stay resident, Q and
+// dO pass through a ring of four 64-column panels that the producer fills in
+// exactly the order the MMA warp takes them, and the LSE / D slices through a
+// two-stage ring of their own that the P / dS warps hand back after their dS
+// phase.
 #include <cuda_bf16.h>
 
 #include <type_traits>

@@ -33,6 +33,7 @@ def rel_l2(a, ref):
 @pytest.mark.parametrize("B,H,N,d,causal,lens,p", [
     (2, 3, 300, 64, True, None, 0.1),
     (1, 2, 520, 128, False, (200, 520), 0.0),
+    (1, 2, 400, 256, True, None, 0.1),          # the 256-wide backward (two CTAs per key tile)
 ])
 def test_noalloc_backward_matches_oracle_and_workspace_backward(lib, B, H, N, d, causal, lens,
                                                                 p):
