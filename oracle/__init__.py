@@ -8,7 +8,11 @@ links or calls it, and it never imports the CUDA library.
 from .attention_ref import (  # noqa: F401
     BLOCK,
     attention_backward,
+    attention_backward_gqa,
     attention_forward,
+    attention_forward_gqa,
+    gqa_expand,
+    gqa_reduce,
     dropout_keep,
     dropout_scale,
     dropout_threshold,

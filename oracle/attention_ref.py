@@ -390,3 +390,40 @@ def head_backward_block(q, k, v, dout, lse, delta, scale, causal=False, n_q=None
     dp = (dout @ v.T) * z * rscale
     ds = p * (dp - np.asarray(delta, dtype=np.float64)[:, None])
     return scale * (ds @ k), scale * (ds.T @ q), (p * z * rscale).T @ dout
+
+
+# ----------------------------------------------------------------------------
+# grouped K / V heads (an extension the pages do not treat)
+# ----------------------------------------------------------------------------
+
+def gqa_expand(x, group, axis=1):
+    """K or V with H_kv heads on `axis`, each repeated for the `group` query
+    heads that share it: query head h reads K / V head h // group."""
+    return np.repeat(np.asarray(x, dtype=np.float64), group, axis=axis)
+
+
+def gqa_reduce(dx, group, axis=1):
+    """The gradient of a K / V head shared by `group` query heads: the sum of
+    the gradients of its copies (the chain rule through the repetition)."""
+    dx = np.moveaxis(np.asarray(dx, dtype=np.float64), axis, 0)
+    dx = dx.reshape((dx.shape[0] // group, group) + dx.shape[1:]).sum(axis=1)
+    return np.moveaxis(dx, 0, axis)
+
+
+def attention_forward_gqa(q, k, v, scale, causal=False, seqlens=None, dropout_p=0.0, seed=0,
+                          block_mask=None):
+    """O, LSE when k, v ([B, H_kv, N, d]) have fewer heads than q ([B, H, N, d]):
+    standard attention against the K / V head of each query head's group.
+    Dropout keeps its (b, h, i, j) keying with h the query head."""
+    group = q.shape[1] // k.shape[1]
+    return attention_forward(q, gqa_expand(k, group), gqa_expand(v, group), scale, causal,
+                             seqlens, dropout_p, seed, block_mask)
+
+
+def attention_backward_gqa(q, k, v, dout, scale, causal=False, seqlens=None, dropout_p=0.0,
+                           seed=0, block_mask=None):
+    """dQ [B, H, N, d] and dK, dV [B, H_kv, N, d] of attention_forward_gqa."""
+    group = q.shape[1] // k.shape[1]
+    dq, dk, dv = attention_backward(q, gqa_expand(k, group), gqa_expand(v, group), dout, scale,
+                                    causal, seqlens, dropout_p, seed, block_mask)
+    return dq, gqa_reduce(dk, group), gqa_reduce(dv, group)

@@ -922,3 +922,56 @@ def test_row_and_column_helpers_on_a_diagonal_slice_match_the_whole_problem():
     # the offsets matter: without them the dropout bits are another draw
     wrong_o, _ = head_forward_rows(q[sl], k[sl], v[sl], 0.25, rows, **kw)
     assert not np.allclose(full_o, wrong_o, rtol=0, atol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# grouped K / V heads
+# ---------------------------------------------------------------------------
+
+def test_gqa_forward_uses_the_group_head():
+    """Without dropout each query head's O and LSE are plain attention against
+    K / V head h // G, evaluated head by head; the mapping h % H_kv (or any
+    other) gives different outputs."""
+    from oracle import attention_forward_gqa
+    rng = np.random.default_rng(77)
+    B, H, Hkv, N, d = 2, 6, 2, 9, 4
+    q = _rand((B, H, N, d), rng)
+    k, v = _rand((B, Hkv, N, d), rng), _rand((B, Hkv, N, d), rng)
+    o, lse = attention_forward_gqa(q, k, v, 0.4, True)
+    G = H // Hkv
+    for h in range(H):
+        oh, lh = attention_forward(q[:, h:h + 1], k[:, h // G:h // G + 1], v[:, h // G:h // G + 1],
+                                   0.4, True)
+        assert np.abs(o[:, h:h + 1] - oh).max() < 1e-12
+        assert np.abs(lse[:, h:h + 1] - lh).max() < 1e-12
+    wrong, _ = attention_forward(q[:, 1:2], k[:, 1:2], v[:, 1:2], 0.4, True)  # h % H_kv
+    assert np.abs(o[:, 1:2] - wrong).max() > 1e-3
+
+
+def test_gqa_backward_matches_finite_differences():
+    """dQ and the shared heads' dK, dV (sums over each group) against central
+    differences of L = sum(O * dO), with a causal mask and dropout."""
+    from oracle import attention_backward_gqa, attention_forward_gqa
+    rng = np.random.default_rng(78)
+    B, H, Hkv, N, d, p, seed = 1, 4, 2, 6, 3, 0.3, 11
+    q, do = _rand((B, H, N, d), rng), _rand((B, H, N, d), rng)
+    k, v = _rand((B, Hkv, N, d), rng), _rand((B, Hkv, N, d), rng)
+
+    def loss(q_, k_, v_):
+        o, _ = attention_forward_gqa(q_, k_, v_, 0.7, True, None, p, seed)
+        return float((o * do).sum())
+
+    grads = attention_backward_gqa(q, k, v, do, 0.7, True, None, p, seed)
+    assert grads[1].shape == k.shape and grads[2].shape == v.shape
+    eps = 1e-6
+    for name, x, g in zip("qkv", (q, k, v), grads):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            a = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num[idx] = (loss(*a) - loss(*m)) / (2 * eps)
+        err = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+        assert err < 1e-6, (name, err)
