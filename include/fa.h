@@ -217,6 +217,11 @@ typedef struct {
    * dropout_key0 + seqlen_k at most 2^31 - 1; otherwise FA_ERR_INVALID_ARG.
    * The masks are not moved: they stay relative to the call's own rows. */
   int64_t dropout_row0, dropout_key0;
+  /* Grouped-query attention: K and V (and dK, dV) have heads_kv heads, and
+   * query head h reads K / V head h / (heads / heads_kv); heads_kv must divide
+   * heads (otherwise FA_ERR_INVALID_ARG).  0, or heads: one K / V head per
+   * query head.  dK and dV of a K / V head are the sums over its query heads. */
+  int heads_kv;
 } fa_attention_desc_t;
 
 /* Forward pass for a general layout.  LSE is fp32 [B, H, seqlen_q]

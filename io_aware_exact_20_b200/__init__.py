@@ -96,6 +96,7 @@ class AttentionDesc(ctypes.Structure):
         ("q", Strides), ("k", Strides), ("v", Strides), ("o", Strides), ("dout", Strides),
         ("dq", Strides), ("dk", Strides), ("dv", Strides),
         ("dropout_row0", ctypes.c_int64), ("dropout_key0", ctypes.c_int64),
+        ("heads_kv", ctypes.c_int),
     ]
 
 
@@ -360,11 +361,12 @@ def _desc(q, k, layout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, 
                              f"{'q' if name in _Q_SIDE else 'k'} {tuple(ref.shape)}")
     Bq, Nq, H, d = _dims(q, layout)
     Bk, Nk, Hk, dk = _dims(k, layout)
-    if H != Hk or d != dk:
-        raise ValueError("q and k must have the same heads and head dim")
+    if d != dk or Hk < 1 or H % Hk:
+        raise ValueError("q and k must have the same head dim, and q's heads must be a multiple "
+                         "of k's (grouped-query attention)")
     keep = []
     a = AttentionDesc()
-    a.heads, a.head_dim = H, d
+    a.heads, a.head_dim, a.heads_kv = H, d, Hk
     if layout == "thd":
         if cu_seqlens_q is None or cu_seqlens_k is None:
             raise ValueError("the packed layout needs cu_seqlens_q and cu_seqlens_k")
@@ -407,6 +409,8 @@ def forward_general(q, k, v, *, layout="bhsd", cu_seqlens_q=None, cu_seqlens_k=N
     offsets cu_seqlens_q / cu_seqlens_k ([B + 1]) and the longest lengths.  Any
     strides with d contiguous (multiples of 8 elements).  The causal mask is
     bottom-right aligned per sequence.  LSE: [B, H, N_q] or [H, T_q] (packed).
+    k and v may have fewer heads than q, a divisor of them (grouped-query
+    attention: query head h reads K / V head h // (H / H_kv)).
     dropout_row0 / dropout_key0: positions of the call's first query row and
     first key in the sequence the dropout bits are keyed by (a block of a
     longer sequence); the key position a multiple of 8.

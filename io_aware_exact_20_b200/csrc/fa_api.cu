@@ -79,6 +79,7 @@ struct Problem {
   const uint8_t* block_mask;
   fa_strides_t q, k, v, o, dout, dq, dk, dv;
   int64_t drop_row0, drop_key0;  // dropout positions of the first query row and key
+  int Hkv;                       // K / V heads (H / Hkv query heads share each)
 
   int rows_q() const { return packed ? total_q : nq; }
   int rows_k() const { return packed ? total_k : nk; }
@@ -120,12 +121,17 @@ fa_status_t resolve(const fa_attention_desc_t* a, Problem* p, Uses uses) {
   const int64_t per_tile = (uses == kBackward && D == 256) ? 2 : 1;
   if (static_cast<int64_t>(a->batch) * a->heads * tiles * per_tile > 0x7FFFFFFF)
     return FA_ERR_UNSUPPORTED;
+  // grouped-query attention: heads_kv K / V heads, each shared by heads / heads_kv
+  const int hkv = a->heads_kv == 0 ? a->heads : a->heads_kv;
+  if (hkv < 1 || hkv > a->heads || a->heads % hkv != 0) return FA_ERR_INVALID_ARG;
   const fa_strides_t* all[8] = {&a->q, &a->k, &a->v, &a->o, &a->dout, &a->dq, &a->dk, &a->dv};
+  const bool kv_side[8] = {false, true, true, false, false, false, true, true};
   for (int t = 0; t < (uses == kForward ? 4 : 8); ++t) {
     const fa_strides_t* s = all[t];
     if (!strides_ok(*s, packed)) return FA_ERR_INVALID_ARG;
     // a zero stride would make heads / entries / rows share memory
-    if ((a->heads > 1 && s->head == 0) || (!packed && a->batch > 1 && s->batch == 0) ||
+    const int heads_t = kv_side[t] ? hkv : a->heads;
+    if ((heads_t > 1 && s->head == 0) || (!packed && a->batch > 1 && s->batch == 0) ||
         s->row == 0)
       return FA_ERR_INVALID_ARG;
   }
@@ -135,6 +141,7 @@ fa_status_t resolve(const fa_attention_desc_t* a, Problem* p, Uses uses) {
     return FA_ERR_INVALID_ARG;
   p->drop_row0 = a->dropout_row0;
   p->drop_key0 = a->dropout_key0;
+  p->Hkv = hkv;
   p->B = a->batch;
   p->H = a->heads;
   p->d = a->head_dim;
@@ -202,14 +209,15 @@ fa::Rows kernel_rows(const Problem& p) {
 }
 
 // TMA view {d, rows, H, batch} of a bf16 tensor; box 64 x 128 x 1 x 1.
-bool tmap(CUtensorMap* m, const void* base, const Problem& p, const fa_strides_t& s, int rows) {
+bool tmap(CUtensorMap* m, const void* base, const Problem& p, const fa_strides_t& s, int rows,
+          int heads) {
   fa::TmapDesc t = fa::tmap_desc_zero();
   t.base = base;
   t.dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   t.rank = 4;
   t.dims[0] = static_cast<uint64_t>(p.d);
   t.dims[1] = static_cast<uint64_t>(rows);
-  t.dims[2] = static_cast<uint64_t>(p.H);
+  t.dims[2] = static_cast<uint64_t>(heads);
   t.dims[3] = static_cast<uint64_t>(p.tb());
   // a zero stride (a single head or batch entry) is described as the
   // smallest legal one; that coordinate is always 0
@@ -267,8 +275,8 @@ void set_extents(const Problem& pr, int* status, fa::Extents* e, fa::Rows* rows)
   e->o = span(pr.o, tb, pr.H, pr.rows_q(), pr.d);
   e->dout = span(pr.dout, tb, pr.H, pr.rows_q(), pr.d);
   e->dq = span(pr.dq, tb, pr.H, pr.rows_q(), pr.d);
-  e->dk = span(pr.dk, tb, pr.H, pr.rows_k(), pr.d);
-  e->dv = span(pr.dv, tb, pr.H, pr.rows_k(), pr.d);
+  e->dk = span(pr.dk, tb, pr.Hkv, pr.rows_k(), pr.d);
+  e->dv = span(pr.dv, tb, pr.Hkv, pr.rows_k(), pr.d);
   long long sb = 0, sh = 0;
   lse_strides(pr, &sb, &sh);
   e->lse = (tb - 1) * sb + (pr.H - 1) * sh + pr.rows_q();
@@ -288,8 +296,8 @@ fa_status_t run_fwd(const Problem& pr, const void* q, const void* k, const void*
   int* status = status_word();
   if (status == nullptr) return FA_ERR_CUDA;
   CUtensorMap tq, tk, tv;
-  if (!tmap(&tq, q, pr, pr.q, pr.rows_q()) || !tmap(&tk, k, pr, pr.k, pr.rows_k()) ||
-      !tmap(&tv, v, pr, pr.v, pr.rows_k()))
+  if (!tmap(&tq, q, pr, pr.q, pr.rows_q(), pr.H) || !tmap(&tk, k, pr, pr.k, pr.rows_k(), pr.Hkv) ||
+      !tmap(&tv, v, pr, pr.v, pr.rows_k(), pr.Hkv))
     return FA_ERR_UNSUPPORTED;
   const Dropout dr = dropout_params(pr.dropout_p);
   fa::FwdParams p{};
@@ -305,6 +313,7 @@ fa_status_t run_fwd(const Problem& pr, const void* q, const void* k, const void*
   p.rows = kernel_rows(pr);
   p.B = pr.B;
   p.H = pr.H;
+  p.group = pr.H / pr.Hkv;
   p.d_real = pr.d;
   p.scale_log2 = static_cast<float>(static_cast<double>(pr.scale) * kLog2e);
   p.causal = pr.causal;
@@ -359,11 +368,16 @@ fa_status_t bwd_params(fa::BwdParams* p, const Problem& pr, const void* workspac
   p->rows = kernel_rows(pr);
   p->B = pr.B;
   p->H = pr.H;
+  p->group = pr.H / pr.Hkv;
   p->d_real = pr.d;
   p->scale = pr.scale;
   p->scale_log2 = static_cast<float>(static_cast<double>(pr.scale) * kLog2e);
   p->causal = pr.causal;
-  p->group_heads = fa::order_group_heads(pr.B, pr.H, fa::bwd_head_bytes(pr.nq, pr.D), pr.causal);
+  // the main kernel's units are (b, K / V head, key tile): its head groups are
+  // of K / V heads, each sharing the Q / dO rows of H / Hkv query heads
+  p->group_heads = fa::order_group_heads(pr.B, pr.Hkv,
+                                         (pr.H / pr.Hkv) * fa::bwd_head_bytes(pr.nq, pr.D),
+                                         pr.causal);
   p->drop_threshold = dr.threshold;
   p->drop_rscale = dr.rscale;
   p->seed_lo = static_cast<uint32_t>(pr.seed & 0xFFFFFFFFull);
@@ -386,8 +400,10 @@ struct BwdMaps {
 
 fa_status_t bwd_maps(BwdMaps* m, const Problem& pr, const fa::BwdParams& p, const void* q,
                      const void* k, const void* v, const void* dout) {
-  if (!tmap(&m->q, q, pr, pr.q, pr.rows_q()) || !tmap(&m->k, k, pr, pr.k, pr.rows_k()) ||
-      !tmap(&m->v, v, pr, pr.v, pr.rows_k()) || !tmap(&m->dout, dout, pr, pr.dout, pr.rows_q()))
+  if (!tmap(&m->q, q, pr, pr.q, pr.rows_q(), pr.H) ||
+      !tmap(&m->k, k, pr, pr.k, pr.rows_k(), pr.Hkv) ||
+      !tmap(&m->v, v, pr, pr.v, pr.rows_k(), pr.Hkv) ||
+      !tmap(&m->dout, dout, pr, pr.dout, pr.rows_q(), pr.H))
     return FA_ERR_UNSUPPORTED;
   if (!fa::make_tmap_f32_2d(&m->dq, p.ws_dq, static_cast<uint64_t>(pr.D),
                             static_cast<uint64_t>(p.ws_rows), 128))

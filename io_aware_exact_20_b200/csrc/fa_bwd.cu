@@ -150,10 +150,20 @@ struct BwdLayout {
 // Kernels launched without a block mask, with columns longer than the
 // bitmask, or at d = 128 are built without it (kBits false) and test the
 // mask's bytes directly.
+// One step of a CTA's walk: query tile qb of the group's query head g,
+// packed as g * 2^16 + qb (qb < 2^16 since N <= 2^23) by the general (GEN)
+// instances; the others have one query head per K / V head and walk the query
+// tile index itself.
+using Tile = int;
+template <bool GEN>
+__device__ __forceinline__ int tile_g(Tile t) { return GEN ? t >> 16 : 0; }
+template <bool GEN>
+__device__ __forceinline__ int tile_qb(Tile t) { return GEN ? t & 0xFFFF : t; }
+
 template <bool kBits>
 struct BwdWork {
-  int b, h, bh, kb, kv_len, nqb, qb_begin, nbk, off, qrow, krow, tb, lk;
-  long long ws0;
+  int b, hk, bh, kb, kv_len, nqb, qb_begin, nbk, off, qrow, krow, tb, lk;  // hk: K / V head
+  long long ws0;  // first workspace row of query head hk * G (G = 1: the only one)
   bool alive, causal;
   const uint8_t* bm;
   const uint32_t* bits;  // shared-memory bitmask over the query tiles, or null
@@ -181,6 +191,35 @@ struct BwdWork {
     }
     while (qb < nqb && !act(qb)) ++qb;
     return qb;
+  }
+  // The walk.  GEN: over the G query heads of the group, the same query
+  // tiles for each (the masks do not depend on the head), head after head;
+  // done when tile_g(t) == G.  Otherwise: the query tiles, done at nqb.
+  template <bool GEN>
+  __device__ __forceinline__ Tile first(int G) const {
+    const int qb = next(qb_begin);
+    return GEN && qb >= nqb ? (G << 16) : qb;
+  }
+  template <bool GEN>
+  __device__ __forceinline__ Tile step(Tile t) const {
+    if constexpr (!GEN) {
+      return next(t + 1);
+    } else {
+      const int qb = next(tile_qb<true>(t) + 1);
+      return qb < nqb ? ((t & ~0xFFFF) | qb) : (((t & ~0xFFFF) + 0x10000) | next(qb_begin));
+    }
+  }
+  template <bool GEN>
+  __device__ __forceinline__ bool more(Tile t, int G) const {
+    return GEN ? tile_g<true>(t) < G : t < nqb;
+  }
+  // query head of step t, and the workspace row of its query tile's first row
+  // (ws_hs: workspace rows from one query head to the next)
+  template <bool GEN>
+  __device__ __forceinline__ int hq(Tile t, int G) const { return hk * G + tile_g<GEN>(t); }
+  template <bool GEN>
+  __device__ __forceinline__ long long wsrow(Tile t, long long ws_hs) const {
+    return ws0 + tile_g<GEN>(t) * ws_hs + 128ll * tile_qb<GEN>(t);
   }
 };
 
@@ -276,9 +315,12 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
 // main kernel
 // ---------------------------------------------------------------------------
 
-// POS as in the forward kernel: dropout counters offset by the call's row /
-// key positions (instantiated only with dropout and the direct mask walk).
-template <int D, bool DROPOUT, bool BITS, bool POS = false>
+// GEN: the general instances, which read from the parameters the number of
+// query heads per K / V head (grouped-query attention) and the dropout
+// counters' row / key offsets (as the forward's POS instances); the others
+// see one query head per K / V head and zero offsets at compile time.  Built
+// only with the direct mask walk.
+template <int D, bool DROPOUT, bool BITS, bool GEN = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -308,10 +350,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // d = 256: CTAs 2u and 2u + 1 take the two column halves of unit u
   const int hf = L::RING ? static_cast<int>(blockIdx.x & 1u) : 0;
   const long long unit = L::RING ? static_cast<long long>(blockIdx.x >> 1) : blockIdx.x;
-  grid_unit(unit, p.B * p.H, (p.rows.nk + 127) / 128, p.group_heads, &w.bh,
+  const int G = GEN ? p.group : 1;  // query heads per K / V head
+  const int n_kv_heads = p.H / G;
+  grid_unit(unit, p.B * n_kv_heads, (p.rows.nk + 127) / 128, p.group_heads, &w.bh,
             &w.kb);  // key tile 0 is heaviest
-  w.b = w.bh / p.H;
-  w.h = w.bh % p.H;
+  w.b = w.bh / n_kv_heads;
+  w.hk = w.bh % n_kv_heads;
   {
     const Seq sq = seq_of(p.rows, w.b);
     // a sequence shorter than the longest has no key tile here: leave before
@@ -327,7 +371,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     w.tb = sq.tb;
     w.off = sq.lk - sq.lq;
     w.nqb = (sq.lq + 127) / 128;
-    w.ws0 = ws_row0(p, w.b, w.h, sq.q0);
+    w.ws0 = ws_row0(p, w.b, w.hk * G, sq.q0);
   }
   w.alive = w.kb * 128 < w.kv_len;
   w.causal = p.causal != 0;
@@ -388,8 +432,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int q_first = w.next(w.qb_begin);
-  const bool any_work = q_first < w.nqb;
+  // the walk with this launch's group size and workspace rows per query head
+  const long long ws_hs = p.rows.cu_q == nullptr ? p.Npad : p.Rtot;
+  auto more = [&](Tile t) { return w.template more<GEN>(t, G); };
+  auto next_t = [&](Tile t) { return w.template step<GEN>(t); };
+  const Tile t_first = w.template first<GEN>(G);
+  const bool any_work = more(t_first);
 
   if (warp < 4) {
   if constexpr (L::SPLIT_REGS) setmaxnreg_dec<L::REGS_CTL>();
@@ -403,9 +451,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::TILE);
       for (int pn = 0; pn < L::PANELS; ++pn) {
         tma_load_4d(sbase + L::OFF_K + pn * L::PANEL, &tm_k, bar(L::B_KV), 64 * pn,
-                    w.krow + w.kb * 128, w.h, w.tb);
+                    w.krow + w.kb * 128, w.hk, w.tb);
         tma_load_4d(sbase + L::OFF_V + pn * L::PANEL, &tm_v, bar(L::B_KV), 64 * pn,
-                    w.krow + w.kb * 128, w.h, w.tb);
+                    w.krow + w.kb * 128, w.hk, w.tb);
       }
       if constexpr (L::RING) {
         // Panels in the order the MMA warp consumes them: Q(first), dO(first)
@@ -418,26 +466,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // start; the reload of the Q pair waits for dP^T(n + 1) instead, off
         // the path from one tile's dS to the next tile's dP^T.
         int t = 0, nld = 0;
-        auto panel = [&](const CUtensorMap* m, int pn, int qb) -> bool {
+        auto panel = [&](const CUtensorMap* m, int pn, Tile tt) -> bool {
           const int s = t % L::STAGES;
           if (t >= L::STAGES && !mbar_wait(bar(L::B_QEMPTY + s), ((t / L::STAGES) & 1u) ^ 1u, g))
             return false;
           mbar_arrive_expect_tx(bar(L::B_QFULL + s), L::PANEL);
           tma_load_4d(sbase + L::OFF_Q + s * L::PANEL, m, bar(L::B_QFULL + s), 64 * pn,
-                      w.qrow + qb * 128, w.h, w.tb);
+                      w.qrow + tile_qb<GEN>(tt) * 128, w.template hq<GEN>(tt, G), w.tb);
           ++t;
           return true;
         };
-        auto tile4 = [&](const CUtensorMap* m, int qb) -> bool {
+        auto tile4 = [&](const CUtensorMap* m, Tile tt) -> bool {
           for (int pn = 0; pn < L::PANELS; ++pn)
-            if (!panel(m, pn, qb)) return false;
+            if (!panel(m, pn, tt)) return false;
           return true;
         };
-        auto ld = [&](int qb) -> bool {  // -LSE log2e and -D of the tile's rows
+        auto ld = [&](Tile tt) -> bool {  // -LSE log2e and -D of the tile's rows
           const int s = nld & 1;
           if (nld >= 2 && !mbar_wait(bar(L::B_LDEMPTY + s), ((nld >> 1) & 1u) ^ 1u, g)) return false;
           mbar_arrive_expect_tx(bar(L::B_LDFULL + s), 1024);
-          long long roff = w.ws0 + static_cast<long long>(qb) * 128;
+          long long roff = w.template wsrow<GEN>(tt, ws_hs);
           if (!FA_IN_BOUNDS(p.status, roff, 128, p.ws_rows)) roff = 0;
           bulk_load(sbase + L::OFF_LD + s * 1024, p.ws_lse2 + roff, 512, bar(L::B_LDFULL + s));
           bulk_load(sbase + L::OFF_LD + s * 1024 + 512, p.ws_delta + roff, 512,
@@ -445,13 +493,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ++nld;
           return true;
         };
-        bool ok = ld(q_first) && tile4(&tm_q, q_first) && tile4(&tm_do, q_first);
-        for (int qb = q_first; ok && qb < w.nqb;) {
-          const int qbn = w.next(qb + 1);
-          ok = panel(&tm_do, 2 * hf, qb) && panel(&tm_do, 2 * hf + 1, qb);
-          if (ok && qbn < w.nqb) ok = ld(qbn) && tile4(&tm_q, qbn) && tile4(&tm_do, qbn);
-          if (ok) ok = panel(&tm_q, 2 * hf, qb) && panel(&tm_q, 2 * hf + 1, qb);
-          qb = qbn;
+        bool ok = ld(t_first) && tile4(&tm_q, t_first) && tile4(&tm_do, t_first);
+        for (Tile tc = t_first; ok && more(tc);) {
+          const Tile tn = next_t(tc);
+          ok = panel(&tm_do, 2 * hf, tc) && panel(&tm_do, 2 * hf + 1, tc);
+          if (ok && more(tn)) ok = ld(tn) && tile4(&tm_q, tn) && tile4(&tm_do, tn);
+          if (ok) ok = panel(&tm_q, 2 * hf, tc) && panel(&tm_q, 2 * hf + 1, tc);
+          tc = tn;
         }
         if (*abort_flag) {
           for (int j = max(0, t - L::STAGES); j < t; ++j)
@@ -462,18 +510,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       } else {
       int it = 0;
-      for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
+      for (Tile tc = t_first; more(tc); tc = next_t(tc), ++it) {
         const int s = it % L::STAGES;
         const uint32_t ph = (it / L::STAGES) & 1u;
         if (it >= L::STAGES && !mbar_wait(bar(L::B_QEMPTY + s), ph ^ 1u, g)) break;
         mbar_arrive_expect_tx(bar(L::B_QFULL + s), 2 * L::TILE + 1024);
+        const int hq = w.template hq<GEN>(tc, G);
         for (int pn = 0; pn < L::PANELS; ++pn) {
           tma_load_4d(sbase + L::OFF_Q + s * L::TILE + pn * L::PANEL, &tm_q, bar(L::B_QFULL + s),
-                      64 * pn, w.qrow + qb * 128, w.h, w.tb);
+                      64 * pn, w.qrow + tile_qb<GEN>(tc) * 128, hq, w.tb);
           tma_load_4d(sbase + L::OFF_DO + s * L::TILE + pn * L::PANEL, &tm_do, bar(L::B_QFULL + s),
-                      64 * pn, w.qrow + qb * 128, w.h, w.tb);
+                      64 * pn, w.qrow + tile_qb<GEN>(tc) * 128, hq, w.tb);
         }
-        long long roff = w.ws0 + static_cast<long long>(qb) * 128;
+        long long roff = w.template wsrow<GEN>(tc, ws_hs);
         if (!FA_IN_BOUNDS(p.status, roff, 128, p.ws_rows)) roff = 0;
         bulk_load(sbase + L::OFF_LD + s * 1024, p.ws_lse2 + roff, 512, bar(L::B_QFULL + s));
         bulk_load(sbase + L::OFF_LD + s * 1024 + 512, p.ws_delta + roff, 512, bar(L::B_QFULL + s));
@@ -542,6 +591,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
 
+      // The MMA warp only needs to know whether a tile remains and whether
+      // another follows: the general instances count the steps (G heads times
+      // the active query tiles) instead of walking them, which keeps the walk
+      // out of this 72-register warp.
+      int n_total = 0;
+      if constexpr (GEN) {
+        for (int qb = w.next(w.qb_begin); qb < w.nqb; qb = w.next(qb + 1)) ++n_total;
+        n_total *= G;
+      }
+      auto mma_more = [&](Tile t, int i) { return GEN ? i < n_total : more(t); };
+      auto mma_next = [&](Tile t) { return GEN ? t : next_t(t); };
       if constexpr (L::RING) {
         int c = 0;  // panels taken from the ring
         auto slot = [&](int s) -> uint32_t { return sbase + L::OFF_Q + s * L::PANEL; };
@@ -589,8 +649,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // here; without the two phases PFULL already means dS is ready.
         int it = 0;
         if (ok) ok = ring_sdp(false) && ring_sdp(true);
-        for (int qb = q_first; ok && qb < w.nqb; ++it) {
-          const int qbn = w.next(qb + 1);
+        for (Tile tc = t_first; ok && mma_more(tc, it); ++it) {
+          const Tile tn = mma_next(tc);
           if (!mbar_wait(bar(L::B_PFULL), it & 1u, g)) break;
           tc_fence_after();
           const int sd = take_pair();
@@ -603,14 +663,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                    (it > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(L::B_QEMPTY + sd));
           mma_commit(bar(L::B_QEMPTY + sd + 1));
-          if (qbn < w.nqb && !ring_sdp(false)) break;
+          if (mma_more(tn, it + 1) && !ring_sdp(false)) break;
           if constexpr (kTwoPhase) {
             if (!mbar_wait(bar(L::B_DSFULL), it & 1u, g)) break;
             tc_fence_after();
           }
           issue_dq();
           mma_commit(bar(L::B_DQFULL));
-          if (qbn < w.nqb) {
+          if (mma_more(tn, it + 1)) {
             if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
             tc_fence_after();
             if (!ring_sdp(true)) break;
@@ -621,7 +681,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_commit(bar(L::B_QEMPTY + sq));
           mma_commit(bar(L::B_QEMPTY + sq + 1));
           mma_commit(bar(L::B_DSEMPTY));
-          qb = qbn;
+          tc = tn;
         }
       } else {
       int it = 0;
@@ -632,9 +692,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_sdp(0, true);
       }
       if constexpr (kTwoPhase) {
-        for (int qb = q_first; ok && qb < w.nqb; ++it) {
+        for (Tile tc = t_first; ok && mma_more(tc, it); ++it) {
           const int s = it % L::STAGES;
-          const int qbn = w.next(qb + 1);
+          const Tile tn = mma_next(tc);
           const int sn = (it + 1) % L::STAGES;
           const uint32_t q_addr = sbase + L::OFF_Q + s * L::TILE;
           const uint32_t do_addr = sbase + L::OFF_DO + s * L::TILE;
@@ -647,7 +707,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                    sdesc_sw128(do_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
                    (it > 0 || kk > 0) ? 1u : 0u);
           // the next tile's S^T overwrites S^T / P only after the dV MMAs above
-          if (qbn < w.nqb) {
+          if (mma_more(tn, it + 1)) {
             if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
             tc_fence_after();
             issue_sdp(sn, false);
@@ -675,7 +735,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           mma_commit(bar(L::B_DSEMPTY));
           if constexpr (!L::TMA_REDUCE) mma_commit(bar(L::B_QEMPTY + s));
-          if (qbn < w.nqb) {
+          if (mma_more(tn, it + 1)) {
             // dP^T of the next tile: its columns were read by this tile's dS
             // phase, and (d = 128) hold the dQ tile until it is drained
             if (!L::SEPARATE_DQ) {
@@ -684,7 +744,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             issue_sdp(sn, true);
           }
-          qb = qbn;
+          tc = tn;
         }
       } else {
         // serialized order, once P and dS are both ready: dV, then the next
@@ -693,9 +753,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // by this tile's P / dS warps already), then dK and dQ.  The next
         // tile's S^T / dP^T are ready while dK and dQ still run.  At d = 128
         // the dQ^T tile lives in the dP^T columns, so dP^T comes last.
-        for (int qb = q_first; ok && qb < w.nqb; ++it) {
+        for (Tile tc = t_first; ok && mma_more(tc, it); ++it) {
           const int s = it % L::STAGES;
-          const int qbn = w.next(qb + 1);
+          const Tile tn = mma_next(tc);
           const int sn = (it + 1) % L::STAGES;
           if (!mbar_wait(bar(L::B_PFULL), it & 1u, g)) break;
           tc_fence_after();
@@ -707,7 +767,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_ts(tmem + L::COL_DV, tmem + L::COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
                    sdesc_sw128(do_addr + kk * 2048, L::PANEL, 1024), kIdKQ,
                    (it > 0 || kk > 0) ? 1u : 0u);
-          if (qbn < w.nqb) {
+          if (mma_more(tn, it + 1)) {
             if (!mbar_wait(bar(L::B_QFULL + sn), ((it + 1) / L::STAGES) & 1u, g)) break;
             tc_fence_after();
             issue_sdp(sn, false);
@@ -730,12 +790,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           mma_commit(bar(L::B_DSEMPTY));
           if constexpr (!L::TMA_REDUCE) mma_commit(bar(L::B_QEMPTY + s));
-          if (!L::SEPARATE_DQ && qbn < w.nqb) {
+          if (!L::SEPARATE_DQ && mma_more(tn, it + 1)) {
             if (!mbar_wait(bar(L::B_DQEMPTY), it & 1u, g)) break;
             tc_fence_after();
             issue_sdp(sn, true);
           }
-          qb = qbn;
+          tc = tn;
         }
       }
       }
@@ -755,7 +815,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float2 rs2 = make_float2(p.drop_rscale, p.drop_rscale);
     bool ok = true;
     int it = 0;
-    for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
+    for (Tile tc = t_first; more(tc); tc = next_t(tc), ++it) {
+      const int qb = tile_qb<GEN>(tc);
       const int s = it % L::STAGES;
       // Dropout keep bits of this key for the warpgroup's 64 queries, drawn
       // before the waits (they do not depend on S or dP).  A block covers
@@ -776,10 +837,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t own = 0u;
 #pragma unroll
           for (int gq = 0; gq < 4; ++gq) {
-            const uint32_t qg = (POS ? p.drop_row0 : 0u) +
+            const uint32_t qg = (GEN ? p.drop_row0 : 0u) +
                                 static_cast<uint32_t>(qb * 128 + qoff + 8 * gq + (lane & 7));
-            const Philox4 rnd = philox4x32_10((POS ? p.drop_kgrp0 : 0u) + static_cast<uint32_t>(jg >> 3), qg,
-                                              static_cast<uint32_t>(w.h), static_cast<uint32_t>(w.b),
+            const Philox4 rnd = philox4x32_10((GEN ? p.drop_kgrp0 : 0u) + static_cast<uint32_t>(jg >> 3), qg,
+                                              static_cast<uint32_t>(w.template hq<GEN>(tc, G)), static_cast<uint32_t>(w.b),
                                               p.rk);
             own |= keep_byte(rnd, thr) << (8 * gq);
           }
@@ -1017,8 +1078,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) a[k] = bk[k] = 0u;
         }
-        const long long dv_off = w.tb * p.sdv.b + w.h * p.sdv.h + kr * p.sdv.r + col;
-        const long long dk_off = w.tb * p.sdk.b + w.h * p.sdk.h + kr * p.sdk.r + col;
+        const long long dv_off = w.tb * p.sdv.b + w.hk * p.sdv.h + kr * p.sdv.r + col;
+        const long long dk_off = w.tb * p.sdk.b + w.hk * p.sdk.h + kr * p.sdk.r + col;
         if (row_ok && col < p.d_real && FA_IN_BOUNDS(p.status, dv_off, 32, p.ext.dv) &&
             FA_IN_BOUNDS(p.status, dk_off, 32, p.ext.dk)) {
           uint4* dvp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + dv_off);
@@ -1047,7 +1108,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     int it = 0;
     bool issued = false;
-    for (int qb = q_first; qb < w.nqb; qb = w.next(qb + 1), ++it) {
+    for (Tile tc = t_first; more(tc); tc = next_t(tc), ++it) {
       const int s = it % L::STAGES;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL), it & 1u, g))) break;
       tc_fence_after();
@@ -1063,7 +1124,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // row.  The whole tile comes out of TMEM first and its columns go back
         // to the MMA warp (for the next tile's dP^T) before the reductions.
         const int feat = L::HD * hf + r;
-        float* dst = p.ws_dq + (w.ws0 + static_cast<long long>(qb) * 128) * D + feat;
+        float* dst = p.ws_dq + w.template wsrow<GEN>(tc, ws_hs) * D + feat;
         uint32_t a[128];
         tmem_ld32<0>(lane_addr + L::COL_DQ + 0, a);
         tmem_ld32<32>(lane_addr + L::COL_DQ + 32, a);
@@ -1080,7 +1141,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // warps at a time (d is a multiple of 32)
         // (the tile's rows are consecutive: its first and last accumulator
         // element bound every one it touches)
-        const long long acc0 = (w.ws0 + static_cast<long long>(qb) * 128) * D + feat;
+        const long long acc0 = w.template wsrow<GEN>(tc, ws_hs) * D + feat;
         if (feat < p.d_real && FA_IN_BOUNDS(p.status, acc0, 127ll * D + 1, p.ws_rows * D)) {
 #pragma unroll
           for (int k = 0; k < 128; ++k) red_add_f32(dst + k * D, __uint_as_float(a[k]));
@@ -1114,7 +1175,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0) {
           staged = mbar_wait(bar(L::B_STAGED), it & 1u, g);
           if (staged) {
-            const int32_t y = static_cast<int32_t>(w.ws0 + static_cast<long long>(qb) * 128);
+            const int32_t y = static_cast<int32_t>(w.template wsrow<GEN>(tc, ws_hs));
 #pragma unroll
             for (int b = 0; b < D / 32; ++b) tma_reduce_add_2d(&tm_dq, box(b), 32 * b, y);
             bulk_commit_group();
@@ -1150,13 +1211,13 @@ cudaError_t launch_pre_t(const BwdParams& p, cudaStream_t stream) {
   return launch_overlapped(bwd_pre_kernel<D>, prepost_grid<D>(p), dim3(256), 0, stream, p);
 }
 
-template <int D, bool DROPOUT, bool BITS, bool POS = false>
+template <int D, bool DROPOUT, bool BITS, bool GEN = false>
 cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdParams& p,
                           cudaStream_t stream) {
   using L = BwdLayout<D>;
   static_assert(!BITS || L::BIT_WORDS > 0, "no bitmask at this head dim");
-  auto kern = bwd_main_kernel<D, DROPOUT, BITS, POS>;
+  auto kern = bwd_main_kernel<D, DROPOUT, BITS, GEN>;
   // The setmaxnreg split (d = 128) is sized for exactly 128 registers per
   // thread at launch; with any other count an increase could wait forever.
   static OncePerContext prepared;
@@ -1171,9 +1232,9 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                                 static_cast<int>(L::SMEM));
   });
   if (e != cudaSuccess) return e;
-  // d = 256: two CTAs (column halves) per key tile
-  const long long ctas =
-      static_cast<long long>((p.rows.nk + 127) / 128) * p.B * p.H * (L::RING ? 2 : 1);
+  // one unit per (b, K / V head, key tile); d = 256: two CTAs (column halves) each
+  const long long ctas = static_cast<long long>((p.rows.nk + 127) / 128) * p.B *
+                         (p.H / (GEN ? p.group : 1)) * (L::RING ? 2 : 1);
   if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   return launch_overlapped(kern, dim3(static_cast<unsigned>(ctas)), dim3(kBwdThreads), L::SMEM,
                            stream, tq, tk, tv, tdo, tdq, p);
@@ -1196,10 +1257,17 @@ cudaError_t launch_bwd_pre(int d, const BwdParams& p, cudaStream_t stream) {
 cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdq,
                             const BwdParams& p, cudaStream_t stream) {
-  if (dropout && (p.drop_row0 != 0u || p.drop_kgrp0 != 0u)) {  // a block of a longer sequence
-    if (d == 64) return launch_main_t<64, true, false, true>(tq, tk, tv, tdo, tdq, p, stream);
-    if (d == 128) return launch_main_t<128, true, false, true>(tq, tk, tv, tdo, tdq, p, stream);
-    if (d == 256) return launch_main_t<256, true, false, true>(tq, tk, tv, tdo, tdq, p, stream);
+  // grouped K / V heads, or dropout on a block of a longer sequence
+  if (p.group > 1 || (dropout && (p.drop_row0 != 0u || p.drop_kgrp0 != 0u))) {
+    if (d == 64)
+      return dropout ? launch_main_t<64, true, false, true>(tq, tk, tv, tdo, tdq, p, stream)
+                     : launch_main_t<64, false, false, true>(tq, tk, tv, tdo, tdq, p, stream);
+    if (d == 128)
+      return dropout ? launch_main_t<128, true, false, true>(tq, tk, tv, tdo, tdq, p, stream)
+                     : launch_main_t<128, false, false, true>(tq, tk, tv, tdo, tdq, p, stream);
+    if (d == 256)
+      return dropout ? launch_main_t<256, true, false, true>(tq, tk, tv, tdo, tdq, p, stream)
+                     : launch_main_t<256, false, false, true>(tq, tk, tv, tdo, tdq, p, stream);
     return cudaErrorInvalidValue;
   }
   if (d == 64) {

@@ -338,12 +338,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         mbar_arrive_expect_tx(bar(L::B_KFULL + s), L::TILE);
         for (int pn = 0; pn < L::PANELS; ++pn)
           tma_load_4d(kdst + pn * L::PANEL, &tm_k, bar(L::B_KFULL + s), 64 * pn, w.krow + kb * 128,
-                      w.h, w.tb);
+                      w.h / p.group, w.tb);  // the group's K / V head
         if constexpr (!L::SPLIT_RELEASE) {
           mbar_arrive_expect_tx(bar(L::B_VFULL + s), L::TILE);
           for (int pn = 0; pn < L::PANELS; ++pn)
             tma_load_4d(vdst + pn * L::PANEL, &tm_v, bar(L::B_VFULL + s), 64 * pn,
-                        w.krow + kb * 128, w.h, w.tb);
+                        w.krow + kb * 128, w.h / p.group, w.tb);
         }
       }
       if (*abort_flag) {  // let the copies already issued land before the CTA exits
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         mbar_arrive_expect_tx(bar(L::B_VFULL + s), L::TILE);
         for (int pn = 0; pn < L::PANELS; ++pn)
           tma_load_4d(vdst + pn * L::PANEL, &tm_v, bar(L::B_VFULL + s), 64 * pn, w.krow + kb * 128,
-                      w.h, w.tb);
+                      w.h / p.group, w.tb);
       }
       if (*abort_flag) {
         for (int j = max(0, it - L::STAGES); j < it; ++j)

@@ -170,6 +170,7 @@ struct FwdParams {
   uint32_t drop_kgrp0;        // ... and 8-key group of its key 0 in the keyed sequence
   uint64_t timeout_ns;
   int mask_bitmap;            // block masks: 1 = walk them through a shared-memory bitmask
+  int group;                  // query heads per K / V head (1 = one K / V head each)
 #ifdef FA_DEBUG_BOUNDS
   Extents ext;
 #endif
@@ -211,6 +212,8 @@ struct BwdParams {
   uint32_t drop_row0, drop_kgrp0;  // as in FwdParams
   uint64_t timeout_ns;
   int mask_bitmap;            // as in FwdParams
+  int group;                  // query heads per K / V head; the main kernel's units are
+                              // (b, K / V head, key tile) and walk the group's query heads
 #ifdef FA_DEBUG_BOUNDS
   Extents ext;
 #endif

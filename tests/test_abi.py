@@ -127,6 +127,8 @@ def _desc(lib, **kw):
     (dict(dropout_row0=-1), 1), (dict(dropout_key0=-8), 1),
     (dict(dropout_row0=(1 << 31) - 256), 1),               # row0 + seqlen_q past 2^31 - 1
     (dict(dropout_key0=(1 << 40)), 1),
+    (dict(heads_kv=1), None), (dict(heads_kv=3), None),   # grouped K / V heads (3 query heads)
+    (dict(heads_kv=2), 1), (dict(heads_kv=4), 1), (dict(heads_kv=-1), 1),
 ])
 def test_general_entry_points_validate_before_launching(lib, change, code):
     so = lib.library()

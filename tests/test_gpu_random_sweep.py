@@ -17,7 +17,7 @@ without keys O = 0 and LSE = -inf on both sides, dQ / dK / dV relative L2
 import numpy as np
 import pytest
 
-from oracle import attention_backward, attention_forward
+from oracle import attention_backward_gqa, attention_forward_gqa, gqa_expand, gqa_reduce
 from oracle.varlen_ref import attention_backward_varlen, attention_forward_varlen
 from test_gpu_fwd import compare
 
@@ -32,7 +32,10 @@ def _draw_cases(n, seed=20250611):
     for c in range(n):
         layout = ("bhsd", "bshd", "thd")[c % 3]
         d = int(rng.choice(HEAD_DIMS))
-        B, H = int(rng.integers(1, 4)), int(rng.integers(1, 4))
+        B, H = int(rng.integers(1, 4)), int(rng.integers(1, 5))
+        Hkv = H  # grouped K / V heads now and then: a proper divisor of H
+        if H > 1 and rng.random() < 0.35:
+            Hkv = int(rng.choice([x for x in range(1, H) if H % x == 0]))
         if layout == "thd":
             # lengths per sequence, zero-length ones included
             lq = rng.integers(0, 520, size=B)
@@ -64,7 +67,7 @@ def _draw_cases(n, seed=20250611):
             mask = bm.tolist()
         p = float(rng.choice([0.0, 0.0, 0.1, 0.3]))
         scale = float(d ** -0.5 * rng.uniform(0.5, 1.5))
-        cases.append(dict(case=c, layout=layout, d=d, B=B, H=H, nq=nq, nk=nk, lens=lens,
+        cases.append(dict(case=c, layout=layout, d=d, B=B, H=H, Hkv=Hkv, nq=nq, nk=nk, lens=lens,
                           causal=causal, kv_pad=kv_pad, mask=mask, p=p, scale=scale,
                           seed=int(rng.integers(0, 2 ** 63))))
     return cases
@@ -74,7 +77,8 @@ CASES = _draw_cases(N_CASES)
 
 
 def _case_id(c):
-    parts = [f"c{c['case']:02d}", c["layout"], f"d{c['d']}", f"B{c['B']}H{c['H']}",
+    parts = [f"c{c['case']:02d}", c["layout"], f"d{c['d']}",
+             f"B{c['B']}H{c['H']}" + (f"kv{c['Hkv']}" if c["Hkv"] != c["H"] else ""),
              f"q{c['nq']}k{c['nk']}"]
     if c["causal"]:
         parts.append("causal")
@@ -108,6 +112,7 @@ def test_sweep_covers_every_feature():
     assert any(c["p"] > 0 and c["mask"] is not None for c in CASES)
     assert any(c["lens"] is not None and 0 in c["lens"][0] for c in CASES)
     assert any(c["lens"] is not None and 0 in c["lens"][1] for c in CASES)
+    assert {c["layout"] for c in CASES if c["Hkv"] != c["H"]} == {"bhsd", "bshd", "thd"}
 
 
 @pytest.mark.gpu
@@ -115,7 +120,8 @@ def test_sweep_covers_every_feature():
 def test_random_case_matches_oracle(lib, parity_record, c):
     import torch
     g = torch.Generator().manual_seed(c["seed"] % (2 ** 62))
-    B, H, d, layout = c["B"], c["H"], c["d"], c["layout"]
+    B, H, Hkv, d, layout = c["B"], c["H"], c["Hkv"], c["d"], c["layout"]
+    G = H // Hkv
     bm = None if c["mask"] is None else np.array(c["mask"], dtype=np.uint8)
     kv_pad = None if c["kv_pad"] is None else np.array(c["kv_pad"], dtype=np.int32)
     kw = dict(layout=layout, scale=c["scale"], causal=c["causal"], seqlens_k=kv_pad,
@@ -129,14 +135,14 @@ def test_random_case_matches_oracle(lib, parity_record, c):
         cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
         cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
         hq, hdo = rnd(int(cu_q[-1]), H, d), rnd(int(cu_q[-1]), H, d)
-        hk, hv = rnd(int(cu_k[-1]), H, d), rnd(int(cu_k[-1]), H, d)
+        hk, hv = rnd(int(cu_k[-1]), Hkv, d), rnd(int(cu_k[-1]), Hkv, d)
         kw.update(cu_seqlens_q=cu_q, cu_seqlens_k=cu_k, max_seqlen_q=c["nq"],
                   max_seqlen_k=c["nk"])
         to_dev = lambda x: x.cuda()  # noqa: E731
         to_host = f64
     else:
         hq, hdo = rnd(B, H, c["nq"], d), rnd(B, H, c["nq"], d)
-        hk, hv = rnd(B, H, c["nk"], d), rnd(B, H, c["nk"], d)
+        hk, hv = rnd(B, Hkv, c["nk"], d), rnd(B, Hkv, c["nk"], d)
         if layout == "bshd":
             to_dev = lambda x: x.transpose(1, 2).contiguous().cuda()  # noqa: E731
             to_host = lambda x: f64(x.transpose(1, 2))  # noqa: E731
@@ -152,19 +158,21 @@ def test_random_case_matches_oracle(lib, parity_record, c):
 
     ref_args = (c["scale"], c["causal"], kv_pad, c["p"], c["seed"], bm)
     if layout == "thd":
-        ro, rl = attention_forward_varlen(f64(hq), f64(hk), f64(hv), cu_q, cu_k, *ref_args)
+        ek, ev = gqa_expand(f64(hk), G), gqa_expand(f64(hv), G)  # [T, H, d]
+        ro, rl = attention_forward_varlen(f64(hq), ek, ev, cu_q, cu_k, *ref_args)
         # packed O [T, H, d] and LSE [H, T] viewed as one batch entry
         as_bhsd = lambda x: np.transpose(x, (1, 0, 2))[None]  # noqa: E731
         compare(as_bhsd(to_host(o)), lse.cpu().numpy().astype(np.float64)[None], as_bhsd(ro),
                 rl[None], parity_record)
     else:
-        ro, rl = attention_forward(f64(hq), f64(hk), f64(hv), *ref_args)
+        ro, rl = attention_forward_gqa(f64(hq), f64(hk), f64(hv), *ref_args)
         compare(to_host(o), lse.cpu().numpy().astype(np.float64), ro, rl, parity_record)
 
     if layout == "thd":
-        rg = attention_backward_varlen(f64(hq), f64(hk), f64(hv), f64(hdo), cu_q, cu_k, *ref_args)
+        rq, rk, rv = attention_backward_varlen(f64(hq), ek, ev, f64(hdo), cu_q, cu_k, *ref_args)
+        rg = (rq, gqa_reduce(rk, G), gqa_reduce(rv, G))
     else:
-        rg = attention_backward(f64(hq), f64(hk), f64(hv), f64(hdo), *ref_args)
+        rg = attention_backward_gqa(f64(hq), f64(hk), f64(hv), f64(hdo), *ref_args)
     errs = {}
     for name, a, r in zip(("dq", "dk", "dv"), grads, rg):
         got = to_host(a)
