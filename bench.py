@@ -13,7 +13,9 @@ their predecessor's last wave); the per-launch split comes from a second
 pass of the same steps with an event between every two launches.
 
 The default run times every workload (tiny, GPT-2, BERT, long d=64, long
-d=128, long d=256, block-sparse) one after the other.  The headline ``value`` is the
+d=128, long d=256, block-sparse) one after the other, plus the BERT batch
+packed and the long d=128 workload with grouped K / V heads (4 for the 16
+query heads) through the general entry points.  The headline ``value`` is the
 dense long-sequence case (B=1 H=16 N=16384 d=128 causal) timed over exactly
 K steps; ``per_config`` holds each workload (that one included, timed again
 for at least half a second so the clock record has many samples) with its
@@ -513,10 +515,37 @@ class PackedCase:
             ev[4].record(stream)
 
 
-def measure_packed(fa, w, args, rank, dev, flush, stream, world, local, peak):
-    """per_config entry of the packed BERT-shaped batch."""
+class GqaCase(PackedCase):
+    """The long causal d=128 workload with grouped K / V heads (4 K / V heads
+    for the 16 query heads: each shared by a group of 4), through fa_fwd_ex /
+    fa_bwd_ex.  The FLOPs are those of the same attention without grouping."""
+
+    KV_HEADS = 4
+
+    def __init__(self, fa, w, rank, dev):
+        import torch
+        self.w = w
+        inp = make_inputs(rank_workload(w, rank))
+        self.q, self.do = (inp[x].contiguous().to(dev) for x in ("q", "do"))
+        self.k, self.v = (inp[x][:, :self.KV_HEADS].contiguous().to(dev) for x in ("k", "v"))
+        self.kw = dict(scale=w.scale, causal=w.causal, dropout_p=w.dropout_p,
+                       seed=w.dropout_seed)
+        B, H, N, d = self.q.shape
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = (torch.empty_like(x) for x in (self.q, self.k, self.v))
+        self.ws = torch.empty(fa.general_workspace_size(self.q, self.k, **self.kw),
+                              dtype=torch.uint8, device=dev)
+        self.fa = fa
+        f = attention_flops(B, H, N, d, w.causal)[0]
+        self.flops = (f, 2.5 * f)
+
+
+def measure_packed(fa, w, args, rank, dev, flush, stream, world, local, peak, case_cls=None):
+    """per_config entry of the packed BERT-shaped batch (or, with case_cls, of
+    another fa_fwd_ex / fa_bwd_ex case)."""
     import torch
-    case = PackedCase(fa, w, rank, dev)
+    case = (case_cls or PackedCase)(fa, w, rank, dev)
     for _ in range(args.warmup):
         flush.zero_()
         case.step(stream)
@@ -535,7 +564,13 @@ def measure_packed(fa, w, args, rank, dev, flush, stream, world, local, peak):
     (fwd_ms, _, bwd_ms, _), total_ms, clocks = timed_region(case, steps, flush, stream, dev, world,
                                                            local)
     f_fwd, f_bwd = case.flops
-    entry = {"workload": describe(w) + " packed (fa_fwd_ex / fa_bwd_ex, no padding rows)",
+    if isinstance(case, GqaCase):
+        label = describe(w) + f" with {case.KV_HEADS} K / V heads (fa_fwd_ex / fa_bwd_ex)"
+        note = "as the same attention without grouping: 4 B H N^2 d forward, 2.5x backward, halved causal"
+    else:
+        label = describe(w) + " packed (fa_fwd_ex / fa_bwd_ex, no padding rows)"
+        note = "4 H d sum_b len_b^2 forward, 2.5x backward: every counted pair is valid"
+    entry = {"workload": label,
              "steps": steps, "timed_s": total_ms * 1e-3, "clocks": clocks,
              "device_status": fa.last_device_status(),
              "ms": {"fwd": fwd_ms, "bwd": bwd_ms, "step": total_ms / steps,
@@ -543,8 +578,9 @@ def measure_packed(fa, w, args, rank, dev, flush, stream, world, local, peak):
              "flops_per_launch": {"fwd_kernel": f_fwd, "bwd (3 launches)": f_bwd},
              "tflops": {"fwd": tflops(f_fwd, fwd_ms), "bwd": tflops(f_bwd, bwd_ms),
                         "fwd_bwd": tflops(f_fwd + f_bwd, total_ms / steps)},
-             "flops": "4 H d sum_b len_b^2 forward, 2.5x backward: every counted pair is valid",
-             "tokens": int(case.lens.sum())}
+             "flops": note}
+    if not isinstance(case, GqaCase):
+        entry["tokens"] = int(case.lens.sum())
     entry["pct_of_peak"] = {k: 100.0 * v / peak for k, v in entry["tflops"].items()}
     del case
     torch.cuda.empty_cache()
@@ -777,6 +813,9 @@ def run_ours(args):
             jobs.append((name, measure_config, WORKLOADS[name]))
             if name == "bert":
                 jobs.append(("bert_packed", measure_packed, WORKLOADS[name]))
+            if name == "long128":
+                jobs.append(("long128_gqa4", lambda *a: measure_packed(*a, case_cls=GqaCase),
+                             WORKLOADS[name]))
         for name in PROJ_SHAPES:
             jobs.append((name, measure_projection, name))
         for name, fn, wl in jobs:

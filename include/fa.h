@@ -310,6 +310,13 @@ void fa_set_wait_timeout_ns(uint64_t ns);
  * order of its fp32 reductions. */
 void fa_debug_set_block_mask_bitmap(int enabled);
 
+/* Test support: the number of parts a backward unit of grouped K / V heads
+ * is split into (each walking that share of the group's query heads and
+ * adding its dK / dV into fp32 accumulators).  0, the default, chooses it from
+ * the size of the problem; a value that does not divide the group is ignored.
+ * Applies to workspace sizes computed and launches made after the call. */
+void fa_debug_set_gqa_split(int parts);
+
 /* 1 in the bounds-checking build (FA_DEBUG_BOUNDS: every global-memory access
  * the kernels make outside TMA is checked against its buffer's extent, an
  * out-of-range one skipped and FA_ERR_BOUNDS recorded), 0 otherwise. */

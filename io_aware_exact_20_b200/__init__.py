@@ -128,6 +128,7 @@ SIGNATURES = {
     "fa_debug_wait_timeout": (_i, [_vp]),
     "fa_debug_set_block_mask_bitmap": (None, [_i]),
     "fa_debug_bounds_checking": (_i, []),
+    "fa_debug_set_gqa_split": (None, [_i]),
 }
 
 
@@ -299,6 +300,12 @@ def last_device_status(device=None):
 
 def set_wait_timeout_ns(ns):
     library().fa_set_wait_timeout_ns(int(ns))
+
+
+def set_gqa_split(parts):
+    """Test support: parts per backward unit under grouped K / V heads (0 =
+    chosen from the problem's size; ignored unless it divides the group)."""
+    library().fa_debug_set_gqa_split(int(parts))
 
 
 def set_block_mask_bitmap(enabled):

@@ -255,11 +255,39 @@ int64_t ws_rows(const Problem& p, int* npad, int64_t* rtot) {
   return static_cast<int64_t>(p.H) * *rtot;
 }
 
+// Parts per backward unit under grouped K / V heads: the smallest divisor of
+// the group whose parts give about four units per SM of the 148 (every divisor
+// up to the whole group when there are fewer); 1 without grouping.  A split
+// unit adds its dK / dV into fp32 accumulators converted at the end.
+std::atomic<int> g_gqa_split{0};  // test support: forced parts, 0 = automatic
+
+int split_of(const Problem& p) {
+  if (p.Hkv <= 0 || p.Hkv == p.H) return 1;
+  const int G = p.H / p.Hkv;
+  const int forced = g_gqa_split.load();
+  if (forced > 0 && G % forced == 0) return forced;
+  const int64_t units = static_cast<int64_t>(p.B) * p.Hkv * ((p.nk + 127) / 128) *
+                        (p.D == 256 ? 2 : 1);
+  int s = 1;
+  for (int c = 1; c <= G; ++c) {
+    if (G % c) continue;
+    s = c;
+    if (units * c >= 4 * 148) break;
+  }
+  return s;
+}
+
+// fp32 elements of each dK / dV accumulator of split units ([tb][H_kv][key rows][D])
+int64_t kv_acc_elems(const Problem& p) {
+  if (split_of(p) == 1) return 0;
+  return static_cast<int64_t>(p.tb()) * p.Hkv * p.rows_k() * p.D;
+}
+
 size_t workspace_bytes_of(const Problem& p) {
   int npad = 0;
   int64_t rtot = 0;
   const uint64_t rows = static_cast<uint64_t>(ws_rows(p, &npad, &rtot));
-  const uint64_t bytes = rows * (4ull + 4ull + 4ull * p.D);
+  const uint64_t bytes = rows * (4ull + 4ull + 4ull * p.D) + 8ull * kv_acc_elems(p);
   return static_cast<size_t>((bytes + 255) / 256 * 256);
 }
 
@@ -284,6 +312,7 @@ void set_extents(const Problem& pr, int* status, fa::Extents* e, fa::Rows* rows)
                 ? static_cast<long long>((pr.nq + 127) / 128) * ((pr.nk + 127) / 128)
                 : 0;
   e->seqlens = pr.seqlens != nullptr ? pr.B : 0;
+  e->kvacc = kv_acc_elems(pr);
   rows->n_cu = pr.packed ? pr.B + 1 : 0;
   rows->status = status;
 }
@@ -352,6 +381,9 @@ fa_status_t bwd_params(fa::BwdParams* p, const Problem& pr, const void* workspac
   p->ws_delta = p->ws_lse2 + rows;
   p->ws_dq = p->ws_delta + rows;
   p->ws_rows = rows;
+  p->split = split_of(pr);
+  p->ws_dk = p->split > 1 ? p->ws_dq + rows * pr.D : nullptr;
+  p->ws_dv = p->split > 1 ? p->ws_dk + kv_acc_elems(pr) : nullptr;
   p->Npad = npad;
   p->Rtot = rtot;
   lse_strides(pr, &p->lse_sb, &p->lse_sh);
@@ -432,10 +464,16 @@ fa_status_t run_bwd(const Problem& pr, const void* q, const void* k, const void*
   p.dv = dv;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (fa::launch_bwd_pre(pr.D, p, s) != cudaSuccess) return FA_ERR_CUDA;
+  // split units add their dK / dV into accumulators that start at zero
+  if (p.split > 1 &&
+      cudaMemsetAsync(p.ws_dk, 0, 2 * sizeof(float) * kv_acc_elems(pr), s) != cudaSuccess)
+    return FA_ERR_CUDA;
   if (fa::launch_bwd_main(pr.D, p.drop_threshold != 0, m.q, m.k, m.v, m.dout, m.dq, p, s) !=
       cudaSuccess)
     return FA_ERR_CUDA;
-  return fa::launch_bwd_post(pr.D, p, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  if (fa::launch_bwd_post(pr.D, p, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (p.split > 1 && fa::launch_bwd_kv_post(pr.D, p, s) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
 }
 
 }  // namespace
@@ -458,6 +496,8 @@ const char* fa_status_string(fa_status_t s) {
 void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns < 1000000ull ? 1000000ull : ns); }
 
 void fa_debug_set_block_mask_bitmap(int enabled) { g_mask_bitmap.store(enabled != 0 ? 1 : 0); }
+
+void fa_debug_set_gqa_split(int parts) { g_gqa_split.store(parts > 0 ? parts : 0); }
 
 int fa_debug_bounds_checking(void) {
 #ifdef FA_DEBUG_BOUNDS

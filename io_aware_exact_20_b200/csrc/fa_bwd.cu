@@ -213,10 +213,11 @@ struct BwdWork {
   __device__ __forceinline__ bool more(Tile t, int G) const {
     return GEN ? tile_g<true>(t) < G : t < nqb;
   }
-  // query head of step t, and the workspace row of its query tile's first row
-  // (ws_hs: workspace rows from one query head to the next)
+  // query head of step t (base: the first query head the CTA walks), and the
+  // workspace row of its query tile's first row (ws_hs: workspace rows from
+  // one query head to the next)
   template <bool GEN>
-  __device__ __forceinline__ int hq(Tile t, int G) const { return hk * G + tile_g<GEN>(t); }
+  __device__ __forceinline__ int hq(Tile t, int base) const { return base + tile_g<GEN>(t); }
   template <bool GEN>
   __device__ __forceinline__ long long wsrow(Tile t, long long ws_hs) const {
     return ws0 + tile_g<GEN>(t) * ws_hs + 128ll * tile_qb<GEN>(t);
@@ -311,6 +312,38 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
   *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dq) + dq_off) = out;
 }
 
+// dK, dV = bf16(fp32 accumulators) of split units (grouped K / V heads): grid
+// (blocks of kRowsPerBlock<D> key rows of the longest sequence) x (B * H_kv).
+// The accumulators hold the scaled gradients already.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_kv_post_kernel(const BwdParams p) {
+  constexpr int G = D / 8;
+  griddep_wait();
+  griddep_launch_dependents();
+  const int n_kv = p.H / p.group;
+  const int bh = blockIdx.y;
+  const int b = bh / n_kv, hk = bh % n_kv;
+  const Seq sq = seq_of(p.rows, b);
+  const int j = blockIdx.x * kRowsPerBlock<D> + static_cast<int>(threadIdx.x) / G;
+  const int part = static_cast<int>(threadIdx.x) % G;
+  if (j >= sq.lk || part * 8 >= p.d_real) return;
+  const long long rows_k = p.rows.cu_k == nullptr ? p.rows.nk : p.rows.total_k;
+  const long long kr = static_cast<long long>(sq.k0) + j;
+  const long long acc = ((static_cast<long long>(sq.tb) * n_kv + hk) * rows_k + kr) * D + part * 8;
+  const long long dk_off = sq.tb * p.sdk.b + hk * p.sdk.h + kr * p.sdk.r + part * 8;
+  const long long dv_off = sq.tb * p.sdv.b + hk * p.sdv.h + kr * p.sdv.r + part * 8;
+  if (!FA_IN_BOUNDS(p.status, acc, 8, p.ext.kvacc) || !FA_IN_BOUNDS(p.status, dk_off, 8, p.ext.dk) ||
+      !FA_IN_BOUNDS(p.status, dv_off, 8, p.ext.dv))
+    return;
+  auto cvt = [&](const float* src, void* dst) {
+    const float4 x = reinterpret_cast<const float4*>(src)[0], y = reinterpret_cast<const float4*>(src)[1];
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w),
+                                                pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
+  };
+  cvt(p.ws_dk + acc, static_cast<__nv_bfloat16*>(p.dk) + dk_off);
+  cvt(p.ws_dv + acc, static_cast<__nv_bfloat16*>(p.dv) + dv_off);
+}
+
 // ---------------------------------------------------------------------------
 // main kernel
 // ---------------------------------------------------------------------------
@@ -351,11 +384,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int hf = L::RING ? static_cast<int>(blockIdx.x & 1u) : 0;
   const long long unit = L::RING ? static_cast<long long>(blockIdx.x >> 1) : blockIdx.x;
   const int G = GEN ? p.group : 1;  // query heads per K / V head
+  const int S = GEN ? p.split : 1;  // parts of a unit (adjacent CTAs)
+  const int Gw = G / S;             // query heads one part walks
+  const int part = GEN ? static_cast<int>(unit % S) : 0;
   const int n_kv_heads = p.H / G;
-  grid_unit(unit, p.B * n_kv_heads, (p.rows.nk + 127) / 128, p.group_heads, &w.bh,
-            &w.kb);  // key tile 0 is heaviest
+  grid_unit(GEN ? unit / S : unit, p.B * n_kv_heads, (p.rows.nk + 127) / 128, p.group_heads,
+            &w.bh, &w.kb);  // key tile 0 is heaviest
   w.b = w.bh / n_kv_heads;
   w.hk = w.bh % n_kv_heads;
+  const int hq_base = w.hk * G + part * Gw;  // first query head of this part
   {
     const Seq sq = seq_of(p.rows, w.b);
     // a sequence shorter than the longest has no key tile here: leave before
@@ -371,7 +408,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     w.tb = sq.tb;
     w.off = sq.lk - sq.lq;
     w.nqb = (sq.lq + 127) / 128;
-    w.ws0 = ws_row0(p, w.b, w.hk * G, sq.q0);
+    w.ws0 = ws_row0(p, w.b, hq_base, sq.q0);
   }
   w.alive = w.kb * 128 < w.kv_len;
   w.causal = p.causal != 0;
@@ -434,9 +471,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   // the walk with this launch's group size and workspace rows per query head
   const long long ws_hs = p.rows.cu_q == nullptr ? p.Npad : p.Rtot;
-  auto more = [&](Tile t) { return w.template more<GEN>(t, G); };
+  auto more = [&](Tile t) { return w.template more<GEN>(t, Gw); };
   auto next_t = [&](Tile t) { return w.template step<GEN>(t); };
-  const Tile t_first = w.template first<GEN>(G);
+  const Tile t_first = w.template first<GEN>(Gw);
   const bool any_work = more(t_first);
 
   if (warp < 4) {
@@ -472,7 +509,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             return false;
           mbar_arrive_expect_tx(bar(L::B_QFULL + s), L::PANEL);
           tma_load_4d(sbase + L::OFF_Q + s * L::PANEL, m, bar(L::B_QFULL + s), 64 * pn,
-                      w.qrow + tile_qb<GEN>(tt) * 128, w.template hq<GEN>(tt, G), w.tb);
+                      w.qrow + tile_qb<GEN>(tt) * 128, w.template hq<GEN>(tt, hq_base), w.tb);
           ++t;
           return true;
         };
@@ -515,7 +552,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t ph = (it / L::STAGES) & 1u;
         if (it >= L::STAGES && !mbar_wait(bar(L::B_QEMPTY + s), ph ^ 1u, g)) break;
         mbar_arrive_expect_tx(bar(L::B_QFULL + s), 2 * L::TILE + 1024);
-        const int hq = w.template hq<GEN>(tc, G);
+        const int hq = w.template hq<GEN>(tc, hq_base);
         for (int pn = 0; pn < L::PANELS; ++pn) {
           tma_load_4d(sbase + L::OFF_Q + s * L::TILE + pn * L::PANEL, &tm_q, bar(L::B_QFULL + s),
                       64 * pn, w.qrow + tile_qb<GEN>(tc) * 128, hq, w.tb);
@@ -598,7 +635,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int n_total = 0;
       if constexpr (GEN) {
         for (int qb = w.next(w.qb_begin); qb < w.nqb; qb = w.next(qb + 1)) ++n_total;
-        n_total *= G;
+        n_total *= Gw;
       }
       auto mma_more = [&](Tile t, int i) { return GEN ? i < n_total : more(t); };
       auto mma_next = [&](Tile t) { return GEN ? t : next_t(t); };
@@ -840,7 +877,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint32_t qg = (GEN ? p.drop_row0 : 0u) +
                                 static_cast<uint32_t>(qb * 128 + qoff + 8 * gq + (lane & 7));
             const Philox4 rnd = philox4x32_10((GEN ? p.drop_kgrp0 : 0u) + static_cast<uint32_t>(jg >> 3), qg,
-                                              static_cast<uint32_t>(w.template hq<GEN>(tc, G)), static_cast<uint32_t>(w.b),
+                                              static_cast<uint32_t>(w.template hq<GEN>(tc, hq_base)), static_cast<uint32_t>(w.b),
                                               p.rk);
             own |= keep_byte(rnd, thr) << (8 * gq);
           }
@@ -1080,8 +1117,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         const long long dv_off = w.tb * p.sdv.b + w.hk * p.sdv.h + kr * p.sdv.r + col;
         const long long dk_off = w.tb * p.sdk.b + w.hk * p.sdk.h + kr * p.sdk.r + col;
-        if (row_ok && col < p.d_real && FA_IN_BOUNDS(p.status, dv_off, 32, p.ext.dv) &&
-            FA_IN_BOUNDS(p.status, dk_off, 32, p.ext.dk)) {
+        if (GEN && S > 1) {
+          // one part of a split unit: its dK / dV go into the fp32 accumulators
+          // ([tb][H_kv][key rows][D]), converted once every part is done
+          const long long rows_k = p.rows.cu_k == nullptr ? p.rows.nk : p.rows.total_k;
+          const long long acc =
+              ((static_cast<long long>(w.tb) * n_kv_heads + w.hk) * rows_k + kr) * D + col;
+          if (row_ok && col < p.d_real && any_work && n_it > 0 &&
+              FA_IN_BOUNDS(p.status, acc, 32, p.ext.kvacc)) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              red_add_f32(p.ws_dv + acc + k, __uint_as_float(a[k]) * p.drop_rscale);
+              red_add_f32(p.ws_dk + acc + k, __uint_as_float(bk[k]) * p.scale);
+            }
+          }
+        } else if (row_ok && col < p.d_real && FA_IN_BOUNDS(p.status, dv_off, 32, p.ext.dv) &&
+                   FA_IN_BOUNDS(p.status, dk_off, 32, p.ext.dk)) {
           uint4* dvp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + dv_off);
           uint4* dkp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + dk_off);
 #pragma unroll
@@ -1234,7 +1285,7 @@ cudaError_t launch_main_t(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   if (e != cudaSuccess) return e;
   // one unit per (b, K / V head, key tile); d = 256: two CTAs (column halves) each
   const long long ctas = static_cast<long long>((p.rows.nk + 127) / 128) * p.B *
-                         (p.H / (GEN ? p.group : 1)) * (L::RING ? 2 : 1);
+                         (p.H / (GEN ? p.group : 1)) * (GEN ? p.split : 1) * (L::RING ? 2 : 1);
   if (ctas > 0x7FFFFFFFll) return cudaErrorInvalidConfiguration;
   return launch_overlapped(kern, dim3(static_cast<unsigned>(ctas)), dim3(kBwdThreads), L::SMEM,
                            stream, tq, tk, tv, tdo, tdq, p);
@@ -1285,6 +1336,17 @@ cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CU
                                : launch_main_t<128, false, false>(tq, tk, tv, tdo, tdq, p, stream);
   if (d == 256) return dropout ? launch_main_t<256, true, false>(tq, tk, tv, tdo, tdq, p, stream)
                                : launch_main_t<256, false, false>(tq, tk, tv, tdo, tdq, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_kv_post(int d, const BwdParams& p, cudaStream_t stream) {
+  const long long rows = (static_cast<long long>(p.rows.nk) + 127) / 128 * 128;
+  auto grid = [&](int rpb) {
+    return dim3(static_cast<unsigned>(rows / rpb), static_cast<unsigned>(p.B * (p.H / p.group)), 1);
+  };
+  if (d == 64) return launch_overlapped(bwd_kv_post_kernel<64>, grid(kRowsPerBlock<64>), dim3(256), 0, stream, p);
+  if (d == 128) return launch_overlapped(bwd_kv_post_kernel<128>, grid(kRowsPerBlock<128>), dim3(256), 0, stream, p);
+  if (d == 256) return launch_overlapped(bwd_kv_post_kernel<256>, grid(kRowsPerBlock<256>), dim3(256), 0, stream, p);
   return cudaErrorInvalidValue;
 }
 

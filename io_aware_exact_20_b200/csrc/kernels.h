@@ -84,7 +84,7 @@ enum : int { kStatusOk = 0, kStatusInternal = 3, kStatusTimeout = 4, kStatusBoun
 // Other builds compile the checks away (the macro drops its arguments).
 #ifdef FA_DEBUG_BOUNDS
 struct Extents {
-  long long o, lse, dout, dq, dk, dv, mask, seqlens;
+  long long o, lse, dout, dq, dk, dv, mask, seqlens, kvacc;
 };
 __device__ __forceinline__ bool in_bounds(int* status, long long off, long long width,
                                           long long extent) {
@@ -214,6 +214,12 @@ struct BwdParams {
   int mask_bitmap;            // as in FwdParams
   int group;                  // query heads per K / V head; the main kernel's units are
                               // (b, K / V head, key tile) and walk the group's query heads
+  int split;                  // > 1: each unit splits into `split` parts, part p walking
+                              // query heads [p, p + 1) * group / split of the group and
+                              // adding its dK / dV into ws_dk / ws_dv (general instances)
+  // fp32 dK / dV accumulators [tb][H_kv][key rows][D] when split > 1
+  float* ws_dk;
+  float* ws_dv;
 #ifdef FA_DEBUG_BOUNDS
   Extents ext;
 #endif
@@ -237,6 +243,8 @@ cudaError_t launch_bwd_main(int d, bool dropout, const CUtensorMap& tq, const CU
                             const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdq,
                             const BwdParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_post(int d, const BwdParams& p, cudaStream_t stream);
+// dK, dV from the fp32 accumulators of split units (BwdParams::split > 1)
+cudaError_t launch_bwd_kv_post(int d, const BwdParams& p, cudaStream_t stream);
 
 // Fused QKV projection (fa_proj.cu): x bf16 [B N, d_model], w bf16
 // [3 H d, d_model], bias bf16 [3 H d] or null -> q, k, v bf16 [B, H, N, d].

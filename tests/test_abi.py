@@ -34,6 +34,19 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     so = lib.library()
     assert so.fa_status_string(6).startswith(b"a kernel index was out of bounds")
+    # grouped K / V heads with few units: split parts need fp32 dK / dV accumulators
+    st, sk = lib.Strides(3 * 256 * 64, 256 * 64, 64), lib.Strides(1 * 384 * 64, 384 * 64, 64)
+    a = _desc(lib, heads_kv=1, q=st, o=st, dout=st, dq=st, k=sk, v=sk, dk=sk, dv=sk)
+    base = 2 * 3 * 256 * (8 + 256)
+    lib.set_gqa_split(1)
+    try:
+        assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == base
+        lib.set_gqa_split(3)   # three parts of the group of 3: two accumulators of 2 x 384 x 64
+        assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == base + 2 * 4 * 2 * 384 * 64
+        lib.set_gqa_split(2)   # does not divide the group: the automatic choice (3 here)
+        assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == base + 2 * 4 * 2 * 384 * 64
+    finally:
+        lib.set_gqa_split(0)
     # the default library is the production build (no bounds checks)
     if not os.environ.get("FA_B200_LIBRARY"):
         assert so.fa_debug_bounds_checking() == 0
@@ -136,9 +149,13 @@ def test_general_entry_points_validate_before_launching(lib, change, code):
     a = _desc(lib, **kw)
     ws = so.fa_bwd_ex_workspace_size(ctypes.byref(a))
     if code is None:
-        # padded layout: B * H * ceil(N_q / 128) * 128 rows of 8 + 4 * 64 bytes
+        # padded layout: B * H * ceil(N_q / 128) * 128 rows of 8 + 4 * 64 bytes,
+        # and with grouped K / V heads the split units' dK / dV accumulators
         # (a valid description is never launched here: the addresses are fake)
-        assert ws == 2 * 3 * 256 * (8 + 256)
+        if change.get("heads_kv", 3) == 3:
+            assert ws == 2 * 3 * 256 * (8 + 256)
+        else:
+            assert ws > 2 * 3 * 256 * (8 + 256)
         return
     assert ws == 0
     assert so.fa_fwd_ex(ctypes.byref(a), A16, A16, A16, A16, A16, None) == code

@@ -111,3 +111,29 @@ def test_gqa_forward_equals_repeated_heads(lib):
     torch.cuda.synchronize()
     assert lib.last_device_status() == 0
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("parts", [1, 2, 4])
+@pytest.mark.parametrize("d", [64, 128])
+def test_gqa_backward_split_parts(lib, parity_record, parts, d):
+    """A unit of the grouped backward walks its group's query heads in one
+    thread block (parts = 1: dK / dV accumulate in TMEM and are stored once),
+    or is split into parts that each walk their share and add dK / dV into fp32
+    accumulators converted at the end; every split gives the oracle's result."""
+    import torch
+    B, H, Hkv, N = 1, 8, 2, 520
+    qh, doh = randn((B, H, N, d), 61), randn((B, H, N, d), 62)
+    kh, vh = randn((B, Hkv, N, d), 63), randn((B, Hkv, N, d), 64)
+    kw = dict(causal=True, dropout_p=0.1, seed=65)
+    q, k, v, do = (x.cuda() for x in (qh, kh, vh, doh))
+    lib.set_gqa_split(parts)
+    try:
+        o, lse = lib.forward_general(q, k, v, **kw)
+        grads = lib.backward_general(q, k, v, o, lse, do, **kw)
+        torch.cuda.synchronize()
+        assert lib.last_device_status() == 0
+    finally:
+        lib.set_gqa_split(0)
+    args = (d ** -0.5, True, None, 0.1, 65)
+    rg = attention_backward_gqa(f64(qh), f64(kh), f64(vh), f64(doh), *args)
+    check_grads(tuple(f64(x) for x in grads), rg, parity_record)
