@@ -234,7 +234,10 @@ fa_status_t fa_fwd_ex(const fa_attention_desc_t* desc, const void* q, const void
 /* Workspace bytes of fa_bwd_ex: padded layout B * H * ceil(seqlen_q / 128) * 128
  * rows, packed layout H * (ceil(total_q / 128) * 128 + 256 B) rows, each of
  * 8 + 4 D bytes (D = 64 for d <= 64, 128 for d = 96 / 128, 256 for d = 192 /
- * 256).  0 if the description is invalid. */
+ * 256); with grouped K / V heads whose backward units are split into parts
+ * (few units for the SM count), two fp32 dK / dV accumulators of
+ * tb * heads_kv * key rows * D elements more (tb = B padded, 1 packed; key rows
+ * = seqlen_k padded, total_k packed).  0 if the description is invalid. */
 size_t fa_bwd_ex_workspace_size(const fa_attention_desc_t* desc);
 
 /* Backward pass for a general layout (dQ like Q, dK / dV like K / V; the
