@@ -185,7 +185,6 @@ def test_ring_with_library_kernels_on_one_gpu(lib, parity_record, world, d, caus
     from io_aware_exact_20_b200 import context_parallel as cp
     from io_aware_exact_20_b200.workloads import make_qkvdo
     from oracle import attention_backward, attention_forward
-    from test_gpu_fwd import compare
     B, H, N = 1, 2, 192 * world
     q, k, v, do = make_qkvdo(B, H, N, d, 81)
     n = N // world
@@ -203,6 +202,12 @@ def test_ring_with_library_kernels_on_one_gpu(lib, parity_record, world, d, caus
     f = lambda t: t.float().cpu().numpy().astype(np.float64)  # noqa: E731
     ro, rl = attention_forward(f(q), f(k), f(v), scale, causal, None, p, SEED)
     rg = attention_backward(f(q), f(k), f(v), f(do), scale, causal, None, p, SEED)
+    _check_ring(outs, grads, ro, rl, rg, world, parity_record)
+
+
+def _check_ring(outs, grads, ro, rl, rg, world, parity_record):
+    from test_gpu_fwd import compare
+    f = lambda t: t.float().cpu().numpy().astype(np.float64)  # noqa: E731
     o = np.concatenate([f(outs[r][0]) for r in range(world)], axis=2)
     lse = np.concatenate([outs[r][1].cpu().numpy() for r in range(world)], axis=2)
     compare(o, lse.astype(np.float64), ro, rl, parity_record)
@@ -210,3 +215,35 @@ def test_ring_with_library_kernels_on_one_gpu(lib, parity_record, world, d, caus
         g = np.concatenate([f(grads[r][i]) for r in range(world)], axis=2)
         e = np.linalg.norm(g - rg[i]) / np.linalg.norm(rg[i])
         assert e <= 2e-2, (name, e)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("world,Hkv,p", [(2, 1, 0.1), (4, 2, 0.0)])
+def test_ring_with_grouped_kv_heads(lib, parity_record, world, Hkv, p):
+    """The ring passes K / V chunks with fewer heads than the queries (grouped
+    K / V heads): every call reads K / V head h // (H / H_kv), and the dK / dV
+    accumulators that travel with a chunk have its K / V heads."""
+    import torch
+
+    from io_aware_exact_20_b200 import context_parallel as cp
+    from io_aware_exact_20_b200.workloads import make_qkvdo
+    from oracle import attention_backward_gqa, attention_forward_gqa
+    B, H, N, d = 1, 4, 192 * world, 128
+    q, _, _, do = make_qkvdo(B, H, N, d, 83)
+    _, k, v, _ = make_qkvdo(B, Hkv, N, d, 84)
+    n = N // world
+    ch = [[x[:, :, r * n:(r + 1) * n].contiguous().cuda() for x in (q, k, v, do)]
+          for r in range(world)]
+    kern = cp.LibraryKernels(lib)
+    scale = d ** -0.5
+    outs = cp.run_emulated([cp.ring_forward(r, world, *ch[r][:3], scale, True, kern, p, SEED)
+                            for r in range(world)])
+    grads = cp.run_emulated([cp.ring_backward(r, world, *ch[r][:3], outs[r][0], outs[r][1],
+                                              ch[r][3], scale, True, kern, p, SEED)
+                             for r in range(world)])
+    torch.cuda.synchronize()
+    assert lib.last_device_status() == 0
+    f = lambda t: t.float().cpu().numpy().astype(np.float64)  # noqa: E731
+    ro, rl = attention_forward_gqa(f(q), f(k), f(v), scale, True, None, p, SEED)
+    rg = attention_backward_gqa(f(q), f(k), f(v), f(do), scale, True, None, p, SEED)
+    _check_ring(outs, grads, ro, rl, rg, world, parity_record)
