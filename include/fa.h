@@ -219,8 +219,10 @@ typedef struct {
   int64_t dropout_row0, dropout_key0;
   /* Grouped-query attention: K and V (and dK, dV) have heads_kv heads, and
    * query head h reads K / V head h / (heads / heads_kv); heads_kv must divide
-   * heads (otherwise FA_ERR_INVALID_ARG).  0, or heads: one K / V head per
-   * query head.  dK and dV of a K / V head are the sums over its query heads. */
+   * heads (otherwise FA_ERR_INVALID_ARG), with fewer than 32768 query heads
+   * per K / V head (otherwise FA_ERR_UNSUPPORTED).  0, or heads: one K / V
+   * head per query head.  dK and dV of a K / V head are the sums over its
+   * query heads. */
   int heads_kv;
 } fa_attention_desc_t;
 

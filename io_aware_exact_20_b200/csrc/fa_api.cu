@@ -124,6 +124,8 @@ fa_status_t resolve(const fa_attention_desc_t* a, Problem* p, Uses uses) {
   // grouped-query attention: heads_kv K / V heads, each shared by heads / heads_kv
   const int hkv = a->heads_kv == 0 ? a->heads : a->heads_kv;
   if (hkv < 1 || hkv > a->heads || a->heads % hkv != 0) return FA_ERR_INVALID_ARG;
+  // the backward's walk packs (query head of the group, query tile) in 16 + 16 bits
+  if (a->heads / hkv >= 32768) return FA_ERR_UNSUPPORTED;
   const fa_strides_t* all[8] = {&a->q, &a->k, &a->v, &a->o, &a->dout, &a->dq, &a->dk, &a->dv};
   const bool kv_side[8] = {false, true, true, false, false, false, true, true};
   for (int t = 0; t < (uses == kForward ? 4 : 8); ++t) {

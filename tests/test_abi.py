@@ -142,6 +142,7 @@ def _desc(lib, **kw):
     (dict(dropout_key0=(1 << 40)), 1),
     (dict(heads_kv=1), None), (dict(heads_kv=3), None),   # grouped K / V heads (3 query heads)
     (dict(heads_kv=2), 1), (dict(heads_kv=4), 1), (dict(heads_kv=-1), 1),
+    (dict(batch=1, heads=32768, heads_kv=1), 2),           # group too large for the walk
 ])
 def test_general_entry_points_validate_before_launching(lib, change, code):
     so = lib.library()
