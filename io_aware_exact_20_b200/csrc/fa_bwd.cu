@@ -163,7 +163,7 @@ __device__ __forceinline__ int tile_qb(Tile t) { return GEN ? t & 0xFFFF : t; }
 template <bool kBits>
 struct BwdWork {
   int b, hk, bh, kb, kv_len, nqb, qb_begin, nbk, off, qrow, krow, tb, lk;  // hk: K / V head
-  long long ws0;  // first workspace row of query head hk * G (G = 1: the only one)
+  long long ws0;  // first workspace row of the first query head the CTA walks
   bool alive, causal;
   const uint8_t* bm;
   const uint32_t* bits;  // shared-memory bitmask over the query tiles, or null

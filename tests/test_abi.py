@@ -250,3 +250,26 @@ def test_nvtx_ranges_wrap_the_entry_points(lib, monkeypatch):
     with pytest.raises(ValueError):
         lib.forward(q, q, q)
     assert calls == []
+
+
+def test_gqa_split_is_chosen_from_the_units(lib):
+    """Grouped K / V heads: a backward unit is split into the fewest parts
+    (a divisor of the group) giving about four units per SM (592); the split
+    units' dK / dV accumulators show in the workspace size."""
+    so = lib.library()
+    N, d = 16384, 128
+
+    def ws(B, H, Hkv):
+        st, sk = lib.Strides(H * N * d, N * d, d), lib.Strides(Hkv * N * d, N * d, d)
+        a = _desc(lib, batch=B, heads=H, heads_kv=Hkv, head_dim=d, seqlen_q=N, seqlen_k=N,
+                  q=st, o=st, dout=st, dq=st, k=sk, v=sk, dk=sk, dv=sk)
+        return so.fa_bwd_ex_workspace_size(ctypes.byref(a))
+
+    def base(B, H):
+        return B * H * N * (8 + 4 * d)
+
+    acc = lambda B, Hkv: 2 * 4 * B * Hkv * N * d  # noqa: E731  two fp32 accumulators
+    assert ws(1, 16, 16) == base(1, 16)                  # no grouping: no split
+    assert ws(1, 16, 1) == base(1, 16) + acc(1, 1)       # 128 units: split into 8 parts
+    assert ws(1, 16, 4) == base(1, 16) + acc(1, 4)       # 512 units: 2 parts
+    assert ws(2, 16, 4) == base(2, 16)                   # 1024 units: whole groups
