@@ -162,10 +162,16 @@ def read_peaks():
 
 
 def source_sha(files):
+    """Hash of the kernel sources with their comments and blank space removed
+    (a comment-only edit builds the same kernel and keeps its records)."""
+    import re
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "io_aware_exact_20_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "io_aware_exact_20_b200", "csrc", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
