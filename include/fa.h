@@ -222,7 +222,9 @@ typedef struct {
    * heads (otherwise FA_ERR_INVALID_ARG), with fewer than 32768 query heads
    * per K / V head (otherwise FA_ERR_UNSUPPORTED).  0, or heads: one K / V
    * head per query head.  dK and dV of a K / V head are the sums over its
-   * query heads. */
+   * query heads; when the backward splits a group over several thread blocks
+   * (few K / V heads and key tiles for the GPU), they are added with fp32
+   * atomics like dQ, so their last bits may vary between runs. */
   int heads_kv;
 } fa_attention_desc_t;
 
