@@ -222,9 +222,9 @@ typedef struct {
    * heads (otherwise FA_ERR_INVALID_ARG), with fewer than 32768 query heads
    * per K / V head (otherwise FA_ERR_UNSUPPORTED).  0, or heads: one K / V
    * head per query head.  dK and dV of a K / V head are the sums over its
-   * query heads; when the backward splits a group over several thread blocks
-   * (few K / V heads and key tiles for the GPU), they are added with fp32
-   * atomics like dQ, so their last bits may vary between runs. */
+   * query heads, deterministic as without grouping (when the backward splits
+   * a group over several thread blocks, each writes its own fp32 partial sums
+   * and they are added in a fixed order). */
   int heads_kv;
 } fa_attention_desc_t;
 
@@ -238,10 +238,10 @@ fa_status_t fa_fwd_ex(const fa_attention_desc_t* desc, const void* q, const void
 /* Workspace bytes of fa_bwd_ex: padded layout B * H * ceil(seqlen_q / 128) * 128
  * rows, packed layout H * (ceil(total_q / 128) * 128 + 256 B) rows, each of
  * 8 + 4 D bytes (D = 64 for d <= 64, 128 for d = 96 / 128, 256 for d = 192 /
- * 256); with grouped K / V heads whose backward units are split into parts
- * (few units for the SM count), two fp32 dK / dV accumulators of
- * tb * heads_kv * key rows * D elements more (tb = B padded, 1 packed; key rows
- * = seqlen_k padded, total_k packed).  0 if the description is invalid. */
+ * 256); with grouped K / V heads whose backward units are split into S parts
+ * (few units for the SM count), two fp32 dK / dV areas of
+ * S * tb * heads_kv * key rows * D elements more (tb = B padded, 1 packed; key
+ * rows = seqlen_k padded, total_k packed).  0 if the description is invalid. */
 size_t fa_bwd_ex_workspace_size(const fa_attention_desc_t* desc);
 
 /* Backward pass for a general layout (dQ like Q, dK / dV like K / V; the

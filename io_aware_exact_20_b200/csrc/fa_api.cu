@@ -279,10 +279,12 @@ int split_of(const Problem& p) {
   return s;
 }
 
-// fp32 elements of each dK / dV accumulator of split units ([tb][H_kv][key rows][D])
+// fp32 elements of each of the dK / dV areas of split units: one slice
+// [tb][H_kv][key rows][D] per part
 int64_t kv_acc_elems(const Problem& p) {
-  if (split_of(p) == 1) return 0;
-  return static_cast<int64_t>(p.tb()) * p.Hkv * p.rows_k() * p.D;
+  const int s = split_of(p);
+  if (s == 1) return 0;
+  return static_cast<int64_t>(s) * p.tb() * p.Hkv * p.rows_k() * p.D;
 }
 
 size_t workspace_bytes_of(const Problem& p) {
@@ -384,6 +386,7 @@ fa_status_t bwd_params(fa::BwdParams* p, const Problem& pr, const void* workspac
   p->ws_dq = p->ws_delta + rows;
   p->ws_rows = rows;
   p->split = split_of(pr);
+  p->rows_tb = pr.tb();
   p->ws_dk = p->split > 1 ? p->ws_dq + rows * pr.D : nullptr;
   p->ws_dv = p->split > 1 ? p->ws_dk + kv_acc_elems(pr) : nullptr;
   p->Npad = npad;
@@ -466,10 +469,6 @@ fa_status_t run_bwd(const Problem& pr, const void* q, const void* k, const void*
   p.dv = dv;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (fa::launch_bwd_pre(pr.D, p, s) != cudaSuccess) return FA_ERR_CUDA;
-  // split units add their dK / dV into accumulators that start at zero
-  if (p.split > 1 &&
-      cudaMemsetAsync(p.ws_dk, 0, 2 * sizeof(float) * kv_acc_elems(pr), s) != cudaSuccess)
-    return FA_ERR_CUDA;
   if (fa::launch_bwd_main(pr.D, p.drop_threshold != 0, m.q, m.k, m.v, m.dout, m.dq, p, s) !=
       cudaSuccess)
     return FA_ERR_CUDA;

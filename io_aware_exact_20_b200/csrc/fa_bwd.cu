@@ -312,9 +312,9 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const BwdParams p) {
   *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dq) + dq_off) = out;
 }
 
-// dK, dV = bf16(fp32 accumulators) of split units (grouped K / V heads): grid
-// (blocks of kRowsPerBlock<D> key rows of the longest sequence) x (B * H_kv).
-// The accumulators hold the scaled gradients already.
+// dK, dV = bf16(sum over the parts' fp32 slices) of split units (grouped K / V
+// heads), the parts added in order: grid (blocks of kRowsPerBlock<D> key rows
+// of the longest sequence) x (B * H_kv).  The slices hold scaled gradients.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_kv_post_kernel(const BwdParams p) {
   constexpr int G = D / 8;
@@ -330,13 +330,20 @@ __global__ void __launch_bounds__(256) bwd_kv_post_kernel(const BwdParams p) {
   const long long rows_k = p.rows.cu_k == nullptr ? p.rows.nk : p.rows.total_k;
   const long long kr = static_cast<long long>(sq.k0) + j;
   const long long acc = ((static_cast<long long>(sq.tb) * n_kv + hk) * rows_k + kr) * D + part * 8;
+  const long long slice = static_cast<long long>(p.rows_tb) * n_kv * rows_k * D;
   const long long dk_off = sq.tb * p.sdk.b + hk * p.sdk.h + kr * p.sdk.r + part * 8;
   const long long dv_off = sq.tb * p.sdv.b + hk * p.sdv.h + kr * p.sdv.r + part * 8;
-  if (!FA_IN_BOUNDS(p.status, acc, 8, p.ext.kvacc) || !FA_IN_BOUNDS(p.status, dk_off, 8, p.ext.dk) ||
-      !FA_IN_BOUNDS(p.status, dv_off, 8, p.ext.dv))
+  if (!FA_IN_BOUNDS(p.status, acc + (p.split - 1) * slice, 8, p.ext.kvacc) ||
+      !FA_IN_BOUNDS(p.status, dk_off, 8, p.ext.dk) || !FA_IN_BOUNDS(p.status, dv_off, 8, p.ext.dv))
     return;
   auto cvt = [&](const float* src, void* dst) {
-    const float4 x = reinterpret_cast<const float4*>(src)[0], y = reinterpret_cast<const float4*>(src)[1];
+    float4 x = reinterpret_cast<const float4*>(src)[0], y = reinterpret_cast<const float4*>(src)[1];
+    for (int s = 1; s < p.split; ++s) {  // the parts in order
+      const float4 u = reinterpret_cast<const float4*>(src + s * slice)[0];
+      const float4 t = reinterpret_cast<const float4*>(src + s * slice)[1];
+      x = make_float4(x.x + u.x, x.y + u.y, x.z + u.z, x.w + u.w);
+      y = make_float4(y.x + t.x, y.y + t.y, y.z + t.z, y.w + t.w);
+    }
     *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w),
                                                 pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
   };
@@ -1118,17 +1125,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const long long dv_off = w.tb * p.sdv.b + w.hk * p.sdv.h + kr * p.sdv.r + col;
         const long long dk_off = w.tb * p.sdk.b + w.hk * p.sdk.h + kr * p.sdk.r + col;
         if (GEN && S > 1) {
-          // one part of a split unit: its dK / dV go into the fp32 accumulators
-          // ([tb][H_kv][key rows][D]), converted once every part is done
+          // one part of a split unit: its (scaled) dK / dV go to its own fp32
+          // slice ([part][tb][H_kv][key rows][D]); the conversion sums the
+          // slices in part order, so the result does not depend on timing
           const long long rows_k = p.rows.cu_k == nullptr ? p.rows.nk : p.rows.total_k;
           const long long acc =
-              ((static_cast<long long>(w.tb) * n_kv_heads + w.hk) * rows_k + kr) * D + col;
-          if (row_ok && col < p.d_real && any_work && n_it > 0 &&
-              FA_IN_BOUNDS(p.status, acc, 32, p.ext.kvacc)) {
+              (((static_cast<long long>(part) * p.rows_tb + w.tb) * n_kv_heads + w.hk) * rows_k +
+               kr) * D + col;
+          if (row_ok && col < p.d_real && FA_IN_BOUNDS(p.status, acc, 32, p.ext.kvacc)) {
+            float4* dvp = reinterpret_cast<float4*>(p.ws_dv + acc);
+            float4* dkp = reinterpret_cast<float4*>(p.ws_dk + acc);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              red_add_f32(p.ws_dv + acc + k, __uint_as_float(a[k]) * p.drop_rscale);
-              red_add_f32(p.ws_dk + acc + k, __uint_as_float(bk[k]) * p.scale);
+            for (int k = 0; k < 8; ++k) {
+              const float rs = p.drop_rscale, sc = p.scale;
+              dvp[k] = make_float4(__uint_as_float(a[4 * k]) * rs, __uint_as_float(a[4 * k + 1]) * rs,
+                                   __uint_as_float(a[4 * k + 2]) * rs, __uint_as_float(a[4 * k + 3]) * rs);
+              dkp[k] = make_float4(__uint_as_float(bk[4 * k]) * sc, __uint_as_float(bk[4 * k + 1]) * sc,
+                                   __uint_as_float(bk[4 * k + 2]) * sc,
+                                   __uint_as_float(bk[4 * k + 3]) * sc);
             }
           }
         } else if (row_ok && col < p.d_real && FA_IN_BOUNDS(p.status, dv_off, 32, p.ext.dv) &&

@@ -216,8 +216,9 @@ struct BwdParams {
                               // (b, K / V head, key tile) and walk the group's query heads
   int split;                  // > 1: each unit splits into `split` parts, part p walking
                               // query heads [p, p + 1) * group / split of the group and
-                              // adding its dK / dV into ws_dk / ws_dv (general instances)
-  // fp32 dK / dV accumulators [tb][H_kv][key rows][D] when split > 1
+                              // writing its dK / dV to slice p of ws_dk / ws_dv
+  int rows_tb;                // batch coordinates of the tensors (B padded, 1 packed)
+  // fp32 dK / dV slices [split][rows_tb][H_kv][key rows][D] when split > 1
   float* ws_dk;
   float* ws_dv;
 #ifdef FA_DEBUG_BOUNDS

@@ -41,10 +41,10 @@ def test_status_strings(lib):
     lib.set_gqa_split(1)
     try:
         assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == base
-        lib.set_gqa_split(3)   # three parts of the group of 3: two accumulators of 2 x 384 x 64
-        assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == base + 2 * 4 * 2 * 384 * 64
+        lib.set_gqa_split(3)   # three parts of the group of 3: dK / dV slices of 2 x 384 x 64 each
+        assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == base + 3 * 2 * 4 * 2 * 384 * 64
         lib.set_gqa_split(2)   # does not divide the group: the automatic choice (3 here)
-        assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == base + 2 * 4 * 2 * 384 * 64
+        assert so.fa_bwd_ex_workspace_size(ctypes.byref(a)) == base + 3 * 2 * 4 * 2 * 384 * 64
     finally:
         lib.set_gqa_split(0)
     # the default library is the production build (no bounds checks)
@@ -254,8 +254,8 @@ def test_nvtx_ranges_wrap_the_entry_points(lib, monkeypatch):
 
 def test_gqa_split_is_chosen_from_the_units(lib):
     """Grouped K / V heads: a backward unit is split into the fewest parts
-    (a divisor of the group) giving about four units per SM (592); the split
-    units' dK / dV accumulators show in the workspace size."""
+    (a divisor of the group) giving about four units per SM (592); the parts'
+    dK / dV slices show in the workspace size."""
     so = lib.library()
     N, d = 16384, 128
 
@@ -268,8 +268,8 @@ def test_gqa_split_is_chosen_from_the_units(lib):
     def base(B, H):
         return B * H * N * (8 + 4 * d)
 
-    acc = lambda B, Hkv: 2 * 4 * B * Hkv * N * d  # noqa: E731  two fp32 accumulators
+    acc = lambda S, B, Hkv: S * 2 * 4 * B * Hkv * N * d  # noqa: E731  dK / dV slice per part
     assert ws(1, 16, 16) == base(1, 16)                  # no grouping: no split
-    assert ws(1, 16, 1) == base(1, 16) + acc(1, 1)       # 128 units: split into 8 parts
-    assert ws(1, 16, 4) == base(1, 16) + acc(1, 4)       # 512 units: 2 parts
+    assert ws(1, 16, 1) == base(1, 16) + acc(8, 1, 1)    # 128 units: split into 8 parts
+    assert ws(1, 16, 4) == base(1, 16) + acc(2, 1, 4)    # 512 units: 2 parts
     assert ws(2, 16, 4) == base(2, 16)                   # 1024 units: whole groups

@@ -137,3 +137,23 @@ def test_gqa_backward_split_parts(lib, parity_record, parts, d):
     args = (d ** -0.5, True, None, 0.1, 65)
     rg = attention_backward_gqa(f64(qh), f64(kh), f64(vh), f64(doh), *args)
     check_grads(tuple(f64(x) for x in grads), rg, parity_record)
+
+
+def test_gqa_split_backward_is_repeatable(lib):
+    """Split units write their partial dK / dV to slices summed in a fixed
+    order: two runs give the same dK and dV bits."""
+    import torch
+    B, H, Hkv, N, d = 1, 8, 2, 640, 128
+    q, do = randn((B, H, N, d), 71).cuda(), randn((B, H, N, d), 72).cuda()
+    k, v = randn((B, Hkv, N, d), 73).cuda(), randn((B, Hkv, N, d), 74).cuda()
+    kw = dict(causal=True, dropout_p=0.1, seed=75)
+    lib.set_gqa_split(4)
+    try:
+        o, lse = lib.forward_general(q, k, v, **kw)
+        a = lib.backward_general(q, k, v, o, lse, do, **kw)
+        b = lib.backward_general(q, k, v, o, lse, do, **kw)
+        torch.cuda.synchronize()
+        assert lib.last_device_status() == 0
+    finally:
+        lib.set_gqa_split(0)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
