@@ -64,6 +64,8 @@ HEADLINE = "long128"
 ORDER = ["tiny", "gpt2", "bert", "long64", "long128", "long256", "sparse"]
 UNFUSED_CONFIGS = ("gpt2", "long128")
 FLUSH_BYTES = 256 << 20
+# per_config entries through fa_fwd_ex / fa_bwd_ex: name -> (workload, case class)
+GENERAL_CASES = {"bert_packed": ("bert", "PackedCase"), "long128_gqa4": ("long128", "GqaCase")}
 DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
@@ -84,11 +86,13 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all"] + sorted(WORKLOADS) + sorted(PROJ_SHAPES),
+    ap.add_argument("--workload", choices=["all"] + sorted(WORKLOADS) + sorted(PROJ_SHAPES)
+                    + sorted(GENERAL_CASES),
                     default="all",
                     help="'all' (default): headline plus every workload in per_config; a name: "
                          "that workload alone as the headline (profiling); a qkv_proj_* name: "
-                         "that fused-projection measurement alone")
+                         "that fused-projection measurement alone; bert_packed / long128_gqa4: "
+                         "that general-layout per_config entry alone")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch size (single-workload profiling only)")
     ap.add_argument("--seqlen", type=int, default=None,
@@ -108,7 +112,8 @@ def parse_args(argv=None):
                     help="instead of the bench line: fused vs unfused time and peak memory "
                          "for N = 1K..32K (B=1 H=4 d=128 causal)")
     args = ap.parse_args(argv)
-    if (args.workload == "all" or args.workload in PROJ_SHAPES) and (
+    if (args.workload == "all" or args.workload in PROJ_SHAPES
+            or args.workload in GENERAL_CASES) and (
             args.batch or args.seqlen or args.dropout is not None):
         ap.error("--batch/--seqlen/--dropout need a single attention --workload")
     return args
@@ -760,9 +765,14 @@ def run_ours(args):
 
     if args.unfused_sweep:
         return run_unfused_sweep(args, fa, dev, flush, stream, world, rank)
-    if args.workload in PROJ_SHAPES:
-        r = measure_projection(fa, args.workload, args, rank, dev, flush, stream, world, local,
-                               peak)
+    if args.workload in PROJ_SHAPES or args.workload in GENERAL_CASES:
+        if args.workload in PROJ_SHAPES:
+            r = measure_projection(fa, args.workload, args, rank, dev, flush, stream, world, local,
+                                   peak)
+        else:
+            base, cls = GENERAL_CASES[args.workload]
+            r = measure_packed(fa, WORKLOADS[base], args, rank, dev, flush, stream, world, local,
+                               peak, case_cls=globals()[cls])
         if rank == 0:
             print(json.dumps({"workload": args.workload, **r}), flush=True)
         return 0
